@@ -1,0 +1,44 @@
+"""Mutation check of the oracle's pins: plausible mistakes planted in a copy of the oracle's
+C source (a dropped scale, a wrong GQA head map, a causal off-by-one, a transposed V stride, a
+missing normalisation, a wrong LSE, a wrong mean divisor, a wrong rounding mode) must each be
+caught by at least one pin. The planted copies are built in a temporary directory on the CPU;
+the real oracle is untouched."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = {
+    "dropped_scale": ("s[j] = a->scale * dot;", "s[j] = dot;"),
+    "gqa_modulo_map": ("int64_t g = h / group;", "int64_t g = h % a->hk;"),
+    "causal_off_by_one": ("int64_t last = i + a->sk - a->sq;", "int64_t last = i + a->sk - a->sq - 1;"),
+    "causal_top_left": ("int64_t last = i + a->sk - a->sq;", "int64_t last = i;"),
+    "v_stride_dqk": ("((bi * a->sk + j) * a->hk + g) * a->dv;", "((bi * a->sk + j) * a->hk + g) * a->dqk;"),
+    "no_normalisation": ("o_row[c] /= l;", "o_row[c] /= 1.0;"),
+    "lse_without_max": ("*lse_out = m + log(l);", "*lse_out = log(l);"),
+    "mean_divisor": ("double mean = sum / (double)sk;", "double mean = sum / (double)(sk - 1);"),
+    "round_toward_zero": ("double r = nearbyint(ldexp(ax, -qexp));", "double r = trunc(ldexp(ax, -qexp));"),
+    "max_skips_first": ("double m = s[0];", "double m = 0.0;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not found: {old}"
+    mut_src = tmp_path / "attn_oracle_mutant.c"
+    mut_src.write_text(src.replace(old, new))
+    out = str(tmp_path / f"liboracle_{name}.so")
+    oracle.build(force=True, src=str(mut_src), out=out)
+    lib = oracle.load_library(out)
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib)
+        except (AssertionError, ValueError):
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake {name}"
