@@ -1,0 +1,149 @@
+"""Fused attention forward pass (with per-row log-sum-exp) and the K channel-mean pre-pass on
+B200 (sm_100a), as a thin Python binding over the C ABI of ``libb200attn.so``
+(declared in ``include/b200attn.h``).
+
+The binding only marshals arguments: it checks dtypes/devices/contiguity, allocates outputs
+with ``torch.empty`` and passes raw device pointers plus the current CUDA stream. Every step of
+the computation runs in the library's CUDA kernels; there is no CPU or PyTorch fallback, and
+importing this package fails loudly when the library is missing.
+
+Raw C entry points, with the header's names and argument order, are exposed through ``lib``
+(a ``ctypes.CDLL``): ``lib.attn_fwd``, ``lib.k_smooth_mean``, ``lib.k_smooth_sub``,
+``lib.attn_status_string``, ``lib.attn_debug_status``.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libb200attn.so")
+
+STATUS = {
+    0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_GQA", 4: "ERR_HEADDIM", 5: "ERR_ALIGN",
+    6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
+}
+EXPORTS = ("attn_fwd", "k_smooth_mean", "k_smooth_sub", "attn_status_string",
+           "attn_debug_status")
+
+
+class B200AttnError(RuntimeError):
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)} ({message})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m head_attention_forward_flash_b200.build`"
+            " (or __graft_entry__.build()); there is no fallback implementation")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_int,
+                             ctypes.c_float, vp]
+    lib.attn_fwd.restype = ctypes.c_int
+    lib.k_smooth_mean.argtypes = [vp, vp, i64, i64, i64, i64, vp]
+    lib.k_smooth_mean.restype = ctypes.c_int
+    lib.k_smooth_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.k_smooth_sub.restype = ctypes.c_int
+    lib.attn_status_string.argtypes = [ctypes.c_int]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_debug_status.argtypes = [vp]
+    lib.attn_debug_status.restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise B200AttnError(fn, status, lib.attn_status_string(status).decode())
+
+
+def _stream_ptr(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _want(t, name, dims):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (BSHD)")
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+             return_lse: bool = True):
+    """O = softmax(scale * Q K^T [+ causal mask]) V and the per-row LSE (natural log).
+
+    q [b, sq, hq, dqk], k [b, sk, hk, dqk], v [b, sk, hk, dv]: contiguous bf16 CUDA tensors.
+    Returns ``(out [b, sq, hq, dv] bf16, lse [b, hq, sq] fp32 or None)``.
+    ``scale`` defaults to 1/sqrt(dqk).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _want(t, name, 4)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    b, sq, hq, dqk = q.shape
+    bk, sk, hk, dqk2 = k.shape
+    bv, skv, hkv, dv = v.shape
+    if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
+        raise ValueError("inconsistent q/k/v shapes")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    if out is None:
+        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q.device)
+    st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
+                      1 if causal else 0, float(scale), _stream_ptr(q))
+    _check("attn_fwd", st)
+    return out, lse
+
+
+def k_smooth_mean(k, mean=None):
+    """fp32 channel mean of K over its sequence axis: [b, hk, d]."""
+    import torch
+    _want(k, "k", 4)
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
+    b, sk, hk, d = k.shape
+    if mean is None:
+        mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    _check("k_smooth_mean",
+           lib.k_smooth_mean(k.data_ptr(), mean.data_ptr(), b, hk, sk, d, _stream_ptr(k)))
+    return mean
+
+
+def k_smooth_sub(k, mean, out=None):
+    """bf16(K - mean) with the [b, hk, d] fp32 mean broadcast over the sequence axis."""
+    import torch
+    _want(k, "k", 4)
+    _want(mean, "mean", 3)
+    if k.dtype != torch.bfloat16 or mean.dtype != torch.float32:
+        raise TypeError("k must be bfloat16 and mean float32")
+    b, sk, hk, d = k.shape
+    if tuple(mean.shape) != (b, hk, d):
+        raise ValueError("mean must be [b, hk, d]")
+    if out is None:
+        out = torch.empty_like(k)
+    _check("k_smooth_sub", lib.k_smooth_sub(k.data_ptr(), mean.data_ptr(), out.data_ptr(), b, hk,
+                                            sk, d, _stream_ptr(k)))
+    return out
+
+
+def attn_debug_status(stream=None) -> int:
+    """Synchronise and return/clear the device error word (0 = no kernel gave up a wait)."""
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    return int(lib.attn_debug_status(s))

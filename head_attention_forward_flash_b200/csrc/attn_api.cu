@@ -1,0 +1,238 @@
+// attn_api.cu -- C-ABI entry points attn_fwd, attn_status_string and attn_debug_status:
+// argument checks, TMA descriptor encoding, head-dim dispatch and the kernel launch.
+#include <cmath>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "attn_fwd_kernel.cuh"
+#include "host_common.h"
+
+namespace b200 {
+
+// Device error word written by kernels whose bounded waits give up.
+__device__ int g_attn_status;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+int* status_word()
+{
+    static int* addr[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = static_cast<int*>(p);
+    }
+    return addr[dev];
+}
+
+// 4-D bf16 tensor map over a BSHD tensor [b, s, h, d] (innermost first: d, h, s, b), box
+// {64 channels, 1 head, box_rows rows, 1 batch}, 128-byte swizzle, zero fill out of bounds.
+int encode_bshd(CUtensorMap* map, const void* base, int64_t b, int64_t s, int64_t h, int64_t d,
+                int box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return B200ATTN_ERR_CUDA;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)h, (cuuint64_t)s, (cuuint64_t)b};
+    const cuuint64_t strides[3] = {(cuuint64_t)(d * 2), (cuuint64_t)(h * d * 2),
+                                   (cuuint64_t)(s * h * d * 2)};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+// The TMA unit addresses at most 2^32 elements per dimension and byte strides below 2^40.
+bool tma_extent_ok(int64_t b, int64_t s, int64_t h, int64_t d)
+{
+    const int64_t lim_dim = (int64_t)1 << 31;  // coordinates are signed 32-bit
+    const int64_t lim_stride = (int64_t)1 << 40;
+    if (b >= lim_dim || s >= lim_dim || h >= lim_dim || d >= lim_dim) return false;
+    int64_t st;
+    if (!numel({s, h, d, 2}, &st)) return false;
+    return st < lim_stride;
+}
+
+template <class T, bool CAUSAL>
+int launch_attn(const void* q, const void* k, const void* v, void* out, float* lse, int64_t b,
+                int64_t hq, int64_t hk, int64_t sq, int64_t sk, float scale, cudaStream_t stream)
+{
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    auto kern = attn_fwd_kernel<T, CAUSAL>;
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)T::SMEM_BYTES) != cudaSuccess) {
+            cudaGetLastError();
+            return B200ATTN_ERR_CUDA;
+        }
+        attr_done[dev] = true;
+    }
+    CUtensorMap tk, tv;
+    int rc = encode_bshd(&tk, k, b, sk, hk, T::DQK, T::BN);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, b, sk, hk, T::DV, T::BN);
+    if (rc != B200ATTN_OK) return rc;
+    int* status = status_word();
+    if (!status) return B200ATTN_ERR_CUDA;
+
+    AttnParams p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.o = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.b = b;
+    p.hq = hq;
+    p.hk = hk;
+    p.sq = sq;
+    p.sk = sk;
+    p.group = hq / hk;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    p.n_qtiles = (int)((sq + T::BM - 1) / T::BM);
+    p.status = status;
+    p.timeout_ns = 4000000000ull;  // 4 s: far above any legitimate wait
+
+    dim3 grid((unsigned)(b * hq), (unsigned)p.n_qtiles, 1);
+    kern<<<grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tk, tv, p);
+    if (cudaGetLastError() != cudaSuccess) return B200ATTN_ERR_CUDA;
+    return B200ATTN_OK;
+}
+
+// Head-dim table: (dqk, dv) -> key block width and number of K/V shared-memory slots.
+using T64 = AttnTraits<64, 64, 128, 8>;      // slot 16 KB, 8 slots
+using T128 = AttnTraits<128, 128, 128, 6>;   // slot 32 KB, 6 slots
+using T192 = AttnTraits<192, 128, 128, 4>;   // slot 48 KB (K) / 32 KB used by V, 4 slots
+using T256 = AttnTraits<256, 256, 64, 6>;    // 64-key blocks: slot 32 KB, 6 slots
+
+template <class T>
+int dispatch_causal(int causal, const void* q, const void* k, const void* v, void* out,
+                    float* lse, int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk,
+                    float scale, cudaStream_t st)
+{
+    return causal ? launch_attn<T, true>(q, k, v, out, lse, b, hq, hk, sq, sk, scale, st)
+                  : launch_attn<T, false>(q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+}
+
+// Rows with no key at all (sk == 0): O = 0, LSE = -inf.
+__global__ void fill_empty_rows(__nv_bfloat16* out, int64_t n_out, float* lse, int64_t n_lse)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_out; t += stride)
+        out[t] = __float2bfloat16_rn(0.f);
+    if (lse)
+        for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_lse; t += stride)
+            lse[t] = -INFINITY;
+}
+
+}  // namespace
+}  // namespace b200
+
+using namespace b200;
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk,
+                        int64_t dv, int causal, float scale, void* stream)
+{
+    if (b < 0 || hq < 0 || sq < 0 || sk < 0 || hk <= 0) return B200ATTN_ERR_SHAPE;
+    if (hq % hk != 0) return B200ATTN_ERR_GQA;
+    const bool hd_ok = (dqk == 64 && dv == 64) || (dqk == 128 && dv == 128) ||
+                       (dqk == 192 && dv == 128) || (dqk == 256 && dv == 256);
+    if (!hd_ok) return B200ATTN_ERR_HEADDIM;
+    if (!std::isfinite(scale)) return B200ATTN_ERR_SCALE;
+    int64_t n_q, n_k, n_v, n_o, n_l;
+    if (!numel({b, sq, hq, dqk}, &n_q) || !numel({b, sk, hk, dqk}, &n_k) ||
+        !numel({b, sk, hk, dv}, &n_v) || !numel({b, sq, hq, dv}, &n_o) ||
+        !numel({b, hq, sq}, &n_l) || !numel({n_q, 2}, &n_q) || !numel({n_k, 2}, &n_k) ||
+        !numel({n_v, 2}, &n_v) || !numel({n_o, 2}, &n_o) || !numel({n_l, 4}, &n_l))
+        return B200ATTN_ERR_RANGE;
+    if (n_o == 0) return B200ATTN_OK;  // b, hq or sq is zero: nothing to compute
+    if (!q || !out || (sk > 0 && (!k || !v))) return B200ATTN_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(out, 16) || (k && !aligned(k, 16)) ||
+        (v && !aligned(v, 16)) || (lse && !aligned(lse, 4)))
+        return B200ATTN_ERR_ALIGN;
+    const int64_t n_qtiles = (sq + 127) / 128;
+    if (b * hq > INT32_MAX || n_qtiles > 65535) return B200ATTN_ERR_RANGE;
+    if (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv)))
+        return B200ATTN_ERR_RANGE;
+    int rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (sk == 0) {
+        fill_empty_rows<<<296, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), n_o / 2, lse,
+                                             n_l / 4);
+        return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+    }
+    switch (dqk) {
+    case 64: return dispatch_causal<T64>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    case 128: return dispatch_causal<T128>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    case 192: return dispatch_causal<T192>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    default: return dispatch_causal<T256>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    }
+}
+
+extern "C" const char* attn_status_string(int status)
+{
+    switch (status) {
+    case B200ATTN_OK: return "ok";
+    case B200ATTN_ERR_NULL: return "a required pointer is NULL";
+    case B200ATTN_ERR_SHAPE: return "invalid shape (negative size, or hk <= 0)";
+    case B200ATTN_ERR_GQA: return "hq is not a multiple of hk";
+    case B200ATTN_ERR_HEADDIM:
+        return "unsupported head dims ((dqk,dv) must be (64,64), (128,128), (192,128) or "
+               "(256,256); d for the K mean must be 64, 128 or 256)";
+    case B200ATTN_ERR_ALIGN: return "pointer misaligned (bf16 tensors need 16 bytes, fp32 4)";
+    case B200ATTN_ERR_RANGE: return "size or byte extent out of range";
+    case B200ATTN_ERR_SCALE: return "scale is not finite";
+    case B200ATTN_ERR_ARCH: return "device is not compute capability 10.0 (sm_100)";
+    case B200ATTN_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case B200ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+extern "C" int attn_debug_status(void* stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_attn_status, sizeof v) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_attn_status, &zero, sizeof zero);
+    }
+    return v;
+}

@@ -1,0 +1,54 @@
+// host_common.h -- host-side argument checks shared by the C-ABI entry points.
+// Every check here runs before any CUDA call, so an invalid call launches nothing.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/b200attn.h"
+
+namespace b200 {
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// a * b without signed overflow; false when the product does not fit in int64.
+inline bool mul_ok(int64_t a, int64_t b, int64_t* out)
+{
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / a) return false;
+    *out = a * b;
+    return true;
+}
+
+// Element count of a product of dims; false on overflow.
+inline bool numel(std::initializer_list<int64_t> dims, int64_t* out)
+{
+    int64_t n = 1;
+    for (int64_t d : dims)
+        if (!mul_ok(n, d, &n)) return false;
+    *out = n;
+    return true;
+}
+
+// sm_100 check for the current device (cached per device). Returns a status code.
+inline int check_arch()
+{
+    static int cached[64] = {0};  // 0 unknown, 1 ok, 2 wrong arch
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    if (dev < 64 && cached[dev] != 0) return cached[dev] == 1 ? B200ATTN_OK : B200ATTN_ERR_ARCH;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    const bool ok = (major == 10 && minor == 0);
+    if (dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? B200ATTN_OK : B200ATTN_ERR_ARCH;
+}
+
+}  // namespace b200

@@ -1,0 +1,185 @@
+// kmean.cu -- the K channel-mean pre-pass: k_smooth_mean and k_smooth_sub.
+//
+// K is [b, sk, hk, d] bf16; for a fixed (batch, key position) the hk*d channels of all kv heads
+// are one contiguous row, so the mean over the key axis is a column sum of a [sk, hk*d] matrix
+// per batch: fully coalesced 16-byte loads, one 8-channel group per thread, no shuffles needed.
+// Kernel 1 sums a chunk of key rows per CTA into fp32 partials; kernel 2 folds the partials of
+// each channel in chunk order, so the result is bit-identical from run to run (the two
+// deterministic kernels behind one host call of "[HIP] Mha v4: run the K-smoothing gate as one
+// HIP call", Summary and commit message).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "host_common.h"
+
+namespace b200 {
+namespace {
+
+constexpr int kThreads = 256;      // threads per CTA; each owns 8 consecutive channels
+constexpr int kColsPerCta = kThreads * 8;
+constexpr int kTargetCtas = 4 * 148;  // about four waves of CTAs on the 148 SMs
+constexpr int kMinRowsPerChunk = 16;
+
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& x)
+{
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        acc[2 * t] += __uint_as_float(w[t] << 16);
+        acc[2 * t + 1] += __uint_as_float(w[t] & 0xFFFF0000u);
+    }
+}
+
+// partial[bi][chunk][col] = sum over the chunk's key rows of K[bi, s, col]  (col = g*d + c)
+__global__ void __launch_bounds__(kThreads)
+    k_mean_partial(const uint4* __restrict__ k, float* __restrict__ partial, int64_t sk,
+                   int64_t cols, int64_t rows_per_chunk, int nchunks)
+{
+    const int64_t bi = blockIdx.z;
+    const int chunk = blockIdx.y;
+    const int64_t g8 = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 8-channel group
+    const int64_t c8 = cols / 8;
+    if (g8 >= c8) return;
+    const int64_t s0 = (int64_t)chunk * rows_per_chunk;
+    int64_t s1 = s0 + rows_per_chunk;
+    s1 = s1 < sk ? s1 : sk;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4* src = k + (bi * sk) * c8 + g8;
+    int64_t s = s0;
+    for (; s + 4 <= s1; s += 4) {  // four independent 16-byte loads in flight per thread
+        const uint4 x0 = __ldg(src + (s + 0) * c8);
+        const uint4 x1 = __ldg(src + (s + 1) * c8);
+        const uint4 x2 = __ldg(src + (s + 2) * c8);
+        const uint4 x3 = __ldg(src + (s + 3) * c8);
+        acc_bf16x8(acc, x0);
+        acc_bf16x8(acc, x1);
+        acc_bf16x8(acc, x2);
+        acc_bf16x8(acc, x3);
+    }
+    for (; s < s1; ++s) acc_bf16x8(acc, __ldg(src + s * c8));
+    float4* dst = reinterpret_cast<float4*>(partial + ((bi * nchunks + chunk) * cols) + g8 * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+// mean[bi][col] = (sum over chunks, in chunk order, of partial[bi][chunk][col]) / sk
+__global__ void __launch_bounds__(kThreads)
+    k_mean_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t b,
+                int64_t cols, int nchunks, float sk_f)
+{
+    const int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (t >= b * cols) return;
+    const int64_t bi = t / cols;
+    const int64_t col = t - bi * cols;
+    const float* src = partial + bi * nchunks * cols + col;
+    float sum = 0.f;
+    for (int c = 0; c < nchunks; ++c) sum += src[(int64_t)c * cols];
+    mean[t] = __fdiv_rn(sum, sk_f);
+}
+
+// k_out = bf16_rne(float(K) - mean[bi, col]), 8 channels (16 bytes) per thread per step.
+__global__ void __launch_bounds__(kThreads)
+    k_sub_kernel(const uint4* __restrict__ k, const float* __restrict__ mean,
+                 uint4* __restrict__ k_out, int64_t rows, int64_t sk, int64_t cols)
+{
+    const int64_t c8 = cols / 8;
+    const int64_t n = rows * c8;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x; t < n; t += stride) {
+        const int64_t r = t / c8;            // (bi * sk + s)
+        const int64_t g8 = t - r * c8;
+        const int64_t bi = r / sk;
+        const float4* m = reinterpret_cast<const float4*>(mean + bi * cols + g8 * 8);
+        const float4 m0 = __ldg(m), m1 = __ldg(m + 1);
+        const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+        const uint4 x = __ldg(k + t);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float lo = __fsub_rn(__uint_as_float(w[q] << 16), mv[2 * q]);
+            const float hi = __fsub_rn(__uint_as_float(w[q] & 0xFFFF0000u), mv[2 * q + 1]);
+            __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+            o[q] = *reinterpret_cast<uint32_t*>(&v);
+        }
+        k_out[t] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+int check_kmean_args(const void* k, const void* mean, int64_t b, int64_t hk, int64_t sk,
+                     int64_t d, int64_t* cols_out)
+{
+    if (b < 0 || hk < 0 || sk <= 0) return B200ATTN_ERR_SHAPE;
+    if (!(d == 64 || d == 128 || d == 256)) return B200ATTN_ERR_HEADDIM;
+    int64_t cols, n;
+    if (!numel({hk, d}, &cols) || !numel({b, sk, cols, 2}, &n) || !numel({b, cols, 4}, &n) ||
+        b >= 65536 || sk >= ((int64_t)1 << 40))
+        return B200ATTN_ERR_RANGE;
+    *cols_out = cols;
+    if (b == 0 || hk == 0) return B200ATTN_OK;
+    if (!k || !mean) return B200ATTN_ERR_NULL;
+    if (!aligned(k, 16) || !aligned(mean, 16)) return B200ATTN_ERR_ALIGN;
+    return B200ATTN_OK;
+}
+
+}  // namespace
+}  // namespace b200
+
+using namespace b200;
+
+extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk,
+                             int64_t d, void* stream)
+{
+    int64_t cols = 0;
+    int rc = check_kmean_args(k, mean, b, hk, sk, d, &cols);
+    if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
+    rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const int64_t col_ctas = (cols + kColsPerCta - 1) / kColsPerCta;
+    int64_t nchunks = (kTargetCtas + col_ctas * b - 1) / (col_ctas * b);
+    const int64_t max_chunks = (sk + kMinRowsPerChunk - 1) / kMinRowsPerChunk;
+    if (nchunks > max_chunks) nchunks = max_chunks;
+    if (nchunks > 1024) nchunks = 1024;
+    if (nchunks < 1) nchunks = 1;
+    const int64_t rows_per_chunk = (sk + nchunks - 1) / nchunks;
+    nchunks = (sk + rows_per_chunk - 1) / rows_per_chunk;
+
+    float* partial = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void**>(&partial),
+                        (size_t)(b * nchunks * cols) * sizeof(float), st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    dim3 g1((unsigned)col_ctas, (unsigned)nchunks, (unsigned)b);
+    k_mean_partial<<<g1, kThreads, 0, st>>>(static_cast<const uint4*>(k), partial, sk, cols,
+                                            rows_per_chunk, (int)nchunks);
+    const int64_t n = b * cols;
+    k_mean_fold<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+        partial, mean, b, cols, (int)nchunks, (float)sk);
+    const bool launched = cudaGetLastError() == cudaSuccess;
+    if (cudaFreeAsync(partial, st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    return launched ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+extern "C" int k_smooth_sub(const void* k, const float* mean, void* k_out, int64_t b, int64_t hk,
+                            int64_t sk, int64_t d, void* stream)
+{
+    int64_t cols = 0;
+    int rc = check_kmean_args(k, mean, b, hk, sk, d, &cols);
+    if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
+    if (!k_out) return B200ATTN_ERR_NULL;
+    if (!aligned(k_out, 16)) return B200ATTN_ERR_ALIGN;
+    rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    const int64_t n = b * sk * (cols / 8);
+    int64_t blocks = (n + kThreads - 1) / kThreads;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    k_sub_kernel<<<(unsigned)blocks, kThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4*>(k), mean, static_cast<uint4*>(k_out), b * sk, sk, cols);
+    return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}

@@ -1,0 +1,128 @@
+/*
+ * b200attn.h -- C ABI of the B200 (sm_100a) fused attention forward library (libb200attn.so).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller. The library never frees or
+ *     keeps a caller pointer after the call returns.
+ *   - Tensors are contiguous, BSHD, row-major (last dimension fastest):
+ *       Q [b, sq, hq, dqk], K [b, sk, hk, dqk], V [b, sk, hk, dv], O [b, sq, hq, dv]  (bf16)
+ *       LSE [b, hq, sq] (fp32, natural log), K mean [b, hk, d] (fp32).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
+ *     enqueued asynchronously on it; the call does not synchronise.
+ *   - Return value: B200ATTN_OK (0) on success, otherwise one of the status codes below.
+ *     Argument checks run on the host before any CUDA call; when one fails nothing is launched
+ *     and no output byte is written. attn_status_string() names every code.
+ *   - Sizes are int64_t. Every byte offset the kernels form is 64-bit; extents that the tensor
+ *     memory accelerator (TMA) cannot address are refused with B200ATTN_ERR_RANGE rather than
+ *     truncated (the lesson of "MHA v4: fixes, refactor, new kernel, perf tweaks", the note on
+ *     uint32 kernel-argument strides that truncated silently above 4 GiB).
+ *   - Kernels never read past a tensor's logical end: tile loads past an edge are clipped and
+ *     zero-filled by TMA, and stores are predicated (the same page's notes on speculative
+ *     reads past the logical sequence).
+ */
+#ifndef B200ATTN_H
+#define B200ATTN_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define B200ATTN_API __attribute__((visibility("default")))
+#else
+#define B200ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum b200attn_status {
+    B200ATTN_OK = 0,
+    B200ATTN_ERR_NULL = 1,     /* a required pointer is NULL for a non-empty tensor */
+    B200ATTN_ERR_SHAPE = 2,    /* a size is negative, or hk <= 0 / sk < 0 */
+    B200ATTN_ERR_GQA = 3,      /* hq is not a multiple of hk */
+    B200ATTN_ERR_HEADDIM = 4,  /* (dqk, dv) not in {(64,64),(128,128),(192,128),(256,256)};
+                                  for the K mean, d not in {64, 128, 256} */
+    B200ATTN_ERR_ALIGN = 5,    /* a pointer below its required alignment: 16 bytes for bf16
+                                  tensors and the K mean, 4 bytes for LSE */
+    B200ATTN_ERR_RANGE = 6,    /* a size, byte extent or stride overflows int64 or TMA limits */
+    B200ATTN_ERR_SCALE = 7,    /* scale is NaN or infinite */
+    B200ATTN_ERR_ARCH = 8,     /* the current device is not compute capability 10.0 (sm_100) */
+    B200ATTN_ERR_CUDA = 9,     /* a CUDA runtime / driver call or a kernel launch failed */
+    B200ATTN_ERR_TIMEOUT = 10, /* a kernel gave up on a bounded wait (see attn_debug_status) */
+};
+
+/*
+ * attn_fwd -- fused attention forward pass with per-row log-sum-exp.
+ *
+ * Computes, for every batch bi < b, query head h < hq, query row i < sq, with kv head
+ * g = h / (hq / hk) (consecutive query heads share a kv head; grouped-query attention):
+ *     J = { j < sk : causal == 0  or  j <= i + sk - sq }       (bottom-right causal alignment)
+ *     s_j = scale * <Q[bi,i,h,:], K[bi,j,g,:]>
+ *     O[bi,i,h,:] = sum_{j in J} softmax_J(s)_j * V[bi,j,g,:]        (rounded to bf16, RNE)
+ *     LSE[bi,h,i] = log(sum_{j in J} exp(s_j))                       (fp32, natural log)
+ * A row with an empty J (causal with i < sq - sk) gets O = 0 and LSE = -inf.
+ * This is the multi-head attention forward pass that the Triton "_attn_fwd" kernel of
+ * "Tune MHA config & small-head pipeline pathology" computes (Motivation; shape notation
+ * M = sq, N = sk, K = d_head_qk, d_v, HQ/HK and causal c0/c1 in "Source of shapes" and the
+ * tables after Final status); the pages do not write the formula, and this is its standard
+ * reading.
+ *
+ *   q, k, v  device bf16, 16-byte aligned, shapes as above. Read only.
+ *   out      device bf16 [b, sq, hq, dv], 16-byte aligned. Fully written.
+ *   lse      device fp32 [b, hq, sq], 4-byte aligned, or NULL to skip the LSE.
+ *   b, hq, sq  may be 0 (nothing is launched). sk may be 0 (every row is empty).
+ *   hk       > 0, hq % hk == 0.
+ *   dqk, dv  one of (64,64), (128,128), (192,128), (256,256).
+ *   causal   0 or nonzero.
+ *   scale    finite; usually 1/sqrt(dqk).
+ * Allocates nothing. Safe to call concurrently on different streams.
+ */
+B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+             int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+             int causal, float scale, void* stream);
+
+/*
+ * k_smooth_mean -- fp32 channel mean of K over its sequence axis.
+ *     mean[bi,g,c] = (1/sk) * sum_{s < sk} K[bi,s,g,c]
+ * The per-(batch, head) moments of K over its key axis, folded per head in a fixed order, that
+ * "[HIP] Mha v4: run the K-smoothing gate as one HIP call" computes in two deterministic kernels
+ * behind one host call (Summary; commit message). Here the sample is every key and no gate is
+ * applied. Sums run in fp32 over sequence chunks, then the chunk partials are folded in a fixed
+ * order, so repeated calls give bit-identical results.
+ *
+ *   k     device bf16 [b, sk, hk, d], 16-byte aligned.
+ *   mean  device fp32 [b, hk, d], 16-byte aligned. Fully written.
+ *   d     64, 128 or 256 (the head dims the page's host check accepts). sk > 0.
+ * Takes its partial-sum scratch from cudaMallocAsync on `stream` and frees it on the same
+ * stream, so concurrent calls on different streams do not share scratch.
+ */
+B200ATTN_API int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk, int64_t d,
+                  void* stream);
+
+/*
+ * k_smooth_sub -- subtract the channel mean from K: k_out = bf16_rne(float(K) - mean),
+ * with mean[bi,g,c] broadcast over the sequence axis. This makes the smoothed K that the
+ * attention pass then reads ("mean subtracted before attention"). k_out must not overlap k.
+ *
+ *   k, k_out  device bf16 [b, sk, hk, d], 16-byte aligned.   mean  device fp32 [b, hk, d],
+ *             16-byte aligned.
+ * Allocates nothing.
+ */
+B200ATTN_API int k_smooth_sub(const void* k, const float* mean, void* k_out, int64_t b, int64_t hk,
+                 int64_t sk, int64_t d, void* stream);
+
+/* Static description of a status code (never NULL). */
+B200ATTN_API const char* attn_status_string(int status);
+
+/*
+ * attn_debug_status -- synchronise `stream`, then return and clear the device-side error word
+ * that kernels set when a bounded wait gives up (B200ATTN_ERR_TIMEOUT) instead of hanging.
+ * Returns B200ATTN_OK when no kernel has reported an error since the last call on this device.
+ */
+B200ATTN_API int attn_debug_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* B200ATTN_H */

@@ -1,0 +1,73 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every function the header
+declares, and refuses invalid arguments with the documented status before any CUDA call."""
+import ctypes
+
+import pytest
+
+from libutil import ensure_built, header_functions
+
+ensure_built()
+import head_attention_forward_flash_b200 as b2  # noqa: E402
+
+A = 0x10000  # a fake, 16-byte aligned, never-dereferenced address (checks fail before any use)
+
+
+def test_exports_every_header_function():
+    names = header_functions()
+    assert set(names) == set(b2.EXPORTS), names
+    raw = ctypes.CDLL(b2.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} not exported"
+
+
+def test_status_strings():
+    for code in range(0, 11):
+        s = b2.lib.attn_status_string(code)
+        assert s and s.decode() != "unknown status"
+    assert b2.lib.attn_status_string(99).decode() == "unknown status"
+
+
+def call(q=A, k=A, v=A, o=A, lse=A, b=1, hq=2, hk=1, sq=16, sk=16, dqk=64, dv=64, causal=0,
+         scale=0.125):
+    return b2.lib.attn_fwd(q, k, v, o, lse, b, hq, hk, sq, sk, dqk, dv, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b=-1), 2), (dict(sq=-3), 2), (dict(sk=-1), 2), (dict(hk=0), 2), (dict(hq=-2), 2),
+    (dict(hq=3, hk=2), 3), (dict(hq=6, hk=4), 3),
+    (dict(dqk=96, dv=96), 4), (dict(dqk=128, dv=64), 4), (dict(dqk=192, dv=192), 4),
+    (dict(dqk=32, dv=32), 4),
+    (dict(scale=float("nan")), 7), (dict(scale=float("inf")), 7),
+    (dict(q=None), 1), (dict(o=None), 1), (dict(k=None), 1), (dict(v=None), 1),
+    (dict(q=A + 8), 5), (dict(k=A + 2), 5), (dict(o=A + 4), 5), (dict(lse=A + 2), 5),
+    (dict(b=1 << 40, hq=1 << 40, hk=1), 6), (dict(sq=128 * 65536), 6),
+    (dict(sk=1 << 33, b=1, hk=1), 6),
+])
+def test_attn_fwd_rejects(kw, code):
+    assert call(**kw) == code
+
+
+def test_empty_problem_is_a_no_op():
+    # b, hq or sq == 0: nothing to compute, no pointer is touched, no CUDA call is made.
+    assert call(b=0, q=None, k=None, v=None, o=None, lse=None) == 0
+    assert call(sq=0, q=None, o=None, lse=None) == 0
+    assert call(hq=0, hk=1, q=None, o=None, lse=None) == 0
+
+
+@pytest.mark.parametrize("fn", ["k_smooth_mean", "k_smooth_sub"])
+def test_k_mean_rejects(fn):
+    f = getattr(b2.lib, fn)
+
+    def c(k=A, m=A, b=1, hk=2, sk=8, d=64):
+        if fn == "k_smooth_mean":
+            return f(k, m, b, hk, sk, d, None)
+        return f(k, m, A, b, hk, sk, d, None)
+
+    assert c(d=96) == 4 and c(d=192) == 4
+    assert c(sk=0) == 2 and c(b=-1) == 2 and c(hk=-1) == 2
+    assert c(k=None) == 1 and c(m=None) == 1
+    assert c(k=A + 8) == 5 and c(m=A + 4) == 5
+    assert c(b=0) == 0 and c(hk=0) == 0
+    if fn == "k_smooth_sub":
+        assert f(A, A, None, 1, 2, 8, 64, None) == 1
+        assert f(A, A, A + 2, 1, 2, 8, 64, None) == 5
