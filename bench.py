@@ -1,0 +1,415 @@
+"""Benchmark of the fused attention forward pass on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl reference]
+
+One step = one pass of the hot path over one batch of synthetic input: attn_fwd (plus, for the
+K-mean workload, k_smooth_mean and k_smooth_sub before it). Inputs are seeded N(0,1) bf16 tensors
+of the workload's shape, resident in HBM before timing starts. Each step is timed with CUDA
+events on the launching stream; the L2 cache is flushed (a 256 MiB write) before every step,
+outside the events. Under torchrun every rank runs its own independent batch (weak scaling, no
+data-path collective); the reported time is the max over ranks.
+
+Prints ONE JSON line on rank 0. The metric is attention-forward TFLOP/s with
+FLOPs = 2*b*hq*sq*sk*(dqk+dv), halved for causal, also given as a fraction of B200 dense BF16
+peak (2250 TFLOP/s datasheet) and of the measured cuBLAS bf16 figure.
+
+--impl reference times the CPU oracle (oracle/, plain fp64 C) on the host cores instead, on a
+bounded sample of the same workload's rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU work budget of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------------------------
+def _row_flops(c, rows):
+    """Algorithmic FLOPs of the given output rows: 2 * |allowed keys| * (dqk + dv) each."""
+    total = 0
+    for (_, _, i) in rows:
+        n = min(c["sk"], int(i) + c["sk"] - c["sq"] + 1) if c["causal"] else c["sk"]
+        total += 2 * max(n, 0) * (c["dqk"] + c["dv"])
+    return float(total)
+
+
+class OracleSampler:
+    """Times the CPU oracle on seeded row samples of workload c (inputs drawn once)."""
+
+    def __init__(self, c, inputs=None):
+        import oracle
+        self.oracle = oracle
+        self.c = c
+        q, k, v = inputs if inputs is not None else workloads.config_inputs(c)
+        if c["kmean"]:
+            _, m32 = oracle.k_mean(workloads.bf16_bits(k), c["b"], c["hk"], c["sk"], c["dqk"])
+            self.kb = oracle.k_sub(workloads.bf16_bits(k), m32, c["b"], c["hk"], c["sk"], c["dqk"])
+        else:
+            self.kb = workloads.bf16_bits(k)
+        self.qb, self.vb = workloads.bf16_bits(q), workloads.bf16_bits(v)
+        self.threads = oracle.default_threads()
+        import numpy as np
+        self.np = np
+        all_rows = workloads.sample_rows(c, n_pos=min(c["sq"], 4096)).numpy()
+        rng = np.random.default_rng(3000 + c["id"])
+        self.rows = all_rows[rng.permutation(len(all_rows))]
+        self.cursor = 0
+
+    def run(self, n_rows):
+        np = self.np
+        idx = np.arange(self.cursor, self.cursor + n_rows) % len(self.rows)
+        self.cursor += n_rows
+        rows = self.rows[idx]
+        c = self.c
+        t0 = time.perf_counter()
+        self.oracle.attn_rows(self.qb, self.kb, self.vb, c["b"], c["hq"], c["hk"], c["sq"],
+                              c["sk"], c["dqk"], c["dv"], c["causal"], c["scale"], rows,
+                              nthreads=self.threads)
+        return time.perf_counter() - t0, _row_flops(c, rows), len(rows)
+
+    def rows_for(self, seconds):
+        """Rows that take about `seconds` of oracle time (calibrated on a small sample)."""
+        n = max(self.threads, 8)
+        dt, _, _ = self.run(n)
+        while dt < 0.5 and n < len(self.rows) * 64:
+            n *= 4
+            dt, _, _ = self.run(n)
+        return max(1, int(n * seconds / max(dt, 1e-6)))
+
+
+def cpu_baseline(c, inputs, seconds):
+    s = OracleSampler(c, inputs)
+    n = s.rows_for(seconds)
+    dt, fl, nr = s.run(n)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle",
+            "sample": f"{nr} seeded output rows (all heads/batches, {c['workload']}), "
+                      f"{fl / 1e9:.2f} GFLOP in {dt:.1f} s, fp64 plain C oracle"}
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"b200attn_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sms.append(sm)
+            maxes.append(mx)
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sms:
+            return None
+        load = [s for s in sms if s > 0.5 * max(sms)] or sms
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(maxes),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    import head_attention_forward_flash_b200 as b2
+
+    c = workloads.config(args.config)
+    c_rank = dict(c)
+    c_rank["seed"] = c["seed"] + 7919 * rank  # every rank its own independent batch
+    q_h, k_h, v_h = workloads.config_inputs(c_rank)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty((c["b"], c["sq"], c["hq"], c["dv"]), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((c["b"], c["hq"], c["sq"]), dtype=torch.float32, device=dev)
+    mean = torch.empty((c["b"], c["hk"], c["dqk"]), dtype=torch.float32, device=dev)
+    k_s = torch.empty_like(k) if c["kmean"] else None
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 4 if c["kmean"] else 1
+
+    def step():
+        kk = k
+        if c["kmean"]:
+            b2.k_smooth_mean(k, mean)
+            b2.k_smooth_sub(k, mean, k_s)
+            kk = k_s
+        ev_a0.record(stream)
+        b2.attn_fwd(q, kk, v, causal=c["causal"], scale=c["scale"], out=o, lse=lse)
+        ev_a1.record(stream)
+
+    ev_a0 = torch.cuda.Event(enable_timing=True)
+    ev_a1 = torch.cuda.Event(enable_timing=True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if b2.attn_debug_status() != 0:
+        raise RuntimeError("a kernel reported a bounded-wait timeout during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    a_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    a_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    barrier()
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.start()
+        time.sleep(0.4)
+    for s in range(args.steps):
+        flush.zero_()
+        starts[s].record(stream)
+        ev_a0, ev_a1 = a_starts[s], a_ends[s]
+        step()
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop() if clocks else None
+    step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
+    attn_ms = [a_starts[s].elapsed_time(a_ends[s]) for s in range(args.steps)]
+    status = b2.attn_debug_status()
+    if status != 0:
+        raise RuntimeError(f"a kernel reported status {status} in the timed region")
+
+    ms_local = sum(step_ms) / len(step_ms)
+    ms = max_over_ranks(ms_local)
+    fl = workloads.flops(c)
+    value = world * fl / (ms * 1e-3) / 1e12
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    achieved = fl / (attn_avg_ms * 1e-3) / 1e12
+    peaks, peak_src = measured_peaks()
+    peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    traffic = None
+    try:
+        with open(PROFILED_TRAFFIC_FILE) as f:
+            traffic = json.load(f).get(c["workload"])
+    except (OSError, ValueError):
+        traffic = None
+    srt = sorted(attn_ms)
+    lo, hi = int(0.1 * len(srt)), max(int(0.9 * len(srt)), int(0.1 * len(srt)) + 1)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timing
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        op = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        lp = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        e_steps = max(3, min(args.steps, 10))
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps + 1)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps + 1)]
+
+        def e2e_step():
+            qd = qp.to(dev, non_blocking=True)
+            kd = kp.to(dev, non_blocking=True)
+            vd = vp.to(dev, non_blocking=True)
+            if c["kmean"]:
+                kd = b2.k_smooth_sub(kd, b2.k_smooth_mean(kd))
+            od, ld = b2.attn_fwd(qd, kd, vd, causal=c["causal"], scale=c["scale"])
+            op.copy_(od, non_blocking=True)
+            lp.copy_(ld, non_blocking=True)
+
+        for s in range(e_steps + 1):  # first one is a warm-up
+            flush.zero_()
+            ev0[s].record(stream)
+            e2e_step()
+            ev1[s].record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(sum(ev0[s].elapsed_time(ev1[s]) for s in range(1, e_steps + 1))
+                              / e_steps)
+        h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+        d2h = o.numel() * 2 + lse.numel() * 4
+        e2e = {"value": world * fl / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(c, (q_h, k_h, v_h), args.cpu_seconds)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": "attention fwd TFLOP/s (causal-halved) and % of B200 dense BF16 peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "pct_of_dense_bf16_peak": {"value": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
+                                   "peak_tflops": DATASHEET_BF16_TFLOPS,
+                                   "peak_source": "B200 datasheet dense BF16"},
+        "pct_of_measured_bf16": {"burst": 100.0 * value / world / peak,
+                                 "sustained": 100.0 * value / world /
+                                 peaks.get("bf16_tflops_sustained", FALLBACK[
+                                     "bf16_tflops_sustained"]),
+                                 "source": peak_src},
+        "config": {"workload": c["workload"], "b": c["b"], "hq": c["hq"], "hk": c["hk"],
+                   "sq": c["sq"], "sk": c["sk"], "dqk": c["dqk"], "dv": c["dv"],
+                   "causal": c["causal"], "kmean_prepass": c["kmean"], "scale": c["scale"],
+                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": f"attn_fwd_kernel d{c['dqk']}x{c['dv']}",
+                     "peak_source": f"{peak_src} cuBLAS bf16 burst (kernel timed alone)"},
+        "dispatch_us": {"median": 1e3 * statistics.median(attn_ms),
+                        "trimmed_mean_80": 1e3 * sum(srt[lo:hi]) / max(1, hi - lo),
+                        "max": 1e3 * max(attn_ms), "min": 1e3 * min(attn_ms)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on the host cores
+# ---------------------------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return  # the oracle arm runs on rank 0 only
+    c = workloads.config(args.config)
+    s = OracleSampler(c)
+    per_step = max(0.5, min(8.0, 90.0 / max(1, args.steps + args.warmup)))
+    n = s.rows_for(per_step)
+    for _ in range(args.warmup):
+        s.run(n)
+    times, fls = [], []
+    for _ in range(args.steps):
+        dt, fl, _ = s.run(n)
+        times.append(dt)
+        fls.append(fl)
+    value = sum(fls) / sum(times) / 1e12
+    ms = 1e3 * sum(times) / len(times)
+    sample = (f"{n} seeded output rows per step of {c['workload']} (all heads/batches), "
+              f"fp64 plain C oracle")
+    line = {
+        "impl": "reference",
+        "metric": "attention fwd TFLOP/s (causal-halved) and % of B200 dense BF16 peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": c["workload"], "b": c["b"], "hq": c["hq"], "hk": c["hk"],
+                   "sq": c["sq"], "sk": c["sk"], "dqk": c["dqk"], "dv": c["dv"],
+                   "causal": c["causal"], "kmean_prepass": c["kmean"],
+                   "sample": "bounded row sample per step"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
