@@ -79,6 +79,22 @@ bool tma_extent_ok(int64_t b, int64_t s, int64_t h, int64_t d)
     return st < lim_stride;
 }
 
+int sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <class T, bool CAUSAL>
 int launch_attn(const void* q, const void* k, const void* v, void* out, float* lse, int64_t b,
                 int64_t hq, int64_t hk, int64_t sq, int64_t sk, float scale, cudaStream_t stream)
@@ -98,15 +114,16 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
         }
         attr_done[dev] = true;
     }
-    CUtensorMap tk, tv;
-    int rc = encode_bshd(&tk, k, b, sk, hk, T::DQK, T::BN);
+    CUtensorMap tq, tk, tv;
+    int rc = encode_bshd(&tq, q, b, sq, hq, T::DQK, T::BM);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, b, sk, hk, T::DQK, T::BN);
     if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, b, sk, hk, T::DV, T::BN);
     if (rc != B200ATTN_OK) return rc;
     int* status = status_word();
-    if (!status) return B200ATTN_ERR_CUDA;
+    const int n_sm = sm_count();
+    if (!status || n_sm <= 0) return B200ATTN_ERR_CUDA;
 
     AttnParams p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
     p.o = static_cast<__nv_bfloat16*>(out);
     p.lse = lse;
     p.b = b;
@@ -115,22 +132,26 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.sq = sq;
     p.sk = sk;
     p.group = hq / hk;
-    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    p.n_qtiles = (int)((sq + T::BM - 1) / T::BM);
+    p.n_qtiles = (sq + T::BM - 1) / T::BM;
+    p.n_tiles = b * hq * p.n_qtiles;
+    // The MMA applies the sign of the scale (negate-A bit of the instruction descriptor), so
+    // the softmax only ever sees a non-negative scale.
+    p.scale_log2 = (float)(std::fabs((double)scale) * 1.4426950408889634);
+    p.idesc_qk = T::IDESC_QK | (scale < 0.f ? (1u << 13) : 0u);
     p.status = status;
     p.timeout_ns = 4000000000ull;  // 4 s: far above any legitimate wait
 
-    dim3 grid((unsigned)(b * hq), (unsigned)p.n_qtiles, 1);
-    kern<<<grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tk, tv, p);
+    const int64_t grid = p.n_tiles < n_sm ? p.n_tiles : n_sm;  // persistent: one CTA per SM
+    kern<<<(unsigned)grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return B200ATTN_ERR_CUDA;
     return B200ATTN_OK;
 }
 
 // Head-dim table: (dqk, dv) -> key block width and number of K/V shared-memory slots.
-using T64 = AttnTraits<64, 64, 128, 8>;      // slot 16 KB, 8 slots
-using T128 = AttnTraits<128, 128, 128, 6>;   // slot 32 KB, 6 slots
-using T192 = AttnTraits<192, 128, 128, 4>;   // slot 48 KB (K) / 32 KB used by V, 4 slots
-using T256 = AttnTraits<256, 256, 64, 6>;    // 64-key blocks: slot 32 KB, 6 slots
+using T64 = AttnTraits<64, 64, 128, 8>;     // Q 16 KB + 8 slots of 16 KB
+using T128 = AttnTraits<128, 128, 128, 5>;  // Q 32 KB + 5 slots of 32 KB
+using T192 = AttnTraits<192, 128, 128, 3>;  // Q 48 KB + 3 slots of 48 KB (V uses 32 KB)
+using T256 = AttnTraits<256, 256, 64, 4>;   // 64-key blocks: Q 64 KB + 4 slots of 32 KB
 
 template <class T>
 int dispatch_causal(int causal, const void* q, const void* k, const void* v, void* out,
@@ -178,9 +199,8 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* out, 
     if (!aligned(q, 16) || !aligned(out, 16) || (k && !aligned(k, 16)) ||
         (v && !aligned(v, 16)) || (lse && !aligned(lse, 4)))
         return B200ATTN_ERR_ALIGN;
-    const int64_t n_qtiles = (sq + 127) / 128;
-    if (b * hq > INT32_MAX || n_qtiles > 65535) return B200ATTN_ERR_RANGE;
-    if (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv)))
+    if (!tma_extent_ok(b, sq, hq, dqk) ||
+        (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv))))
         return B200ATTN_ERR_RANGE;
     int rc = check_arch();
     if (rc != B200ATTN_OK) return rc;

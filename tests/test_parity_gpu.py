@@ -74,6 +74,19 @@ def test_small_shapes_match_oracle(b2, case):
                seed=hash(case) % 100000)
 
 
+# More work tiles than SMs, so each persistent CTA walks several tiles (and, with sq > sk, a mix
+# of tiles with and without keys).
+MULTI = [(1, 40, 8, 1000, 1000, dqk, dv, causal) for (dqk, dv) in HEAD_DIMS for causal in (True, False)]
+MULTI += [(1, 64, 4, 1000, 200, 128, 128, True), (2, 24, 24, 700, 900, 64, 64, True)]
+
+
+@pytest.mark.parametrize("case", MULTI, ids=lambda c: "b{}_hq{}_hk{}_sq{}_sk{}_d{}x{}_c{}".format(*c))
+def test_many_tiles_per_cta_match_oracle(b2, case):
+    b, hq, hk, sq, sk, dqk, dv, causal = case
+    check_full(b2, b, hq, hk, sq, sk, dqk, dv, causal, 1.0 / math.sqrt(dqk),
+               seed=hash(case) % 100000)
+
+
 @pytest.mark.parametrize("scale", [0.0, -0.08, 0.5])
 def test_unusual_scales(b2, scale):
     check_full(b2, 1, 2, 1, 200, 200, 128, 128, True, scale, seed=31)
