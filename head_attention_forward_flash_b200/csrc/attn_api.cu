@@ -132,8 +132,8 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.sq = sq;
     p.sk = sk;
     p.group = hq / hk;
-    p.n_qtiles = (sq + T::BM - 1) / T::BM;
-    p.n_tiles = b * hq * p.n_qtiles;
+    p.n_qu = (sq + T::NT * T::BM - 1) / (T::NT * T::BM);
+    p.n_units = b * hq * p.n_qu;
     // The MMA applies the sign of the scale (negate-A bit of the instruction descriptor), so
     // the softmax only ever sees a non-negative scale.
     p.scale_log2 = (float)(std::fabs((double)scale) * 1.4426950408889634);
@@ -141,17 +141,19 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.status = status;
     p.timeout_ns = 4000000000ull;  // 4 s: far above any legitimate wait
 
-    const int64_t grid = p.n_tiles < n_sm ? p.n_tiles : n_sm;  // persistent: one CTA per SM
+    const int64_t grid = p.n_units < n_sm ? p.n_units : n_sm;  // persistent: one CTA per SM
     kern<<<(unsigned)grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     if (cudaGetLastError() != cudaSuccess) return B200ATTN_ERR_CUDA;
     return B200ATTN_OK;
 }
 
-// Head-dim table: (dqk, dv) -> key block width and number of K/V shared-memory slots.
-using T64 = AttnTraits<64, 64, 128, 8>;     // Q 16 KB + 8 slots of 16 KB
-using T128 = AttnTraits<128, 128, 128, 5>;  // Q 32 KB + 5 slots of 32 KB
-using T192 = AttnTraits<192, 128, 128, 3>;  // Q 48 KB + 3 slots of 48 KB (V uses 32 KB)
-using T256 = AttnTraits<256, 256, 64, 4>;   // 64-key blocks: Q 64 KB + 4 slots of 32 KB
+// Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, Q in TMEM,
+// K slots, V slots>. Tensor memory holds two score buffers, one O per query tile and (when it
+// fits) each tile's Q; shared memory holds the Q staging buffer and the K / V rings.
+using T64 = AttnTraits<64, 64, 128, 2, true, 5, 5>;       // smem 32 + 80 + 80 KB
+using T128 = AttnTraits<128, 128, 128, 2, false, 3, 2>;   // smem 64 + 96 + 64 KB
+using T192 = AttnTraits<192, 128, 128, 2, false, 2, 1>;   // smem 96 + 96 + 32 KB
+using T256 = AttnTraits<256, 256, 64, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
 template <class T>
 int dispatch_causal(int causal, const void* q, const void* k, const void* v, void* out,

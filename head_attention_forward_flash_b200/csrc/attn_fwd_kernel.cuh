@@ -5,27 +5,36 @@
 // forward of "Tune MHA config & small-head pipeline pathology" (Motivation; shapes in "Source of
 // shapes"), re-designed for the 5th-generation tensor core.
 //
-// Persistent kernel: one CTA per SM walks a list of work tiles (one 128-row query tile of one
-// (batch, query head)), ordered so that the tiles that see the most keys (causal) come first.
-// The pipeline does not drain between tiles.
+// Work unit: NT consecutive 128-row query tiles (NT = 2, or 1 for d256) of one (batch, query
+// head). Every K/V tile brought into shared memory serves all NT query tiles, which halves the
+// L2 -> SM traffic per FLOP and doubles the time each K/V slot can hide load latency. Persistent
+// kernel: one CTA per SM walks its units head-major (CTAs working at the same time share K/V
+// in L2), the units that see the most keys (causal) first within a head. The pipeline does not
+// drain between units.
 //
-// Roles (192 threads; at most two warps per SM sub-partition, so a softmax thread can keep its
-// whole score row in registers):
-//   warps 0-3  softmax + epilogue: thread t owns query row t (= TMEM lane t). Copies its Q row
-//              from the shared-memory staging buffer into TMEM, turns each score block S into P
-//              (online softmax: exp2 with the scale folded into one FMA, lazy rescaling of O),
-//              and writes the finished O row (divided by the row sum) and LSE. A tile's epilogue
-//              runs right after the next tile's first P is handed over, so the wait for the last
-//              P V of the tile overlaps useful work.
-//   warp 4     MMA issuer (one thread): S = Q K^T and O += P V, A operand from TMEM (Q, then P),
-//              B operand from shared memory (K, V), fp32 accumulators in TMEM.
-//   warp 5     TMA producer (one thread): the next tile's Q into the staging buffer, and K, V
-//              tiles through a ring of shared-memory slots in the MMA warp's order
-//              (K0, K1, V0, K2, V1, ...).
+// Items: the pipeline steps through "items" (key block j, query tile t) in the order
+// (0,0) (0,1) (1,0) (1,1) ... for NT = 2, or (0) (1) (2) ... for NT = 1. Item g uses score buffer
+// g % 2, so one item's Q K^T runs on the tensor core while the previous item's softmax runs.
 //
-// Tensor memory (128 lanes x 512 columns of 32 bit): S0 | S1 (two BN-wide score buffers, so one
-// block's Q K^T overlaps the previous block's softmax; P in bf16 pairs overwrites the first BN/2
-// columns of its own S buffer) | O (DV fp32 columns) | Q (DQK/2 columns of bf16 pairs).
+// Roles (NT softmax warpgroups + 2 warps: 320 threads for NT = 2, 192 for NT = 1):
+//   warps 4t..4t+3  softmax + epilogue of query tile t: thread r owns row r of tile t (= TMEM
+//              lane r). Turns each score block S into P (online softmax: exp2 with the scale
+//              folded into one FMA, lazy rescaling of O), and writes the finished O rows (divided
+//              by the row sums) and LSE; a unit's epilogue runs right after the next unit's
+//              first P of the tile is handed over. When Q lives in TMEM, each warpgroup also
+//              copies its tile's Q from the shared-memory staging buffer into TMEM. With two
+//              warpgroups the two tiles' softmax run side by side (two warps per SM
+//              sub-partition); each thread then reads its score row from TMEM twice (max, then
+//              exp) in 32-column chunks, so that its registers stay within the 10-warp budget.
+//   warp 4*NT  MMA issuer (one thread): S = Q K^T and O += P V. A operand: Q from TMEM or shared
+//              memory, then P from TMEM; B operand: K, V from shared memory; fp32 accumulators
+//              in TMEM.
+//   warp 4*NT+1 TMA producer (one thread): each unit's Q into the staging buffer, and K, V tiles
+//              through two rings of shared-memory slots, in the order the MMA warp takes them.
+//
+// Tensor memory (128 lanes x 512 columns of 32 bit): S0 | S1 (BN columns each; P in bf16 pairs
+// overwrites the first BN/2 columns of its own S buffer) | O for each query tile (DV fp32
+// columns each) | Q for each query tile when it lives in TMEM (DQK/2 columns of bf16 pairs).
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets the device error word and a
 // CTA-wide abort flag, every role then leaves its loops, in-flight TMA loads and MMAs are drained
@@ -45,43 +54,50 @@ struct AttnParams {
     __nv_bfloat16* o;
     float* lse;  // may be null
     int64_t b, hq, hk, sq, sk;
-    int64_t group;     // hq / hk
-    int64_t n_qtiles;  // ceil(sq / 128)
-    int64_t n_tiles;   // b * hq * n_qtiles
-    float scale_log2;  // |scale| * log2(e); the sign of scale is applied by the MMA (negate A)
+    int64_t group;    // hq / hk
+    int64_t n_qu;     // query units per (batch, head): ceil(sq / (NT * 128))
+    int64_t n_units;  // b * hq * n_qu
+    float scale_log2; // |scale| * log2(e); the sign of scale is applied by the MMA (negate A)
     uint32_t idesc_qk;
-    int* status;  // device error word
+    int* status;      // device error word
     unsigned long long timeout_ns;
 };
 
-template <int DQK_, int DV_, int BN_, int NSLOT_>
+template <int DQK_, int DV_, int BN_, int NT_, bool Q_TMEM_, int NK_, int NV_>
 struct AttnTraits {
     static constexpr int DQK = DQK_;
     static constexpr int DV = DV_;
-    static constexpr int BN = BN_;  // keys per block
-    static constexpr int BM = 128;  // query rows per tile
-    static constexpr int NSLOT = NSLOT_;
-    static constexpr int QCH = DQK / 64;  // 128-byte (64-element) column chunks of a Q/K row
+    static constexpr int BN = BN_;          // keys per block
+    static constexpr int BM = 128;          // query rows per tile
+    static constexpr int NT = NT_;          // query tiles per unit
+    static constexpr bool Q_TMEM = Q_TMEM_; // Q as the TMEM A operand (else from shared memory)
+    static constexpr int NK = NK_;          // K slots
+    static constexpr int NV = NV_;          // V slots
+    static constexpr int QCH = DQK / 64;    // 128-byte (64-element) column chunks of a Q/K row
     static constexpr int VCH = DV / 64;
     static constexpr uint32_t CHUNK_BYTES = BN * 128;   // one 64-column TMA box of K or V
     static constexpr uint32_t QCHUNK_BYTES = BM * 128;  // one 64-column TMA box of Q
-    static constexpr uint32_t Q_BYTES = BM * DQK * 2;
+    static constexpr uint32_t Q_TILE_BYTES = BM * DQK * 2;
+    static constexpr uint32_t Q_BYTES = NT * Q_TILE_BYTES;
     static constexpr uint32_t K_TILE_BYTES = BN * DQK * 2;
     static constexpr uint32_t V_TILE_BYTES = BN * DV * 2;
-    static constexpr uint32_t SLOT_BYTES = K_TILE_BYTES > V_TILE_BYTES ? K_TILE_BYTES
-                                                                        : V_TILE_BYTES;
-    static constexpr uint32_t S_COL = 0;
-    static constexpr uint32_t O_COL = 2 * BN;
-    static constexpr uint32_t Q_COL = 2 * BN + DV;
+    // tensor memory columns
+    static constexpr uint32_t O_COL0 = 2 * BN;
+    static constexpr uint32_t Q_COL0 = 2 * BN + NT * DV;
     static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(2 * BN + DV + DQK / 2 <= 512, "tensor memory budget");
+    static_assert(2 * BN + NT * DV + (Q_TMEM ? NT * DQK / 2 : 0) <= 512, "tensor memory budget");
     static_assert(DQK % 64 == 0 && DV % 64 == 0 && BN % 64 == 0 && BN <= 256 && DV <= 256, "");
-    // shared memory: [Q staging][K/V slots][barriers][TMEM base, abort flag]
-    static constexpr uint32_t SLOTS_OFF = Q_BYTES;
-    static constexpr uint32_t BARS_OFF = SLOTS_OFF + NSLOT * SLOT_BYTES;
-    static constexpr int NBAR = 2 * NSLOT + 11;
+    static_assert(NT == 1 || NT == 2, "");
+    // shared memory: [Q staging][K slots][V slots][barriers][TMEM base, abort flag]
+    static constexpr uint32_t K_OFF = Q_BYTES;
+    static constexpr uint32_t V_OFF = K_OFF + NK * K_TILE_BYTES;
+    static constexpr uint32_t BARS_OFF = V_OFF + NV * V_TILE_BYTES;
+    static constexpr int NBAR = 2 * NK + 2 * NV + 11;
     static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
-    static constexpr int NUM_THREADS = 192;
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static constexpr int NUM_THREADS = 128 * NT + 64;
+    static constexpr int MMA_WARP = 4 * NT;
+    static constexpr int TMA_WARP = 4 * NT + 1;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BN, false, false);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, DV, false, true);
 };
@@ -100,28 +116,26 @@ __device__ __noinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
     }
 }
 
-// One work tile: (batch, query head, 128-row query tile) and the key blocks it needs.
-struct TileInfo {
+// One work unit: (batch, query head, NT query tiles starting at row q0) and its key blocks.
+struct UnitInfo {
     int64_t bi, h, g, q0;
-    int n_blocks;   // key blocks with at least one allowed key for some row of the tile
+    int n_blocks;   // key blocks with at least one allowed key for some row of the unit
     int mask_from;  // blocks >= mask_from need the per-key mask (causal diagonal, ragged tail)
 };
 
-template <int BN, bool CAUSAL>
-__device__ __forceinline__ TileInfo tile_info(const AttnParams& p, int64_t u)
+template <int BN, int NT, bool CAUSAL>
+__device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
 {
-    TileInfo t;
-    const int64_t bh_count = p.b * p.hq;
-    const int64_t qi = u / bh_count;
-    const int64_t qt = p.n_qtiles - 1 - qi;  // tiles that see the most keys first
-    const int64_t bh = u - qi * bh_count;
+    UnitInfo t;
+    const int64_t bh = u / p.n_qu;
+    const int64_t qu = p.n_qu - 1 - (u - bh * p.n_qu);  // within a head: most keys first
     t.bi = bh / p.hq;
     t.h = bh - t.bi * p.hq;
     t.g = t.h / p.group;
-    t.q0 = qt * 128;
+    t.q0 = qu * (NT * 128);
     const int64_t n_kv = (p.sk + BN - 1) / BN;
     if (CAUSAL) {
-        const int64_t last_row = (t.q0 + 127 < p.sq - 1) ? t.q0 + 127 : p.sq - 1;
+        const int64_t last_row = (t.q0 + NT * 128 - 1 < p.sq - 1) ? t.q0 + NT * 128 - 1 : p.sq - 1;
         const int64_t last_key = last_row + p.sk - p.sq;
         int64_t nb = last_key < 0 ? 0 : last_key / BN + 1;
         nb = nb < n_kv ? nb : n_kv;
@@ -144,58 +158,68 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     const __grid_constant__ CUtensorMap tmap_v, const AttnParams p)
 {
     constexpr int BN = T::BN;
-    constexpr int NSLOT = T::NSLOT;
+    constexpr int NT = T::NT;
+    constexpr int NK = T::NK;
+    constexpr int NV = T::NV;
     constexpr uint32_t FULL = 0xffffffffu;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);  // SW128 needs 1 KB
     const uint32_t sbase = smem_addr(smem);
     const uint32_t q_stage = sbase;
-    const uint32_t slots = sbase + T::SLOTS_OFF;
+    const uint32_t k_slots = sbase + T::K_OFF;
+    const uint32_t v_slots = sbase + T::V_OFF;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BARS_OFF);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + T::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     auto bar = [&](int i) { return smem_addr(&bars[i]); };
-    auto bar_full = [&](int s) { return bar(s); };
-    auto bar_empty = [&](int s) { return bar(NSLOT + s); };
-    auto bar_s_full = [&](int s) { return bar(2 * NSLOT + s); };
-    auto bar_p_full = [&](int s) { return bar(2 * NSLOT + 2 + s); };
-    const uint32_t bar_pv_done = bar(2 * NSLOT + 4);
-    const uint32_t bar_q_full = bar(2 * NSLOT + 5);
-    const uint32_t bar_q_empty = bar(2 * NSLOT + 6);
-    const uint32_t bar_q_tmem = bar(2 * NSLOT + 7);
-    const uint32_t bar_o_full = bar(2 * NSLOT + 8);
-    const uint32_t bar_o_free = bar(2 * NSLOT + 9);
-    const uint32_t bar_mma_done = bar(2 * NSLOT + 10);
+    auto bar_kfull = [&](int s) { return bar(s); };
+    auto bar_kempty = [&](int s) { return bar(NK + s); };
+    auto bar_vfull = [&](int s) { return bar(2 * NK + s); };
+    auto bar_vempty = [&](int s) { return bar(2 * NK + NV + s); };
+    constexpr int B0 = 2 * NK + 2 * NV;
+    auto bar_s_full = [&](int s) { return bar(B0 + s); };
+    auto bar_p_full = [&](int s) { return bar(B0 + 2 + s); };
+    const uint32_t bar_pv_done = bar(B0 + 4);
+    const uint32_t bar_q_full = bar(B0 + 5);
+    const uint32_t bar_q_empty = bar(B0 + 6);
+    const uint32_t bar_q_tmem = bar(B0 + 7);
+    const uint32_t bar_o_full = bar(B0 + 8);
+    const uint32_t bar_o_free = bar(B0 + 9);
+    const uint32_t bar_mma_done = bar(B0 + 10);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NSLOT; ++s) {
-            mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+        for (int s = 0; s < NK; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+        }
+        for (int s = 0; s < NV; ++s) {
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_vempty(s), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_s_full(s), 1);
-            mbar_init(bar_p_full(s), 128);
+            mbar_init(bar_p_full(s), 128);  // one warpgroup writes each P
         }
         mbar_init(bar_pv_done, 1);
         mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_empty, 128);
-        mbar_init(bar_q_tmem, 128);
+        mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : 1);  // softmax copy-out / last Q K^T
+        mbar_init(bar_q_tmem, 128 * NT);
         mbar_init(bar_o_full, 1);
-        mbar_init(bar_o_free, 128);
+        mbar_init(bar_o_free, 128 * NT);
         mbar_init(bar_mma_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 4) {
+    if (warp == T::MMA_WARP) {
         tmem_alloc(smem_addr(tmem_holder), T::TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp == 5 && lane == 0) {
+    if (warp == T::TMA_WARP && lane == 0) {
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
@@ -205,207 +229,246 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_holder;
     const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
-
     const int64_t u0 = blockIdx.x;
     const int64_t ustep = gridDim.x;
 
-    // First tile of this CTA's list (from u) that has at least one key block, or -1.
+    // First unit of this CTA's list (from u) with at least one key block, or -1.
     auto busy_from = [&](int64_t u) -> int64_t {
-        for (; u < p.n_tiles; u += ustep)
-            if (tile_info<BN, CAUSAL>(p, u).n_blocks > 0) return u;
+        for (; u < p.n_units; u += ustep)
+            if (unit_info<BN, NT, CAUSAL>(p, u).n_blocks > 0) return u;
         return -1;
     };
 
-    if (warp >= 4) {
-        if (warp == 5) {
+    if (warp == T::TMA_WARP) {
         // ------------------------------ TMA producer ------------------------------
+        // Walks the MMA warp's item sequence and issues each load at the point the MMA warp
+        // will first need it (K_j at the Q K^T of item (j, 0), V_j at the P V of item (j, 0)).
         if (lane == 0) {
-            int kv_it = 0;  // K/V items issued
-            int q_cnt = 0;  // Q tiles issued
+            int kq = 0, vq = 0;  // K / V items issued
+            int q_cnt = 0;       // Q units issued
             bool ok = true;
             auto load_q = [&](int64_t u) {
-                const TileInfo t = tile_info<BN, CAUSAL>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
                 if (!mbar_wait(bar_q_empty, (uint32_t)(q_cnt & 1) ^ 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
                 mbar_arrive_expect_tx(bar_q_full, T::Q_BYTES);
-                for (int ch = 0; ch < T::QCH; ++ch)
-                    tma_load_4d(q_stage + ch * T::QCHUNK_BYTES, &tmap_q, bar_q_full, ch * 64,
-                                (int)t.h, (int)t.q0, (int)t.bi);
+                for (int tt = 0; tt < NT; ++tt)
+                    for (int ch = 0; ch < T::QCH; ++ch)
+                        tma_load_4d(q_stage + tt * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES, &tmap_q,
+                                    bar_q_full, ch * 64, (int)t.h, (int)(t.q0 + tt * 128),
+                                    (int)t.bi);
                 ++q_cnt;
             };
-            auto load_kv = [&](bool is_k, const TileInfo& t, int j) {
-                const int slot = kv_it % NSLOT;
-                const uint32_t phase = (uint32_t)(kv_it / NSLOT) & 1u;
-                if (!mbar_wait(bar_empty(slot), phase ^ 1u, wc, kErrTimeout)) {
+            auto load_k = [&](const UnitInfo& t, int j) {
+                const int slot = kq % NK;
+                if (!mbar_wait(bar_kempty(slot), (uint32_t)((kq / NK) & 1) ^ 1u, wc,
+                               kErrTimeout)) {
                     ok = false;
                     return;
                 }
-                const uint32_t dst = slots + slot * T::SLOT_BYTES;
-                mbar_arrive_expect_tx(bar_full(slot), is_k ? T::K_TILE_BYTES : T::V_TILE_BYTES);
-                const int nch = is_k ? T::QCH : T::VCH;
-                for (int ch = 0; ch < nch; ++ch)
-                    tma_load_4d(dst + ch * T::CHUNK_BYTES,
-                                is_k ? (const void*)&tmap_k : (const void*)&tmap_v,
-                                bar_full(slot), ch * 64, (int)t.g, j * BN, (int)t.bi);
-                ++kv_it;
+                const uint32_t dst = k_slots + slot * T::K_TILE_BYTES;
+                mbar_arrive_expect_tx(bar_kfull(slot), T::K_TILE_BYTES);
+                for (int ch = 0; ch < T::QCH; ++ch)
+                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_k, bar_kfull(slot), ch * 64,
+                                (int)t.g, j * BN, (int)t.bi);
+                ++kq;
             };
-            // Items go out in the MMA warp's order: K of global block g, then V of block g-1
-            // (also across tiles: a tile's last V follows the next tile's first K).
-            bool pend = false;
-            TileInfo pend_t{};
-            int pend_j = 0;
+            auto load_v = [&](const UnitInfo& t, int j) {
+                const int slot = vq % NV;
+                if (!mbar_wait(bar_vempty(slot), (uint32_t)((vq / NV) & 1) ^ 1u, wc,
+                               kErrTimeout)) {
+                    ok = false;
+                    return;
+                }
+                const uint32_t dst = v_slots + slot * T::V_TILE_BYTES;
+                mbar_arrive_expect_tx(bar_vfull(slot), T::V_TILE_BYTES);
+                for (int ch = 0; ch < T::VCH; ++ch)
+                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_v, bar_vfull(slot), ch * 64,
+                                (int)t.g, j * BN, (int)t.bi);
+                ++vq;
+            };
+            bool pend = false;  // the P V step still owed for the previous item
+            UnitInfo pend_t{};
+            int pend_j = 0, pend_tt = 0;
             int64_t u = busy_from(u0);
             if (u >= 0) load_q(u);
             while (u >= 0 && ok) {
-                const TileInfo t = tile_info<BN, CAUSAL>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
                 const int64_t un = busy_from(u + ustep);
                 for (int j = 0; j < t.n_blocks && ok; ++j) {
-                    load_kv(true, t, j);
-                    if (ok && pend) load_kv(false, pend_t, pend_j);
-                    pend = true;
-                    pend_t = t;
-                    pend_j = j;
-                    // Stage the next tile's Q as soon as this tile's Q has left the buffer.
-                    if (ok && j == 0 && un >= 0) load_q(un);
+                    for (int tt = 0; tt < NT && ok; ++tt) {
+                        if (tt == 0) load_k(t, j);  // the Q K^T step of item (j, tt)
+                        if (ok && T::Q_TMEM && j == 0 && tt == 0 && un >= 0)
+                            load_q(un);  // the staging buffer was emptied into TMEM
+                        if (ok && pend && pend_tt == 0) load_v(pend_t, pend_j);  // P V step
+                        pend = true;
+                        pend_t = t;
+                        pend_j = j;
+                        pend_tt = tt;
+                    }
                 }
+                // With Q read from shared memory, the next unit's Q can only replace this one
+                // after the unit's last Q K^T (the MMA warp commits bar_q_empty then).
+                if (ok && !T::Q_TMEM && un >= 0) load_q(un);
                 u = un;
             }
-            if (ok && pend) load_kv(false, pend_t, pend_j);
+            if (ok && pend && pend_tt == 0) load_v(pend_t, pend_j);
             // Nothing may be in flight when the CTA exits: wait for the last load of each slot
             // and for the last Q load.
-            const int n_drain = kv_it < NSLOT ? kv_it : NSLOT;
-            for (int d = 0; d < n_drain; ++d) {
-                const int idx = kv_it - 1 - d;
-                mbar_wait_drain(bar_full(idx % NSLOT), (uint32_t)(idx / NSLOT) & 1u, p.timeout_ns,
+            for (int d = 0; d < (kq < NK ? kq : NK); ++d) {
+                const int idx = kq - 1 - d;
+                mbar_wait_drain(bar_kfull(idx % NK), (uint32_t)(idx / NK) & 1u, p.timeout_ns,
+                                p.status);
+            }
+            for (int d = 0; d < (vq < NV ? vq : NV); ++d) {
+                const int idx = vq - 1 - d;
+                mbar_wait_drain(bar_vfull(idx % NV), (uint32_t)(idx / NV) & 1u, p.timeout_ns,
                                 p.status);
             }
             if (q_cnt > 0)
                 mbar_wait_drain(bar_q_full, (uint32_t)(q_cnt - 1) & 1u, p.timeout_ns, p.status);
         }
-        } else {
+    } else if (warp == T::MMA_WARP) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
             bool ok = true;
-            int kv_it = 0;   // K/V items consumed
-            int64_t gb = 0;  // global block counter (S buffer index and barrier phases)
-            int tiles = 0;   // busy tiles started
-            auto take = [&](uint32_t& addr, int& slot) -> bool {
-                slot = kv_it % NSLOT;
-                const uint32_t phase = (uint32_t)(kv_it / NSLOT) & 1u;
-                ++kv_it;
-                if (!mbar_wait(bar_full(slot), phase, wc, kErrTimeout)) return false;
-                addr = slots + slot * T::SLOT_BYTES;
-                return true;
-            };
-            auto qk = [&](int64_t gblk) {
-                uint32_t kaddr;
-                int slot;
-                if (!take(kaddr, slot)) {
-                    ok = false;
-                    return;
+            int kq = 0, vq = 0;  // K / V items taken
+            int64_t gi = 0;      // global item counter (score buffer and barrier phases)
+            int units = 0;       // busy units started
+            uint32_t kaddr = 0, vaddr = 0;
+            int kslot = 0, vslot = 0;
+            // Q K^T of item gi = (block j, tile tt) of the current unit.
+            auto qk = [&](int j, int tt, bool last_item) {
+                if (tt == 0) {
+                    kslot = kq % NK;
+                    const uint32_t phase = (uint32_t)(kq / NK) & 1u;
+                    ++kq;
+                    if (!mbar_wait(bar_kfull(kslot), phase, wc, kErrTimeout)) {
+                        ok = false;
+                        return;
+                    }
+                    kaddr = k_slots + kslot * T::K_TILE_BYTES;
                 }
-                const uint32_t d_tmem = tmem + T::S_COL + (uint32_t)(gblk & 1) * BN;
+                const uint32_t d_tmem = tmem + (uint32_t)(gi & 1) * BN;
 #pragma unroll
                 for (int kk = 0; kk < T::DQK / 16; ++kk) {
                     const uint64_t bdesc = make_sdesc_sw128(
                         kaddr + (kk >> 2) * T::CHUNK_BYTES + (kk & 3) * 32, 16, 1024);
-                    mma_ts(d_tmem, tmem + T::Q_COL + kk * 8, bdesc, p.idesc_qk, kk > 0 ? 1u : 0u);
+                    if (T::Q_TMEM) {
+                        mma_ts(d_tmem, tmem + T::Q_COL0 + tt * (T::DQK / 2) + kk * 8, bdesc,
+                               p.idesc_qk, kk > 0 ? 1u : 0u);
+                    } else {
+                        const uint64_t adesc = make_sdesc_sw128(
+                            q_stage + tt * T::Q_TILE_BYTES + (kk >> 2) * T::QCHUNK_BYTES +
+                                (kk & 3) * 32,
+                            16, 1024);
+                        mma_ss(d_tmem, adesc, bdesc, p.idesc_qk, kk > 0 ? 1u : 0u);
+                    }
                 }
-                tc_commit(bar_s_full(gblk & 1));
-                tc_commit(bar_empty(slot));
+                tc_commit(bar_s_full(gi & 1));
+                if (tt == NT - 1) tc_commit(bar_kempty(kslot));
+                if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
             };
-            // P V for global block gblk; `first` / `last`: its position inside tile `tile_idx`.
-            auto pv = [&](int64_t gblk, bool first, bool last, int tile_idx) {
-                if (!mbar_wait(bar_p_full(gblk & 1), (uint32_t)(gblk >> 1) & 1u, wc,
-                               kErrTimeout)) {
+            // P V of item g = (block j, tile tt) of busy unit number uidx.
+            auto pv = [&](int64_t g, int j, int tt, bool last_item, int uidx) {
+                if (!mbar_wait(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
-                if (first && tile_idx > 0 &&
-                    !mbar_wait(bar_o_free, (uint32_t)(tile_idx - 1) & 1u, wc, kErrTimeout)) {
+                if (j == 0 && tt == 0 && uidx > 0 &&
+                    !mbar_wait(bar_o_free, (uint32_t)(uidx - 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
                 tc_fence_after_sync();
-                uint32_t vaddr;
-                int slot;
-                if (!take(vaddr, slot)) {
-                    ok = false;
-                    return;
+                if (tt == 0) {
+                    vslot = vq % NV;
+                    const uint32_t phase = (uint32_t)(vq / NV) & 1u;
+                    ++vq;
+                    if (!mbar_wait(bar_vfull(vslot), phase, wc, kErrTimeout)) {
+                        ok = false;
+                        return;
+                    }
+                    vaddr = v_slots + vslot * T::V_TILE_BYTES;
                 }
-                const uint32_t p_tmem = tmem + T::S_COL + (uint32_t)(gblk & 1) * BN;
+                const uint32_t p_tmem = tmem + (uint32_t)(g & 1) * BN;
+                const uint32_t o_tmem = tmem + T::O_COL0 + tt * T::DV;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t bdesc =
                         make_sdesc_sw128(vaddr + kk * 2048, T::CHUNK_BYTES, 1024);
-                    mma_ts(tmem + T::O_COL, p_tmem + kk * 8, bdesc, T::IDESC_PV,
-                           (!first || kk > 0) ? 1u : 0u);
+                    mma_ts(o_tmem, p_tmem + kk * 8, bdesc, T::IDESC_PV,
+                           (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(bar_pv_done);
-                tc_commit(bar_empty(slot));
-                if (last) tc_commit(bar_o_full);
+                if (NT == 1) tc_commit(bar_pv_done);
+                if (tt == NT - 1) tc_commit(bar_vempty(vslot));
+                if (last_item) tc_commit(bar_o_full);
             };
-            // The P V of a tile's last block is issued after the next tile's first Q K^T, so the
-            // next tile's first S is computed while the softmax finishes this tile.
-            bool pend = false, pend_first = false, pend_last = false;
-            int pend_tile = 0;
+            // The P V of each item is issued after the next item's Q K^T (also across units), so
+            // the tensor core computes the next S while the softmax works on this one.
+            bool pend = false, pend_last = false;
+            int pend_j = 0, pend_tt = 0, pend_u = 0;
             int64_t pend_g = 0;
-            for (int64_t u = u0; u < p.n_tiles && ok; u += ustep) {
-                const TileInfo t = tile_info<BN, CAUSAL>(p, u);
+            for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
+                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
                 if (t.n_blocks == 0) continue;
-                if (!mbar_wait(bar_q_tmem, (uint32_t)(tiles & 1), wc, kErrTimeout)) {
+                const uint32_t qbar = T::Q_TMEM ? bar_q_tmem : bar_q_full;
+                if (!mbar_wait(qbar, (uint32_t)(units & 1), wc, kErrTimeout)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after_sync();
                 for (int j = 0; j < t.n_blocks && ok; ++j) {
-                    qk(gb);
-                    if (!ok) break;
-                    if (pend) pv(pend_g, pend_first, pend_last, pend_tile);
-                    pend = true;
-                    pend_g = gb;
-                    pend_first = (j == 0);
-                    pend_last = (j == t.n_blocks - 1);
-                    pend_tile = tiles;
-                    ++gb;
+                    for (int tt = 0; tt < NT && ok; ++tt) {
+                        const bool last_item = (j == t.n_blocks - 1) && (tt == NT - 1);
+                        qk(j, tt, last_item);
+                        if (!ok) break;
+                        if (pend) pv(pend_g, pend_j, pend_tt, pend_last, pend_u);
+                        pend = true;
+                        pend_g = gi;
+                        pend_j = j;
+                        pend_tt = tt;
+                        pend_last = last_item;
+                        pend_u = units;
+                        ++gi;
+                    }
                 }
-                ++tiles;
+                ++units;
             }
-            if (ok && pend) pv(pend_g, pend_first, pend_last, pend_tile);
+            if (ok && pend) pv(pend_g, pend_j, pend_tt, pend_last, pend_u);
             tc_commit(bar_mma_done);  // drain every MMA this thread issued before teardown
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
-        }
     } else {
-        // --------------------------- softmax + epilogue warps 0-3 ---------------------------
-        const int row = threadIdx.x;  // TMEM lane
-        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        // ---------------------- softmax + epilogue warpgroups (warps 0 .. 4*NT-1) ----------------------
+        const int wg = warp >> 2;           // the query tile this warpgroup owns
+        const int row = threadIdx.x & 127;  // TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float sl2 = p.scale_log2;
         bool ok = true;
-        int64_t gb = 0;
-        int tiles = 0;  // busy tiles whose key blocks are done
+        int64_t wi = 0;  // items of this warpgroup's tile processed so far
+        int units = 0;   // busy units whose items are done
 
-        // Staged Q tile number qidx (128-byte swizzled rows, as TMA wrote them) -> this row's
-        // TMEM columns; then release the staging buffer and tell the MMA warp.
+        // Staged Q of busy unit number qidx, tile wg (128-byte swizzled rows, as TMA wrote them)
+        // -> this row's TMEM columns; then release the staging buffer and tell the MMA warp.
         auto copy_q = [&](int qidx) -> bool {
             if (!__all_sync(FULL, mbar_wait(bar_q_full, (uint32_t)(qidx & 1), wc, kErrTimeout)))
                 return false;
 #pragma unroll
             for (int ch = 0; ch < T::QCH; ++ch) {
                 uint32_t r[32];
-                const uint8_t* rowp = smem + ch * T::QCHUNK_BYTES + row * 128;
+                const uint8_t* rowp = smem + wg * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES + row * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
-                    const uint4 x =
-                        *reinterpret_cast<const uint4*>(rowp + ((c ^ (row & 7)) << 4));
+                    const uint4 x = *reinterpret_cast<const uint4*>(rowp + ((c ^ (row & 7)) << 4));
                     r[4 * c + 0] = x.x;
                     r[4 * c + 1] = x.y;
                     r[4 * c + 2] = x.z;
                     r[4 * c + 3] = x.w;
                 }
-                tmem_st32(tl + T::Q_COL + ch * 32, r);
+                tmem_st32(tl + T::Q_COL0 + wg * (T::DQK / 2) + ch * 32, r);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -414,14 +477,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             return true;
         };
 
-        // Epilogue of busy tile number tile_idx: wait for its last P V, read this row of O from
-        // TMEM (then free the accumulator for the next tile), write O / l in bf16 and the LSE.
-        auto epilogue = [&](const TileInfo& t, float m_ref, float l, int tile_idx) -> bool {
-            if (!__all_sync(FULL, mbar_wait(bar_o_full, (uint32_t)(tile_idx & 1), wc,
-                                            kErrTimeout)))
+        // Epilogue of busy unit number uidx: wait for its last P V, read this row of O (tile wg)
+        // from TMEM (then free the accumulators for the next unit), write O / l and the LSE.
+        auto epilogue = [&](const UnitInfo& t, float m_ref, float l, int uidx) -> bool {
+            if (!__all_sync(FULL, mbar_wait(bar_o_full, (uint32_t)(uidx & 1), wc, kErrTimeout)))
                 return false;
             tc_fence_after_sync();
-            const int64_t i = t.q0 + row;
+            const int64_t i = t.q0 + wg * 128 + row;
             const bool row_valid = i < p.sq;
             uint4* dst = reinterpret_cast<uint4*>(
                 p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
@@ -429,10 +491,10 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll 1
             for (int c = 0; c < T::DV / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tl + T::O_COL + c * 32, r);
+                tmem_ld32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
                 tmem_wait_ld();
                 if (c == T::DV / 32 - 1) {
-                    // O has been read out: the next tile's first P V may overwrite it.
+                    // this tile's O has been read out: the next unit's P V may overwrite it
                     tc_fence_before_sync();
                     mbar_arrive(bar_o_free);
                 }
@@ -454,18 +516,28 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             return true;
         };
 
-        bool pend = false;  // a finished tile whose epilogue has not run yet
-        TileInfo pend_t{};
+        // exp2(s * sl2 - m) for two scores, and their bf16 pair; masked keys give exactly 0.
+        auto p_pair = [&](uint32_t s0, uint32_t s1, float neg_m, bool v0, bool v1, float& p0,
+                          float& p1) -> uint32_t {
+            p0 = ex2(fmaf(__uint_as_float(s0), sl2, neg_m));
+            p1 = ex2(fmaf(__uint_as_float(s1), sl2, neg_m));
+            p0 = v0 ? p0 : 0.f;
+            p1 = v1 ? p1 : 0.f;
+            return pack_bf16x2(p0, p1);
+        };
+
+        bool pend = false;  // a finished unit whose epilogue has not run yet
+        UnitInfo pend_t{};
         float pend_m = 0.f, pend_l = 0.f;
         int pend_idx = 0;
-        if (busy_from(u0) >= 0) ok = copy_q(0);
-        for (int64_t u = u0; u < p.n_tiles && ok; u += ustep) {
-            const TileInfo t = tile_info<BN, CAUSAL>(p, u);
-            if (t.n_blocks == 0) {  // no key at all for any row of this tile: O = 0, LSE = -inf
-                const int64_t i = t.q0 + row;
+        if (T::Q_TMEM && busy_from(u0) >= 0) ok = copy_q(0);
+        for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
+            const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+            const int64_t i = t.q0 + wg * 128 + row;
+            if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
                 if (i < p.sq) {
-                    uint4* dst = reinterpret_cast<uint4*>(
-                        p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
+                    uint4* dst =
+                        reinterpret_cast<uint4*>(p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
 #pragma unroll 1
                     for (int c = 0; c < T::DV / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
                     if (p.lse) p.lse[(t.bi * p.hq + t.h) * p.sq + i] = -INFINITY;
@@ -473,111 +545,191 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 continue;
             }
             const int64_t un = busy_from(u + ustep);
-            const int64_t i = t.q0 + row;
             const int64_t lim_row = CAUSAL ? i + p.sk - p.sq : p.sk - 1;
             const int64_t lim = lim_row < p.sk - 1 ? lim_row : p.sk - 1;  // last allowed key
             float m_ref = -INFINITY;  // exponent reference (log2 units); moves lazily
             float l = 0.f;            // sum of exp2(x - m_ref) over the keys seen so far
 
-            for (int j = 0; j < t.n_blocks; ++j, ++gb) {
-                const int sb = (int)(gb & 1);
-                ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(gb >> 1) & 1u, wc,
-                                                kErrTimeout));
+            for (int j = 0; j < t.n_blocks; ++j, ++wi) {
+                // score buffer and its phase: one buffer per tile with two tiles, alternating
+                // buffers with one tile
+                const int sb = NT == 2 ? wg : (int)(wi & 1);
+                const uint32_t sph = NT == 2 ? (uint32_t)(wi & 1) : (uint32_t)(wi >> 1) & 1u;
+                const uint32_t s_col = tl + sb * BN;
+                ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), sph, wc, kErrTimeout));
                 if (!ok) break;
                 tc_fence_after_sync();
-                if (j == t.n_blocks - 1 && un >= 0) {
-                    // Every Q K^T of this tile is complete (its last S has landed), so the Q
-                    // columns can take the next tile's Q now, ahead of this block's softmax.
-                    ok = copy_q(tiles + 1);
+                if (T::Q_TMEM && j == t.n_blocks - 1 && un >= 0) {
+                    // Every Q K^T of this tile in this unit is complete (its last S has landed),
+                    // so its Q columns can take the next unit's Q now, ahead of this softmax.
+                    ok = copy_q(units + 1);
                     if (!ok) break;
                 }
-                uint32_t sr[BN];
-#pragma unroll
-                for (int c = 0; c < BN / 32; ++c)
-                    tmem_ld32(tl + T::S_COL + sb * BN + c * 32,
-                              *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-                tmem_wait_ld();
-
                 const bool masked_block = j >= t.mask_from;
-                // keys kbase + c with c <= rel are allowed (rel < 0: none, rel >= BN - 1: all)
+                // keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all)
                 int64_t rel64 = lim - (int64_t)j * BN;
                 rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
                 const int rel = (int)rel64;
-                float mx[4];
+
+                float bmax;
+                float rs = 0.f;  // sum of this block's p (relative to the reference after it)
+                float m_new, alpha = 1.f;
+                bool need;
+                if (NT == 1) {
+                    // ---- single pass: the whole score row stays in registers
+                    uint32_t sr[BN];
 #pragma unroll
-                for (int a = 0; a < 4; ++a) mx[a] = -INFINITY;
-                if (masked_block) {
+                    for (int c = 0; c < BN / 32; ++c)
+                        tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                    tmem_wait_ld();
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    if (masked_block) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const float s = (c <= rel) ? __uint_as_float(sr[c]) : -INFINITY;
-                        mx[c & 3] = fmaxf(mx[c & 3], s);
-                        sr[c] = __float_as_uint(s);
+                        for (int c = 0; c < BN; ++c)
+                            mx[c & 3] = fmaxf(mx[c & 3], c <= rel ? __uint_as_float(sr[c]) : -INFINITY);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < BN; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
                     }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c)
-                        mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
-                }
-                const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
-                const float m_new = fmaxf(m_ref, m_blk);
-                // Lazy rescale: keep the old reference while the running max stays within 2^8 of
-                // it; the final O / l uses the same reference, so the result is exact either way.
-                const bool need = m_new > m_ref + 8.0f;
-                float alpha = 1.f;
-                if (need) {
-                    alpha = ex2(m_ref - m_new);
-                    m_ref = m_new;
-                    l *= alpha;
-                }
-                if (j > 0 && __any_sync(FULL, need)) {
-                    // O holds blocks < j: wait for the previous P V, then scale O in place. When
-                    // S_gb has landed, P V of block gb-2 is complete (it was issued before this
-                    // Q K^T), so bar_pv_done is in phase gb-1 or gb and the parity test on phase
-                    // gb-1 is unambiguous.
-                    ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(gb - 1) & 1u, wc,
-                                                    kErrTimeout));
-                    if (!ok) break;
-                    tc_fence_after_sync();
+                    bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
+                    m_new = fmaxf(m_ref, m_blk);
+                    need = m_new > m_ref + 8.0f;
+                    if (need) {
+                        alpha = ex2(m_ref - m_new);
+                        m_ref = m_new;
+                        l *= alpha;
+                    }
+                    if (j > 0 && __any_sync(FULL, need)) {
+                        // O holds blocks < j: wait for the previous P V (item wi-1; bar_pv_done
+                        // is then in phase wi-1 or wi, so the parity test is unambiguous), then
+                        // scale O in place.
+                        ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(wi - 1) & 1u, wc,
+                                                        kErrTimeout));
+                        if (!ok) break;
+                        tc_fence_after_sync();
 #pragma unroll 1
-                    for (int c = 0; c < T::DV / 32; ++c) {
-                        uint32_t r[32];
-                        tmem_ld32(tl + T::O_COL + c * 32, r);
-                        tmem_wait_ld();
+                        for (int c = 0; c < T::DV / 32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(tl + T::O_COL0 + c * 32, r);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                        tmem_st32(tl + T::O_COL + c * 32, r);
-                    }
-                }
-                const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                float acc[4];
-#pragma unroll
-                for (int a = 0; a < 4; ++a) acc[a] = 0.f;
-#pragma unroll
-                for (int h2 = 0; h2 < BN / 64; ++h2) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        const int e = h2 * 64 + 2 * c;
-                        float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, neg_m));
-                        float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, neg_m));
-                        if (masked_block) {  // masked keys hold -inf: exactly 0 for any scale
-                            p0 = (e <= rel) ? p0 : 0.f;
-                            p1 = (e + 1 <= rel) ? p1 : 0.f;
+                            for (int e = 0; e < 32; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(tl + T::O_COL0 + c * 32, r);
                         }
-                        acc[(2 * c) & 3] += p0;
-                        acc[(2 * c + 1) & 3] += p1;
-                        pk[c] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(tl + T::S_COL + sb * BN + h2 * 32, pk);
+                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int h2 = 0; h2 < BN / 64; ++h2) {
+                        uint32_t pk[32];
+                        if (masked_block) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const int e = h2 * 64 + 2 * c;
+                                float p0, p1;
+                                pk[c] = p_pair(sr[e], sr[e + 1], neg_m, e <= rel, e + 1 <= rel, p0, p1);
+                                acc[(2 * c) & 3] += p0;
+                                acc[(2 * c + 1) & 3] += p1;
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const int e = h2 * 64 + 2 * c;
+                                float p0, p1;
+                                pk[c] = p_pair(sr[e], sr[e + 1], neg_m, true, true, p0, p1);
+                                acc[(2 * c) & 3] += p0;
+                                acc[(2 * c + 1) & 3] += p1;
+                            }
+                        }
+                        tmem_st32(s_col + h2 * 32, pk);
+                    }
+                    rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                } else {
+                    // ---- two passes over TMEM in 32-column chunks (max, then exp), so that few
+                    // registers are live; the next chunk's load overlaps this chunk's math.
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32(s_col, ra);
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t (&cur)[32] = (c & 1) ? rb : ra;
+                        uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
+                        tmem_wait_ld();
+                        if (c + 1 < BN / 32) tmem_ld32(s_col + (c + 1) * 32, nxt);
+                        if (masked_block) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                mx[e & 3] = fmaxf(mx[e & 3], c * 32 + e <= rel ? __uint_as_float(cur[e]) : -INFINITY);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(cur[e]));
+                        }
+                    }
+                    bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
+                    m_new = fmaxf(m_ref, m_blk);
+                    need = m_new > m_ref + 8.0f;
+                    if (need) {
+                        alpha = ex2(m_ref - m_new);
+                        m_ref = m_new;
+                        l *= alpha;
+                    }
+                    if (j > 0 && __any_sync(FULL, need)) {
+                        // O holds blocks < j of this tile. Its last P V (item of block j-1) was
+                        // issued before this block's Q K^T, so it is complete now that S has
+                        // landed: scale O in place.
+#pragma unroll 1
+                        for (int c = 0; c < T::DV / 32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
+                        }
+                    }
+                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    tmem_ld32(s_col, ra);
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c) {
+                        uint32_t (&cur)[32] = (c & 1) ? rb : ra;
+                        uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
+                        tmem_wait_ld();
+                        if (c + 1 < BN / 32) tmem_ld32(s_col + (c + 1) * 32, nxt);
+                        uint32_t pk[16];
+                        if (masked_block) {
+#pragma unroll
+                            for (int e2 = 0; e2 < 16; ++e2) {
+                                const int e = c * 32 + 2 * e2;
+                                float p0, p1;
+                                pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, e <= rel, e + 1 <= rel, p0, p1);
+                                acc[(2 * e2) & 3] += p0;
+                                acc[(2 * e2 + 1) & 3] += p1;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e2 = 0; e2 < 16; ++e2) {
+                                float p0, p1;
+                                pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, true, true, p0, p1);
+                                acc[(2 * e2) & 3] += p0;
+                                acc[(2 * e2 + 1) & 3] += p1;
+                            }
+                        }
+                        // P chunk c (16 columns of bf16 pairs) overwrites S columns already read
+                        tmem_st16(s_col + c * 16, pk);
+                    }
+                    rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
                 }
-                l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                l += rs;
                 tmem_wait_st();
                 tc_fence_before_sync();
                 mbar_arrive(bar_p_full(sb));
                 if (j == 0 && pend) {
-                    // The previous tile's epilogue, now that this tile's first P is handed over.
+                    // The previous unit's epilogue, now that this unit's first P is out.
                     pend = false;
                     ok = epilogue(pend_t, pend_m, pend_l, pend_idx);
                     if (!ok) break;
@@ -588,8 +740,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             pend_t = t;
             pend_m = m_ref;
             pend_l = l;
-            pend_idx = tiles;
-            ++tiles;
+            pend_idx = units;
+            ++units;
         }
         if (ok && pend) ok = epilogue(pend_t, pend_m, pend_l, pend_idx);
     }
@@ -597,7 +749,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     // ---- teardown: every tcgen05 access is complete (MMAs drained, loads waited) ----
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == T::MMA_WARP) {
         __syncwarp();
         tc_fence_after_sync();
         tmem_dealloc(tmem, T::TMEM_COLS);
