@@ -8,8 +8,8 @@ the computation runs in the library's CUDA kernels; there is no CPU or PyTorch f
 importing this package fails loudly when the library is missing.
 
 Raw C entry points, with the header's names and argument order, are exposed through ``lib``
-(a ``ctypes.CDLL``): ``lib.attn_fwd``, ``lib.k_smooth_mean``, ``lib.k_smooth_sub``,
-``lib.attn_status_string``, ``lib.attn_debug_status``.
+(a ``ctypes.CDLL``): ``lib.attn_fwd``, ``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``,
+``lib.k_smooth_sub``, ``lib.attn_status_string``, ``lib.attn_debug_status``.
 """
 from __future__ import annotations
 
@@ -23,9 +23,10 @@ LIB_PATH = os.path.join(_HERE, "libb200attn.so")
 STATUS = {
     0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_GQA", 4: "ERR_HEADDIM", 5: "ERR_ALIGN",
     6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
+    11: "ERR_SCRATCH",
 }
-EXPORTS = ("attn_fwd", "k_smooth_mean", "k_smooth_sub", "attn_status_string",
-           "attn_debug_status")
+EXPORTS = ("attn_fwd", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+           "attn_status_string", "attn_debug_status")
 
 
 class B200AttnError(RuntimeError):
@@ -46,6 +47,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd.restype = ctypes.c_int
     lib.k_smooth_mean.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean.restype = ctypes.c_int
+    lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
+    lib.k_smooth_mean_noalloc.restype = ctypes.c_int
     lib.k_smooth_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_sub.restype = ctypes.c_int
     lib.attn_status_string.argtypes = [ctypes.c_int]
@@ -122,6 +125,20 @@ def k_smooth_mean(k, mean=None):
         mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
     _check("k_smooth_mean",
            lib.k_smooth_mean(k.data_ptr(), mean.data_ptr(), b, hk, sk, d, _stream_ptr(k)))
+    return mean
+
+
+def k_smooth_mean_noalloc(k, mean):
+    """k_smooth_mean without any device allocation inside the call (fixed library scratch);
+    ``mean`` [b, hk, d] fp32 must be supplied by the caller."""
+    import torch
+    _want(k, "k", 4)
+    _want(mean, "mean", 3)
+    if k.dtype != torch.bfloat16 or mean.dtype != torch.float32:
+        raise TypeError("k must be bfloat16 and mean float32")
+    b, sk, hk, d = k.shape
+    _check("k_smooth_mean_noalloc", lib.k_smooth_mean_noalloc(k.data_ptr(), mean.data_ptr(), b, hk,
+                                                              sk, d, _stream_ptr(k)))
     return mean
 
 

@@ -237,6 +237,8 @@ extern "C" const char* attn_status_string(int status)
     case B200ATTN_ERR_ARCH: return "device is not compute capability 10.0 (sm_100)";
     case B200ATTN_ERR_CUDA: return "CUDA call or kernel launch failed";
     case B200ATTN_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case B200ATTN_ERR_SCRATCH:
+        return "b*hk*d exceeds the fixed scratch of k_smooth_mean_noalloc (2^20 floats)";
     default: return "unknown status";
     }
 }

@@ -106,6 +106,11 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// Fixed partial-sum scratch for k_smooth_mean_noalloc: file-scope device memory that every GPU
+// loading this library holds until the process exits. 1 Mi floats (4 MiB).
+constexpr int64_t kNoAllocScratchFloats = (int64_t)1 << 20;
+__device__ __align__(256) float g_kmean_scratch[kNoAllocScratchFloats];
+
 int check_kmean_args(const void* k, const void* mean, int64_t b, int64_t hk, int64_t sk,
                      int64_t d, int64_t* cols_out)
 {
@@ -164,6 +169,61 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
         return B200ATTN_ERR_CUDA;
     }
     return launched ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+// Device address of g_kmean_scratch on the current device, looked up once per device (the
+// host-side name of a __device__ array is not a device address).
+static float* noalloc_scratch()
+{
+    static float* addr[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_kmean_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        addr[dev] = static_cast<float*>(p);
+    }
+    return addr[dev];
+}
+
+extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk,
+                                     int64_t d, void* stream)
+{
+    int64_t cols = 0;
+    int rc = check_kmean_args(k, mean, b, hk, sk, d, &cols);
+    if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
+    if (b * cols > kNoAllocScratchFloats) return B200ATTN_ERR_SCRATCH;
+    rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    float* partial = noalloc_scratch();
+    if (!partial) return B200ATTN_ERR_CUDA;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // Same split as k_smooth_mean, capped so that the partials fit in the fixed scratch.
+    const int64_t col_ctas = (cols + kColsPerCta - 1) / kColsPerCta;
+    int64_t nchunks = (kTargetCtas + col_ctas * b - 1) / (col_ctas * b);
+    const int64_t max_chunks = (sk + kMinRowsPerChunk - 1) / kMinRowsPerChunk;
+    if (nchunks > max_chunks) nchunks = max_chunks;
+    if (nchunks > 1024) nchunks = 1024;
+    if (nchunks > kNoAllocScratchFloats / (b * cols)) nchunks = kNoAllocScratchFloats / (b * cols);
+    if (nchunks < 1) nchunks = 1;
+    const int64_t rows_per_chunk = (sk + nchunks - 1) / nchunks;
+    nchunks = (sk + rows_per_chunk - 1) / rows_per_chunk;
+
+    // Every partial the fold reads is written by k_mean_partial first, so nothing needs clearing.
+    dim3 g1((unsigned)col_ctas, (unsigned)nchunks, (unsigned)b);
+    k_mean_partial<<<g1, kThreads, 0, st>>>(static_cast<const uint4*>(k), partial, sk, cols,
+                                            rows_per_chunk, (int)nchunks);
+    const int64_t n = b * cols;
+    k_mean_fold<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+        partial, mean, b, cols, (int)nchunks, (float)sk);
+    return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
 extern "C" int k_smooth_sub(const void* k, const float* mean, void* k_out, int64_t b, int64_t hk,

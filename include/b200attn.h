@@ -49,6 +49,7 @@ enum b200attn_status {
     B200ATTN_ERR_ARCH = 8,     /* the current device is not compute capability 10.0 (sm_100) */
     B200ATTN_ERR_CUDA = 9,     /* a CUDA runtime / driver call or a kernel launch failed */
     B200ATTN_ERR_TIMEOUT = 10, /* a kernel gave up on a bounded wait (see attn_debug_status) */
+    B200ATTN_ERR_SCRATCH = 11, /* b*hk*d exceeds the fixed scratch of k_smooth_mean_noalloc */
 };
 
 /*
@@ -98,6 +99,30 @@ B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out
  */
 B200ATTN_API int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk, int64_t d,
                   void* stream);
+
+/*
+ * k_smooth_mean_noalloc -- k_smooth_mean for callers that must not allocate device memory.
+ *
+ * No counterpart on the reference pages: this entry point exists for callers that cannot let a
+ * library allocate during a call -- for example a serving process that reserves all device
+ * memory for its own pool at start-up (so a cudaMallocAsync inside the call could fail, or
+ * stall the stream while the driver maps memory), or code that must keep its memory use fixed
+ * and known in advance. It computes the same mean as k_smooth_mean with the same two kernels,
+ * but takes the partial sums from a fixed file-scope device array of 2^20 floats (4 MiB) that
+ * every GPU which loads this library holds until the process exits. It never calls cudaMalloc,
+ * cudaFree or any allocating routine.
+ *
+ *   Arguments, layout and alignment as for k_smooth_mean.
+ *   Limit: b * hk * d <= 2^20 (one fp32 partial row per batch must fit); larger problems are
+ *   refused with B200ATTN_ERR_SCRATCH before anything is launched. Long sequences are folded in
+ *   fewer, longer chunks so that the partials always fit.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current; make that first call before any stream capture.
+ *   Every call on a device shares the one array and leaves its contents behind: calls whose
+ *   kernels overlap on the GPU (for example on two streams) race, so serialise them.
+ */
+B200ATTN_API int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int64_t hk,
+                                       int64_t sk, int64_t d, void* stream);
 
 /*
  * k_smooth_sub -- subtract the channel mean from K: k_out = bf16_rne(float(K) - mean),

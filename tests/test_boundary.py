@@ -21,7 +21,7 @@ def test_exports_every_header_function():
 
 
 def test_status_strings():
-    for code in range(0, 11):
+    for code in range(0, 12):
         s = b2.lib.attn_status_string(code)
         assert s and s.decode() != "unknown status"
     assert b2.lib.attn_status_string(99).decode() == "unknown status"
@@ -52,6 +52,12 @@ def test_empty_problem_is_a_no_op():
     assert call(b=0, q=None, k=None, v=None, o=None, lse=None) == 0
     assert call(sq=0, q=None, o=None, lse=None) == 0
     assert call(hq=0, hk=1, q=None, o=None, lse=None) == 0
+
+
+def test_noalloc_mean_size_limit():
+    # b * hk * d above the fixed 2^20-float scratch is refused before any CUDA call
+    assert b2.lib.k_smooth_mean_noalloc(A, A, 1, 4097, 16, 256, None) == 11
+    assert b2.lib.k_smooth_mean_noalloc(A, A, 1, 4, 16, 96, None) == 4
 
 
 @pytest.mark.parametrize("fn", ["k_smooth_mean", "k_smooth_sub"])
