@@ -94,8 +94,10 @@ B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out
  *   k     device bf16 [b, sk, hk, d], 16-byte aligned.
  *   mean  device fp32 [b, hk, d], 16-byte aligned. Fully written.
  *   d     64, 128 or 256 (the head dims the page's host check accepts). sk > 0.
- * Takes its partial-sum scratch from cudaMallocAsync on `stream` and frees it on the same
- * stream, so concurrent calls on different streams do not share scratch.
+ * Takes its partial-sum scratch (b * hk * d * chunks floats, at most 4 MiB per 1024 channels)
+ * from a library-owned stream-ordered memory pool on `stream` and frees it on the same stream,
+ * so concurrent calls on different streams never share scratch. The pool keeps freed memory for
+ * later calls (it is created on the first call on a device and lives until the process exits).
  */
 B200ATTN_API int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk, int64_t d,
                   void* stream);
