@@ -147,13 +147,14 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     return B200ATTN_OK;
 }
 
-// Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, Q in TMEM,
-// K slots, V slots>. Tensor memory holds two score buffers, one O per query tile and (when it
-// fits) each tile's Q; shared memory holds the Q staging buffer and the K / V rings.
-using T64 = AttnTraits<64, 64, 128, 2, true, 5, 5>;       // smem 32 + 80 + 80 KB
-using T128 = AttnTraits<128, 128, 128, 2, false, 3, 2>;   // smem 64 + 96 + 64 KB
-using T192 = AttnTraits<192, 128, 128, 2, false, 2, 1>;   // smem 96 + 96 + 32 KB
-using T256 = AttnTraits<256, 256, 64, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
+// Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, softmax
+// warpgroups, Q in TMEM, K slots, V slots>. Tensor memory holds two score buffers, one O per query
+// tile and (when it fits) each tile's Q; shared memory holds the Q staging buffer and the K / V
+// rings. The (tiles, warpgroups) choice per head dim is the measured fastest on B200.
+using T64 = AttnTraits<64, 64, 128, 1, 1, true, 6, 6>;       // smem 16 + 96 + 96 KB
+using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2>;   // smem 64 + 96 + 64 KB
+using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1>;   // smem 96 + 96 + 32 KB
+using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
 template <class T>
 int dispatch_causal(int causal, const void* q, const void* k, const void* v, void* out,

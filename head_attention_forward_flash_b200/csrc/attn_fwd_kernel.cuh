@@ -16,21 +16,24 @@
 // (0,0) (0,1) (1,0) (1,1) ... for NT = 2, or (0) (1) (2) ... for NT = 1. Item g uses score buffer
 // g % 2, so one item's Q K^T runs on the tensor core while the previous item's softmax runs.
 //
-// Roles (NT softmax warpgroups + 2 warps: 320 threads for NT = 2, 192 for NT = 1):
-//   warps 4t..4t+3  softmax + epilogue of query tile t: thread r owns row r of tile t (= TMEM
-//              lane r). Turns each score block S into P (online softmax: exp2 with the scale
-//              folded into one FMA, lazy rescaling of O), and writes the finished O rows (divided
-//              by the row sums) and LSE; a unit's epilogue runs right after the next unit's
-//              first P of the tile is handed over. When Q lives in TMEM, each warpgroup also
-//              copies its tile's Q from the shared-memory staging buffer into TMEM. With two
-//              warpgroups the two tiles' softmax run side by side (two warps per SM
-//              sub-partition); each thread then reads its score row from TMEM twice (max, then
-//              exp) in 32-column chunks, so that its registers stay within the 10-warp budget.
-//   warp 4*NT  MMA issuer (one thread): S = Q K^T and O += P V. A operand: Q from TMEM or shared
-//              memory, then P from TMEM; B operand: K, V from shared memory; fp32 accumulators
-//              in TMEM.
-//   warp 4*NT+1 TMA producer (one thread): each unit's Q into the staging buffer, and K, V tiles
-//              through two rings of shared-memory slots, in the order the MMA warp takes them.
+// Roles (NSM softmax warpgroups + 2 warps): NSM = 1 (192 threads) or NSM = NT = 2 (320 threads).
+//   softmax + epilogue warps: thread r owns row r (= TMEM lane r) of a query tile. Turns each
+//              score block S into P (online softmax: exp2 with the scale folded into one FMA,
+//              lazy rescaling of O), and writes each tile's finished O rows (divided by the row
+//              sums) and LSE right after handing over that tile's first P of the next unit. When
+//              Q lives in TMEM they also copy each tile's Q from the shared-memory staging buffer
+//              into TMEM once the tile's last Q K^T of the current unit has landed.
+//              NSM = 1: warps 0-3 take every item in order and keep the whole score row in
+//              registers (at most two warps per SM sub-partition allow up to 255 registers).
+//              NSM = 2: warps 4t..4t+3 own query tile t, so the two tiles' softmax run side by
+//              side; within the 10-warp register budget each thread reads its score row from
+//              TMEM twice (max, then exp) in 32-column chunks.
+//   warp 4*NSM   MMA issuer (one thread): S = Q K^T and O += P V. A operand: Q from TMEM or
+//              shared memory, then P from TMEM; B operand: K, V from shared memory; fp32
+//              accumulators in TMEM.
+//   warp 4*NSM+1 TMA producer (one thread): each unit's Q into the staging buffer, and K, V
+//              tiles through two rings of shared-memory slots, in the order the MMA warp takes
+//              them.
 //
 // Tensor memory (128 lanes x 512 columns of 32 bit): S0 | S1 (BN columns each; P in bf16 pairs
 // overwrites the first BN/2 columns of its own S buffer) | O for each query tile (DV fp32
@@ -63,13 +66,14 @@ struct AttnParams {
     unsigned long long timeout_ns;
 };
 
-template <int DQK_, int DV_, int BN_, int NT_, bool Q_TMEM_, int NK_, int NV_>
+template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_>
 struct AttnTraits {
     static constexpr int DQK = DQK_;
     static constexpr int DV = DV_;
     static constexpr int BN = BN_;          // keys per block
     static constexpr int BM = 128;          // query rows per tile
     static constexpr int NT = NT_;          // query tiles per unit
+    static constexpr int NSM = NSM_;        // softmax warpgroups: 1 (all tiles) or NT (one each)
     static constexpr bool Q_TMEM = Q_TMEM_; // Q as the TMEM A operand (else from shared memory)
     static constexpr int NK = NK_;          // K slots
     static constexpr int NV = NV_;          // V slots
@@ -92,12 +96,13 @@ struct AttnTraits {
     static constexpr uint32_t K_OFF = Q_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NK * K_TILE_BYTES;
     static constexpr uint32_t BARS_OFF = V_OFF + NV * V_TILE_BYTES;
-    static constexpr int NBAR = 2 * NK + 2 * NV + 11;
+    static constexpr int NBAR = 2 * NK + 2 * NV + 8 + 3 * NT;
     static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static constexpr int NUM_THREADS = 128 * NT + 64;
-    static constexpr int MMA_WARP = 4 * NT;
-    static constexpr int TMA_WARP = 4 * NT + 1;
+    static_assert(NSM == 1 || NSM == NT, "");
+    static constexpr int NUM_THREADS = 128 * NSM + 64;
+    static constexpr int MMA_WARP = 4 * NSM;
+    static constexpr int TMA_WARP = 4 * NSM + 1;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BN, false, false);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, DV, false, true);
 };
@@ -184,10 +189,11 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     const uint32_t bar_pv_done = bar(B0 + 4);
     const uint32_t bar_q_full = bar(B0 + 5);
     const uint32_t bar_q_empty = bar(B0 + 6);
-    const uint32_t bar_q_tmem = bar(B0 + 7);
-    const uint32_t bar_o_full = bar(B0 + 8);
-    const uint32_t bar_o_free = bar(B0 + 9);
-    const uint32_t bar_mma_done = bar(B0 + 10);
+    const uint32_t bar_mma_done = bar(B0 + 7);
+    // per query tile: its Q is in TMEM / its O is final / its O has been read out
+    auto bar_q_tmem = [&](int t) { return bar(B0 + 8 + t); };
+    auto bar_o_full = [&](int t) { return bar(B0 + 8 + NT + t); };
+    auto bar_o_free = [&](int t) { return bar(B0 + 8 + 2 * NT + t); };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -207,11 +213,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         }
         mbar_init(bar_pv_done, 1);
         mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : 1);  // softmax copy-out / last Q K^T
-        mbar_init(bar_q_tmem, 128 * NT);
-        mbar_init(bar_o_full, 1);
-        mbar_init(bar_o_free, 128 * NT);
+        mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : 1);  // per-tile copy-out / last Q K^T
         mbar_init(bar_mma_done, 1);
+        for (int t = 0; t < NT; ++t) {
+            mbar_init(bar_q_tmem(t), 128);
+            mbar_init(bar_o_full(t), 1);
+            mbar_init(bar_o_free(t), 128);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -341,6 +349,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int kslot = 0, vslot = 0;
             // Q K^T of item gi = (block j, tile tt) of the current unit.
             auto qk = [&](int j, int tt, bool last_item) {
+                if (T::Q_TMEM && j == 0) {  // this tile's Q of the new unit must be in TMEM
+                    if (!mbar_wait(bar_q_tmem(tt), (uint32_t)(units & 1), wc, kErrTimeout)) {
+                        ok = false;
+                        return;
+                    }
+                    tc_fence_after_sync();
+                }
                 if (tt == 0) {
                     kslot = kq % NK;
                     const uint32_t phase = (uint32_t)(kq / NK) & 1u;
@@ -372,13 +387,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
             };
             // P V of item g = (block j, tile tt) of busy unit number uidx.
-            auto pv = [&](int64_t g, int j, int tt, bool last_item, int uidx) {
+            auto pv = [&](int64_t g, int j, int tt, bool last_block, int uidx) {
                 if (!mbar_wait(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
-                if (j == 0 && tt == 0 && uidx > 0 &&
-                    !mbar_wait(bar_o_free, (uint32_t)(uidx - 1) & 1u, wc, kErrTimeout)) {
+                if (j == 0 && uidx > 0 &&
+                    !mbar_wait(bar_o_free(tt), (uint32_t)(uidx - 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
@@ -404,7 +419,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 if (NT == 1) tc_commit(bar_pv_done);
                 if (tt == NT - 1) tc_commit(bar_vempty(vslot));
-                if (last_item) tc_commit(bar_o_full);
+                if (last_block) tc_commit(bar_o_full(tt));
             };
             // The P V of each item is issued after the next item's Q K^T (also across units), so
             // the tensor core computes the next S while the softmax works on this one.
@@ -414,12 +429,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
                 const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
                 if (t.n_blocks == 0) continue;
-                const uint32_t qbar = T::Q_TMEM ? bar_q_tmem : bar_q_full;
-                if (!mbar_wait(qbar, (uint32_t)(units & 1), wc, kErrTimeout)) {
-                    ok = false;
-                    break;
+                if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
+                    if (!mbar_wait(bar_q_full, (uint32_t)(units & 1), wc, kErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
                 }
-                tc_fence_after_sync();
                 for (int j = 0; j < t.n_blocks && ok; ++j) {
                     for (int tt = 0; tt < NT && ok; ++tt) {
                         const bool last_item = (j == t.n_blocks - 1) && (tt == NT - 1);
@@ -430,7 +446,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         pend_g = gi;
                         pend_j = j;
                         pend_tt = tt;
-                        pend_last = last_item;
+                        pend_last = (j == t.n_blocks - 1);
                         pend_u = units;
                         ++gi;
                     }
@@ -442,7 +458,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
     } else {
-        // ---------------------- softmax + epilogue warpgroups (warps 0 .. 4*NT-1) ----------------------
+        if constexpr (T::NSM == 2) {
+        // ------------- two softmax + epilogue warpgroups, one per query tile (warps 0-7) -------------
         const int wg = warp >> 2;           // the query tile this warpgroup owns
         const int row = threadIdx.x & 127;  // TMEM lane
         const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -472,7 +489,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             }
             tmem_wait_st();
             tc_fence_before_sync();
-            mbar_arrive(bar_q_tmem);
+            mbar_arrive(bar_q_tmem(wg));
             mbar_arrive(bar_q_empty);
             return true;
         };
@@ -480,7 +497,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         // Epilogue of busy unit number uidx: wait for its last P V, read this row of O (tile wg)
         // from TMEM (then free the accumulators for the next unit), write O / l and the LSE.
         auto epilogue = [&](const UnitInfo& t, float m_ref, float l, int uidx) -> bool {
-            if (!__all_sync(FULL, mbar_wait(bar_o_full, (uint32_t)(uidx & 1), wc, kErrTimeout)))
+            if (!__all_sync(FULL,
+                            mbar_wait(bar_o_full(wg), (uint32_t)(uidx & 1), wc, kErrTimeout)))
                 return false;
             tc_fence_after_sync();
             const int64_t i = t.q0 + wg * 128 + row;
@@ -496,7 +514,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 if (c == T::DV / 32 - 1) {
                     // this tile's O has been read out: the next unit's P V may overwrite it
                     tc_fence_before_sync();
-                    mbar_arrive(bar_o_free);
+                    mbar_arrive(bar_o_free(wg));
                 }
                 uint32_t w[16];
 #pragma unroll
@@ -744,6 +762,247 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             ++units;
         }
         if (ok && pend) ok = epilogue(pend_t, pend_m, pend_l, pend_idx);
+        } else {
+        // --------------------------- softmax + epilogue warps 0-3 ---------------------------
+        const int row = threadIdx.x;  // TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        int64_t gi = 0;  // global item counter (score buffer gi % 2, phase (gi / 2) % 2)
+        int units = 0;   // busy units whose items are done
+
+        // Staged Q of busy unit number qidx, tile tt (128-byte swizzled rows, as TMA wrote them)
+        // -> this row's TMEM columns of that tile; then tell the MMA warp and the producer.
+        auto copy_q = [&](int qidx, int tt) -> bool {
+            if (!__all_sync(FULL, mbar_wait(bar_q_full, (uint32_t)(qidx & 1), wc, kErrTimeout)))
+                return false;
+#pragma unroll
+            for (int ch = 0; ch < T::QCH; ++ch) {
+                uint32_t r[32];
+                const uint8_t* rowp = smem + tt * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(rowp + ((c ^ (row & 7)) << 4));
+                    r[4 * c + 0] = x.x;
+                    r[4 * c + 1] = x.y;
+                    r[4 * c + 2] = x.z;
+                    r[4 * c + 3] = x.w;
+                }
+                tmem_st32(tl + T::Q_COL0 + tt * (T::DQK / 2) + ch * 32, r);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(bar_q_tmem(tt));
+            mbar_arrive(bar_q_empty);
+            return true;
+        };
+
+        // Epilogue of tile tt of busy unit number uidx: wait for that tile's last P V, read this
+        // row of its O from TMEM (then free the accumulator), write O / l in bf16 and the LSE.
+        auto epilogue = [&](const UnitInfo& t, int tt, float m_ref, float l, int uidx) -> bool {
+            if (!__all_sync(FULL,
+                            mbar_wait(bar_o_full(tt), (uint32_t)(uidx & 1), wc, kErrTimeout)))
+                return false;
+            tc_fence_after_sync();
+            const int64_t i = t.q0 + tt * 128 + row;
+            const bool row_valid = i < p.sq;
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+            for (int c = 0; c < T::DV / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                tmem_wait_ld();
+                if (c == T::DV / 32 - 1) {
+                    // this tile's O has been read out: the next unit's P V may overwrite it
+                    tc_fence_before_sync();
+                    mbar_arrive(bar_o_free(tt));
+                }
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                       __uint_as_float(r[2 * e + 1]) * inv_l);
+                if (row_valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        dst[c * 4 + q4] =
+                            make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                }
+            }
+            if (row_valid && p.lse)
+                p.lse[(t.bi * p.hq + t.h) * p.sq + i] =
+                    l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            return true;
+        };
+
+        bool pend = false;  // a finished unit whose epilogues have not run yet
+        UnitInfo pend_t{};
+        float pend_m[NT], pend_l[NT];
+#pragma unroll
+        for (int tt = 0; tt < NT; ++tt) pend_m[tt] = pend_l[tt] = 0.f;
+        int pend_idx = 0;
+        if (T::Q_TMEM && busy_from(u0) >= 0)
+            for (int tt = 0; tt < NT && ok; ++tt) ok = copy_q(0, tt);
+        for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
+            const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+            if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt) {
+                    const int64_t i = t.q0 + tt * 128 + row;
+                    if (i < p.sq) {
+                        uint4* dst = reinterpret_cast<uint4*>(
+                            p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
+#pragma unroll 1
+                        for (int c = 0; c < T::DV / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+                        if (p.lse) p.lse[(t.bi * p.hq + t.h) * p.sq + i] = -INFINITY;
+                    }
+                }
+                continue;
+            }
+            const int64_t un = busy_from(u + ustep);
+            int64_t lim[NT];  // last allowed key of this thread's row in each tile
+            float m_ref[NT];  // exponent reference (log2 units); moves lazily
+            float l[NT];      // sum of exp2(x - m_ref) over the keys seen so far
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+                const int64_t i = t.q0 + tt * 128 + row;
+                const int64_t lim_row = CAUSAL ? i + p.sk - p.sq : p.sk - 1;
+                lim[tt] = lim_row < p.sk - 1 ? lim_row : p.sk - 1;
+                m_ref[tt] = -INFINITY;
+                l[tt] = 0.f;
+            }
+
+            for (int j = 0; j < t.n_blocks && ok; ++j) {
+#pragma unroll
+                for (int tt = 0; tt < NT; ++tt, ++gi) {
+                    const int sb = (int)(gi & 1);
+                    const uint32_t s_col = tl + sb * BN;
+                    ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(gi >> 1) & 1u, wc,
+                                                    kErrTimeout));
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    if (T::Q_TMEM && j == t.n_blocks - 1 && un >= 0) {
+                        // This tile's last Q K^T of the unit is complete (its S has landed), so
+                        // its Q columns can take the next unit's Q now, ahead of this softmax.
+                        ok = copy_q(units + 1, tt);
+                        if (!ok) break;
+                    }
+                    uint32_t sr[BN];
+#pragma unroll
+                    for (int c = 0; c < BN / 32; ++c)
+                        tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+                    tmem_wait_ld();
+
+                    const bool masked_block = j >= t.mask_from;
+                    // keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all)
+                    int64_t rel64 = lim[tt] - (int64_t)j * BN;
+                    rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
+                    const int rel = (int)rel64;
+                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    if (masked_block) {
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            mx[c & 3] = fmaxf(mx[c & 3],
+                                              c <= rel ? __uint_as_float(sr[c]) : -INFINITY);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < BN; ++c)
+                            mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
+                    }
+                    const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
+                    const float m_new = fmaxf(m_ref[tt], m_blk);
+                    // Lazy rescale: keep the old reference while the running max stays within
+                    // 2^8 of it; the final O / l uses the same reference, so the result is exact.
+                    const bool need = m_new > m_ref[tt] + 8.0f;
+                    float alpha = 1.f;
+                    if (need) {
+                        alpha = ex2(m_ref[tt] - m_new);
+                        m_ref[tt] = m_new;
+                        l[tt] *= alpha;
+                    }
+                    if (j > 0 && __any_sync(FULL, need)) {
+                        // O holds blocks < j of this tile: scale it in place once its last P V
+                        // is complete. With two tiles that P V is item gi-2, issued before this
+                        // item's Q K^T, so it is complete now that S has landed. With one tile it
+                        // is item gi-1: wait for it (bar_pv_done is then in phase gi-1 or gi, so
+                        // the parity test on phase gi-1 is unambiguous).
+                        if (NT == 1) {
+                            ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(gi - 1) & 1u,
+                                                            wc, kErrTimeout));
+                            if (!ok) break;
+                            tc_fence_after_sync();
+                        }
+#pragma unroll 1
+                        for (int c = 0; c < T::DV / 32; ++c) {
+                            uint32_t r[32];
+                            tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                            tmem_st32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                        }
+                    }
+                    const float neg_m = (m_ref[tt] == -INFINITY) ? 0.f : -m_ref[tt];
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int h2 = 0; h2 < BN / 64; ++h2) {
+                        uint32_t pk[32];
+                        if (masked_block) {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const int e = h2 * 64 + 2 * c;
+                                float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, neg_m));
+                                float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, neg_m));
+                                p0 = (e <= rel) ? p0 : 0.f;  // masked keys: exactly 0
+                                p1 = (e + 1 <= rel) ? p1 : 0.f;
+                                acc[(2 * c) & 3] += p0;
+                                acc[(2 * c + 1) & 3] += p1;
+                                pk[c] = pack_bf16x2(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 32; ++c) {
+                                const int e = h2 * 64 + 2 * c;
+                                const float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, neg_m));
+                                const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, neg_m));
+                                acc[(2 * c) & 3] += p0;
+                                acc[(2 * c + 1) & 3] += p1;
+                                pk[c] = pack_bf16x2(p0, p1);
+                            }
+                        }
+                        tmem_st32(s_col + h2 * 32, pk);
+                    }
+                    l[tt] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    mbar_arrive(bar_p_full(sb));
+                    if (j == 0 && pend) {
+                        // Tile tt of the previous unit, now that its successor's first P is out.
+                        ok = epilogue(pend_t, tt, pend_m[tt], pend_l[tt], pend_idx);
+                        if (tt == NT - 1) pend = false;
+                        if (!ok) break;
+                    }
+                }
+            }
+            if (!ok) break;
+            pend = true;
+            pend_t = t;
+#pragma unroll
+            for (int tt = 0; tt < NT; ++tt) {
+                pend_m[tt] = m_ref[tt];
+                pend_l[tt] = l[tt];
+            }
+            pend_idx = units;
+            ++units;
+        }
+        if (ok && pend)
+            for (int tt = 0; tt < NT && ok; ++tt)
+                ok = epilogue(pend_t, tt, pend_m[tt], pend_l[tt], pend_idx);
+        }
     }
 
     // ---- teardown: every tcgen05 access is complete (MMAs drained, loads waited) ----
