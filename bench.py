@@ -131,56 +131,71 @@ def cpu_baseline(c, inputs, seconds):
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event (throttle) reasons during the timed region.
 
-    def __init__(self, gpu_index):
+    Polls NVML every few milliseconds from a thread (the timed regions are short); reports None
+    when NVML is not available."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, gpu_index, period_s=0.004):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = os.path.join("/tmp", f"b200attn_clocks_{os.getpid()}.csv")
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._thread = None
+        self._stop = False
+
+    def _poll(self, nvml, h):
+        while not self._stop:
+            try:
+                self.samples.append(nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM))
+                bits = nvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:  # pragma: no cover
+                pass
+            time.sleep(self.period)
 
     def start(self):
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+            import pynvml as nvml
+            import threading
+            nvml.nvmlInit()
+            h = nvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = nvml.nvmlDeviceGetMaxClockInfo(h, nvml.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._poll, args=(nvml, h), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
 
     def stop(self):
-        if self.proc is None:
+        if self._thread is None:
             return None
-        time.sleep(0.3)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        sms, maxes, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm, mx = float(parts[1]), float(parts[2])
-            except ValueError:
-                continue
-            sms.append(sm)
-            maxes.append(mx)
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        os.unlink(self.path)
-        if not sms:
+        self._stop = True
+        self._thread.join(timeout=5)
+        if not self.samples:
             return None
-        load = [s for s in sms if s > 0.5 * max(sms)] or sms
-        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(maxes),
-                "reasons": sorted(reasons), "samples": len(sms)}
+        load = [x for x in self.samples if x > 0.5 * max(self.samples)] or self.samples
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "NVML, polled every 4 ms during the timed region"}
+
+
+def attn_source_hash():
+    """Hash of the attention kernel's sources (profiled traffic is valid only for these)."""
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "head_attention_forward_flash_b200", "csrc")
+    for f in ("attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------------------------
@@ -254,7 +269,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     if clocks:
         clocks.start()
-        time.sleep(0.4)
+        time.sleep(0.05)
     for s in range(args.steps):
         flush.zero_()
         starts[s].record(stream)
@@ -264,6 +279,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop() if clocks else None
+    if clk is not None and "reasons" in clk and clk["sm_max_mhz"] is None:
+        clk["sm_max_mhz"] = clk["sm_mhz"]
     step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
     attn_ms = [a_starts[s].elapsed_time(a_ends[s]) for s in range(args.steps)]
     status = b2.attn_debug_status()
@@ -281,7 +298,9 @@ def run_gpu(args):
     traffic = None
     try:
         with open(PROFILED_TRAFFIC_FILE) as f:
-            traffic = json.load(f).get(c["workload"])
+            prof = json.load(f)
+        if prof.get("attn_source_hash") == attn_source_hash():
+            traffic = prof.get(c["workload"])
     except (OSError, ValueError):
         traffic = None
     srt = sorted(attn_ms)

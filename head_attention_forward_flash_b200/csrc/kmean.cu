@@ -4,7 +4,7 @@
 // are one contiguous row, so the mean over the key axis is a column sum of a [sk, hk*d] matrix
 // per batch: fully coalesced 16-byte loads, one 8-channel group per thread, no shuffles needed.
 // Kernel 1 sums a chunk of key rows per CTA into fp32 partials; kernel 2 folds the partials of
-// each channel in chunk order, so the result is bit-identical from run to run (the two
+// each channel in a fixed order, so the result is bit-identical from run to run (the two
 // deterministic kernels behind one host call of "[HIP] Mha v4: run the K-smoothing gate as one
 // HIP call", Summary and commit message).
 #include <cuda_bf16.h>
@@ -62,19 +62,31 @@ __global__ void __launch_bounds__(kThreads)
     dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
 }
 
-// mean[bi][col] = (sum over chunks, in chunk order, of partial[bi][chunk][col]) / sk
+// mean[bi][col] = (sum of partial[bi][chunk][col] over the chunks) / sk, 32 columns per CTA:
+// warp w sums chunks w, w+8, w+16, ... in order, then the eight warp sums are added in warp order,
+// so the result does not depend on timing.
 __global__ void __launch_bounds__(kThreads)
-    k_mean_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t b,
-                int64_t cols, int nchunks, float sk_f)
+    k_mean_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t cols,
+                int nchunks, float sk_f)
 {
-    const int64_t t = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (t >= b * cols) return;
-    const int64_t bi = t / cols;
-    const int64_t col = t - bi * cols;
-    const float* src = partial + bi * nchunks * cols + col;
+    __shared__ float red[kThreads / 32][32];
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const int64_t col = (int64_t)blockIdx.x * 32 + lane;
+    const int64_t bi = blockIdx.y;
     float sum = 0.f;
-    for (int c = 0; c < nchunks; ++c) sum += src[(int64_t)c * cols];
-    mean[t] = __fdiv_rn(sum, sk_f);
+    if (col < cols) {
+        const float* src = partial + bi * nchunks * cols + col;
+        for (int c = w; c < nchunks; c += kThreads / 32) sum += src[(int64_t)c * cols];
+    }
+    red[w][lane] = sum;
+    __syncthreads();
+    if (w == 0 && col < cols) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < kThreads / 32; ++q) t += red[q][lane];
+        mean[bi * cols + col] = __fdiv_rn(t, sk_f);
+    }
 }
 
 // k_out = bf16_rne(float(K) - mean[bi, col]), 8 channels (16 bytes) per thread per step.
@@ -190,9 +202,8 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
     dim3 g1((unsigned)col_ctas, (unsigned)nchunks, (unsigned)b);
     k_mean_partial<<<g1, kThreads, 0, st>>>(static_cast<const uint4*>(k), partial, sk, cols,
                                             rows_per_chunk, (int)nchunks);
-    const int64_t n = b * cols;
-    k_mean_fold<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, st>>>(
-        partial, mean, b, cols, (int)nchunks, (float)sk);
+    k_mean_fold<<<dim3((unsigned)((cols + 31) / 32), (unsigned)b), kThreads, 0, st>>>(
+        partial, mean, cols, (int)nchunks, (float)sk);
     const bool launched = cudaGetLastError() == cudaSuccess;
     if (cudaFreeAsync(partial, st) != cudaSuccess) {
         cudaGetLastError();
@@ -250,9 +261,8 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     dim3 g1((unsigned)col_ctas, (unsigned)nchunks, (unsigned)b);
     k_mean_partial<<<g1, kThreads, 0, st>>>(static_cast<const uint4*>(k), partial, sk, cols,
                                             rows_per_chunk, (int)nchunks);
-    const int64_t n = b * cols;
-    k_mean_fold<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, st>>>(
-        partial, mean, b, cols, (int)nchunks, (float)sk);
+    k_mean_fold<<<dim3((unsigned)((cols + 31) / 32), (unsigned)b), kThreads, 0, st>>>(
+        partial, mean, cols, (int)nchunks, (float)sk);
     return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
