@@ -19,7 +19,8 @@
 // Roles (NSM softmax warpgroups + 2 warps): NSM = 1 (192 threads) or NSM = NT = 2 (320 threads).
 //   softmax + epilogue warps: thread r owns row r (= TMEM lane r) of a query tile. Turns each
 //              score block S into P (online softmax: exp2 with the scale folded into one FMA,
-//              lazy rescaling of O), and writes each tile's finished O rows (divided by the row
+//              lazy rescaling of O; the FMA and the row-sum adds run as packed fp32x2
+//              instructions, two scores each), and writes each tile's finished O rows (divided by the row
 //              sums) and LSE right after handing over that tile's first P of the next unit. When
 //              Q lives in TMEM they also copy each tile's Q from the shared-memory staging buffer
 //              into TMEM once the tile's last Q K^T of the current unit has landed.
@@ -537,8 +538,10 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         // exp2(s * sl2 - m) for two scores, and their bf16 pair; masked keys give exactly 0.
         auto p_pair = [&](uint32_t s0, uint32_t s1, float neg_m, bool v0, bool v1, float& p0,
                           float& p1) -> uint32_t {
-            p0 = ex2(fmaf(__uint_as_float(s0), sl2, neg_m));
-            p1 = ex2(fmaf(__uint_as_float(s1), sl2, neg_m));
+            float x0, x1;
+            fma2(__uint_as_float(s0), __uint_as_float(s1), sl2, neg_m, x0, x1);
+            p0 = ex2(x0);
+            p1 = ex2(x1);
             p0 = v0 ? p0 : 0.f;
             p1 = v1 ? p1 : 0.f;
             return pack_bf16x2(p0, p1);
@@ -725,16 +728,14 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                                 const int e = c * 32 + 2 * e2;
                                 float p0, p1;
                                 pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, e <= rel, e + 1 <= rel, p0, p1);
-                                acc[(2 * e2) & 3] += p0;
-                                acc[(2 * e2 + 1) & 3] += p1;
+                                add2(acc[(2 * e2) & 3], acc[(2 * e2 + 1) & 3], p0, p1);
                             }
                         } else {
 #pragma unroll
                             for (int e2 = 0; e2 < 16; ++e2) {
                                 float p0, p1;
                                 pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, true, true, p0, p1);
-                                acc[(2 * e2) & 3] += p0;
-                                acc[(2 * e2 + 1) & 3] += p1;
+                                add2(acc[(2 * e2) & 3], acc[(2 * e2 + 1) & 3], p0, p1);
                             }
                         }
                         // P chunk c (16 columns of bf16 pairs) overwrites S columns already read
@@ -955,22 +956,24 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll
                             for (int c = 0; c < 32; ++c) {
                                 const int e = h2 * 64 + 2 * c;
-                                float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, neg_m));
-                                float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, neg_m));
+                                float x0, x1;
+                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, neg_m,
+                                     x0, x1);
+                                float p0 = ex2(x0), p1 = ex2(x1);
                                 p0 = (e <= rel) ? p0 : 0.f;  // masked keys: exactly 0
                                 p1 = (e + 1 <= rel) ? p1 : 0.f;
-                                acc[(2 * c) & 3] += p0;
-                                acc[(2 * c + 1) & 3] += p1;
+                                add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
                                 pk[c] = pack_bf16x2(p0, p1);
                             }
                         } else {
 #pragma unroll
                             for (int c = 0; c < 32; ++c) {
                                 const int e = h2 * 64 + 2 * c;
-                                const float p0 = ex2(fmaf(__uint_as_float(sr[e]), sl2, neg_m));
-                                const float p1 = ex2(fmaf(__uint_as_float(sr[e + 1]), sl2, neg_m));
-                                acc[(2 * c) & 3] += p0;
-                                acc[(2 * c + 1) & 3] += p1;
+                                float x0, x1;
+                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, neg_m,
+                                     x0, x1);
+                                const float p0 = ex2(x0), p1 = ex2(x1);
+                                add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
                                 pk[c] = pack_bf16x2(p0, p1);
                             }
                         }
