@@ -112,12 +112,27 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
             cudaGetLastError();
             return B200ATTN_ERR_CUDA;
         }
+        // With two softmax warpgroups the kernel moves registers between warpgroups; the
+        // softmax warps' raise is granted only from what the block was launched with, so a
+        // build launched with fewer registers per thread would stall for good: refuse it.
+        if (T::NSM == 2) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+                cudaGetLastError();
+                return B200ATTN_ERR_CUDA;
+            }
+            if ((int64_t)fa.numRegs * T::NUM_THREADS <
+                (int64_t)2 * 128 * T::SOFTMAX_REGS + 128 * T::AUX_REGS)
+                return B200ATTN_ERR_CUDA;
+        }
         attr_done[dev] = true;
     }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     int rc = encode_bshd(&tq, q, b, sq, hq, T::DQK, T::BM);
     if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, b, sk, hk, T::DQK, T::BN);
     if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, b, sk, hk, T::DV, T::BN);
+    // O is stored per warp: boxes of 32 rows (only used when the kernel stages O for TMA)
+    if (rc == B200ATTN_OK) rc = encode_bshd(&to, out, b, sq, hq, T::DV, 32);
     if (rc != B200ATTN_OK) return rc;
     int* status = status_word();
     const int n_sm = sm_count();
@@ -133,25 +148,34 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.sk = sk;
     p.group = hq / hk;
     p.n_qu = (sq + T::NT * T::BM - 1) / (T::NT * T::BM);
-    p.n_units = b * hq * p.n_qu;
+    p.n_units = b * hq * p.n_qu;  // below 2^31 (checked by attn_fwd)
+    p.div_nqu = make_fastdiv((uint32_t)p.n_qu);
+    p.div_hq = make_fastdiv((uint32_t)hq);
+    p.div_group = make_fastdiv((uint32_t)p.group);
     // The MMA applies the sign of the scale (negate-A bit of the instruction descriptor), so
-    // the softmax only ever sees a non-negative scale.
-    p.scale_log2 = (float)(std::fabs((double)scale) * 1.4426950408889634);
+    // the softmax only ever sees a non-negative factor. It is kept at 2^-100 or more, so that a
+    // masked score of -inf always maps to exp2(-inf) = 0. For |scale| below that (scale 0
+    // included) and scores below 2^40 in magnitude, every exp2 argument is then below 2^-60,
+    // so each p rounds to exactly 1 in fp32 -- the same weights the unclamped scale gives.
+    const double sl2 = std::fabs((double)scale) * 1.4426950408889634;
+    p.scale_log2 = (float)(sl2 > 0x1p-100 ? sl2 : 0x1p-100);
     p.idesc_qk = T::IDESC_QK | (scale < 0.f ? (1u << 13) : 0u);
     p.status = status;
     p.timeout_ns = 4000000000ull;  // 4 s: far above any legitimate wait
 
     const int64_t grid = p.n_units < n_sm ? p.n_units : n_sm;  // persistent: one CTA per SM
-    kern<<<(unsigned)grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    kern<<<(unsigned)grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
     if (cudaGetLastError() != cudaSuccess) return B200ATTN_ERR_CUDA;
     return B200ATTN_OK;
 }
 
 // Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, softmax
-// warpgroups, Q in TMEM, K slots, V slots>. Tensor memory holds two score buffers, one O per query
-// tile and (when it fits) each tile's Q; shared memory holds the Q staging buffer and the K / V
-// rings. The (tiles, warpgroups) choice per head dim is the measured fastest on B200.
-using T64 = AttnTraits<64, 64, 128, 1, 1, true, 6, 6>;       // smem 16 + 96 + 96 KB
+// warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe>. Tensor
+// memory holds two score buffers, one O per query tile and (when it fits) each tile's Q; shared
+// memory holds the Q staging buffer and the K / V rings. The (tiles, warpgroups) choice per head
+// dim is the measured fastest on B200. d64 is bound by the exp2 rate, so 3 of every 8 score
+// pairs take the FMA-pipe exp2 there.
+using T64 = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 KB
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2>;   // smem 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1>;   // smem 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
@@ -204,6 +228,10 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* out, 
         return B200ATTN_ERR_ALIGN;
     if (!tma_extent_ok(b, sq, hq, dqk) ||
         (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv))))
+        return B200ATTN_ERR_RANGE;
+    // Work units (b * hq * query tiles) are numbered in 31 bits.
+    int64_t n_units;
+    if (!numel({b, hq, (sq + 127) / 128}, &n_units) || n_units >= ((int64_t)1 << 31))
         return B200ATTN_ERR_RANGE;
     int rc = check_arch();
     if (rc != B200ATTN_OK) return rc;

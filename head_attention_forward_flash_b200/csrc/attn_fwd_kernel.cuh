@@ -60,14 +60,16 @@ struct AttnParams {
     int64_t b, hq, hk, sq, sk;
     int64_t group;    // hq / hk
     int64_t n_qu;     // query units per (batch, head): ceil(sq / (NT * 128))
-    int64_t n_units;  // b * hq * n_qu
+    int64_t n_units;  // b * hq * n_qu (below 2^31)
+    FastDiv div_nqu, div_hq, div_group;  // by n_qu, hq and group
     float scale_log2; // |scale| * log2(e); the sign of scale is applied by the MMA (negate A)
     uint32_t idesc_qk;
     int* status;      // device error word
     unsigned long long timeout_ns;
 };
 
-template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_>
+template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_,
+          uint32_t EXP_FMA_PAIRS_ = 0>
 struct AttnTraits {
     static constexpr int DQK = DQK_;
     static constexpr int DV = DV_;
@@ -93,24 +95,48 @@ struct AttnTraits {
     static_assert(2 * BN + NT * DV + (Q_TMEM ? NT * DQK / 2 : 0) <= 512, "tensor memory budget");
     static_assert(DQK % 64 == 0 && DV % 64 == 0 && BN % 64 == 0 && BN <= 256 && DV <= 256, "");
     static_assert(NT == 1 || NT == 2, "");
-    // shared memory: [Q staging][K slots][V slots][barriers][TMEM base, abort flag]
+    // shared memory: [Q staging][K slots][V slots][O staging, if used][barriers][TMEM base,
+    // abort flag]
     static constexpr uint32_t K_OFF = Q_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NK * K_TILE_BYTES;
-    static constexpr uint32_t BARS_OFF = V_OFF + NV * V_TILE_BYTES;
+    static constexpr uint32_t O_OFF = V_OFF + NV * V_TILE_BYTES;
     static constexpr int NBAR = 2 * NK + 2 * NV + 8 + 3 * NT;
+    // The epilogue writes O through a shared-memory tile and TMA stores (one per warp and
+    // 64-column box: slab o_slab(tile, box, warp % 4), 32 rows x 128 bytes) when the tiles fit
+    // next to the rings; otherwise each thread stores its own row.
+    static constexpr uint32_t O_STAGE_BYTES = NT * BM * DV * 2;
+    static constexpr bool O_TMA = 1024 + O_OFF + O_STAGE_BYTES + NBAR * 8 + 16 <= 232448;
+    static constexpr uint32_t o_slab(int tt, int bx, int w4)
+    {
+        return (uint32_t)(((tt * (DV / 64) + bx) * 4 + w4) * 4096);
+    }
+    static constexpr uint32_t BARS_OFF = O_OFF + (O_TMA ? O_STAGE_BYTES : 0);
     static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(NSM == 1 || NSM == NT, "");
-    static constexpr int NUM_THREADS = 128 * NSM + 64;
+    // Threads: NSM softmax warpgroups, then the MMA warp and the TMA warp. With two softmax
+    // warpgroups the block is three full warpgroups (two warps idle) so that registers can
+    // move between them: at launch every thread has LAUNCH_REGS (the cap for 384 threads);
+    // the third warpgroup drops to AUX_REGS and the softmax warpgroups rise to SOFTMAX_REGS,
+    // which keeps the block's total unchanged (a larger total would never be granted).
+    static constexpr int NUM_THREADS = NSM == 1 ? 192 : 384;
     static constexpr int MMA_WARP = 4 * NSM;
     static constexpr int TMA_WARP = 4 * NSM + 1;
+    static constexpr int LAUNCH_REGS = 168;
+    static constexpr int SOFTMAX_REGS = 224;
+    static constexpr int AUX_REGS = 56;
+    static_assert(NSM == 1 || 2 * 128 * SOFTMAX_REGS + 128 * AUX_REGS <= NUM_THREADS * LAUNCH_REGS,
+                  "register split exceeds the launch allocation");
+    // Score pairs whose exp2 runs on the FMA pipe (exp2_fma_pair) rather than the MUFU unit: bit
+    // k set = pairs with index k mod 8 in each row, in the one-warpgroup softmax.
+    static constexpr uint32_t EXP_FMA_PAIRS = EXP_FMA_PAIRS_;
     static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BN, false, false);
     static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, DV, false, true);
 };
 
 // Wait bounded only by time (used to drain in-flight copies / MMAs before exit, also after an
 // abort, so it ignores the abort flag).
-__device__ __noinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
                                              unsigned long long timeout_ns, int* status)
 {
     const uint64_t t0 = global_timer_ns();
@@ -133,11 +159,14 @@ template <int BN, int NT, bool CAUSAL>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
 {
     UnitInfo t;
-    const int64_t bh = u / p.n_qu;
-    const int64_t qu = p.n_qu - 1 - (u - bh * p.n_qu);  // within a head: most keys first
-    t.bi = bh / p.hq;
-    t.h = bh - t.bi * p.hq;
-    t.g = t.h / p.group;
+    const uint32_t uu = (uint32_t)u;
+    const uint32_t bh = fast_div(uu, p.div_nqu);
+    const uint32_t qu = p.div_nqu.d - 1 - (uu - bh * p.div_nqu.d);  // within a head: most keys first
+    const uint32_t bi = fast_div(bh, p.div_hq);
+    const uint32_t h = bh - bi * p.div_hq.d;
+    t.bi = bi;
+    t.h = h;
+    t.g = fast_div(h, p.div_group);
     t.q0 = qu * (NT * 128);
     const int64_t n_kv = (p.sk + BN - 1) / BN;
     if (CAUSAL) {
@@ -161,7 +190,8 @@ template <class T, bool CAUSAL>
 __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
-                    const __grid_constant__ CUtensorMap tmap_v, const AttnParams p)
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_o, const AttnParams p)
 {
     constexpr int BN = T::BN;
     constexpr int NT = T::NT;
@@ -248,6 +278,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         return -1;
     };
 
+    if constexpr (T::NSM == 2) {
+        if (warp >= T::MMA_WARP) setmaxnreg_dec<T::AUX_REGS>();  // registers to the softmax
+    }
     if (warp == T::TMA_WARP) {
         // ------------------------------ TMA producer ------------------------------
         // Walks the MMA warp's item sequence and issues each load at the point the MMA warp
@@ -458,318 +491,21 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             tc_commit(bar_mma_done);  // drain every MMA this thread issued before teardown
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
-    } else {
-        if constexpr (T::NSM == 2) {
-        // ------------- two softmax + epilogue warpgroups, one per query tile (warps 0-7) -------------
-        const int wg = warp >> 2;           // the query tile this warpgroup owns
-        const int row = threadIdx.x & 127;  // TMEM lane
-        const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    } else if (warp < T::MMA_WARP) {
+        // ---------------- softmax + epilogue warpgroups (warps 0 .. 4*NSM-1) ----------------
+        // NSM = 1: the warpgroup takes every query tile's items in order. NSM = 2: warpgroup w
+        // takes the items of query tile w. Either way each thread keeps its whole score row of
+        // the current item in registers (one TMEM read, a single pass).
+        if constexpr (T::NSM == 2) setmaxnreg_inc<T::SOFTMAX_REGS>();
+        constexpr int NTW = T::NSM == 1 ? NT : 1;  // query tiles this warpgroup handles
+        const int wg = warp >> 2;
+        const int w4 = warp & 3;                  // TMEM lanes 32*w4 .. 32*w4+31
+        const int row = threadIdx.x & 127;        // TMEM lane = row of the query tile
+        const uint32_t tl = tmem + ((uint32_t)(w4 * 32) << 16);
         const float sl2 = p.scale_log2;
+        auto tile_of = [&](int k) { return T::NSM == 1 ? k : wg; };
         bool ok = true;
-        int64_t wi = 0;  // items of this warpgroup's tile processed so far
-        int units = 0;   // busy units whose items are done
-
-        // Staged Q of busy unit number qidx, tile wg (128-byte swizzled rows, as TMA wrote them)
-        // -> this row's TMEM columns; then release the staging buffer and tell the MMA warp.
-        auto copy_q = [&](int qidx) -> bool {
-            if (!__all_sync(FULL, mbar_wait(bar_q_full, (uint32_t)(qidx & 1), wc, kErrTimeout)))
-                return false;
-#pragma unroll
-            for (int ch = 0; ch < T::QCH; ++ch) {
-                uint32_t r[32];
-                const uint8_t* rowp = smem + wg * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES + row * 128;
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 x = *reinterpret_cast<const uint4*>(rowp + ((c ^ (row & 7)) << 4));
-                    r[4 * c + 0] = x.x;
-                    r[4 * c + 1] = x.y;
-                    r[4 * c + 2] = x.z;
-                    r[4 * c + 3] = x.w;
-                }
-                tmem_st32(tl + T::Q_COL0 + wg * (T::DQK / 2) + ch * 32, r);
-            }
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(bar_q_tmem(wg));
-            mbar_arrive(bar_q_empty);
-            return true;
-        };
-
-        // Epilogue of busy unit number uidx: wait for its last P V, read this row of O (tile wg)
-        // from TMEM (then free the accumulators for the next unit), write O / l and the LSE.
-        auto epilogue = [&](const UnitInfo& t, float m_ref, float l, int uidx) -> bool {
-            if (!__all_sync(FULL,
-                            mbar_wait(bar_o_full(wg), (uint32_t)(uidx & 1), wc, kErrTimeout)))
-                return false;
-            tc_fence_after_sync();
-            const int64_t i = t.q0 + wg * 128 + row;
-            const bool row_valid = i < p.sq;
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-            for (int c = 0; c < T::DV / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
-                tmem_wait_ld();
-                if (c == T::DV / 32 - 1) {
-                    // this tile's O has been read out: the next unit's P V may overwrite it
-                    tc_fence_before_sync();
-                    mbar_arrive(bar_o_free(wg));
-                }
-                uint32_t w[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
-                                       __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (row_valid) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        dst[c * 4 + q4] =
-                            make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
-                }
-            }
-            if (row_valid && p.lse)
-                p.lse[(t.bi * p.hq + t.h) * p.sq + i] =
-                    l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
-            return true;
-        };
-
-        // exp2(s * sl2 - m) for two scores, and their bf16 pair; masked keys give exactly 0.
-        auto p_pair = [&](uint32_t s0, uint32_t s1, float neg_m, bool v0, bool v1, float& p0,
-                          float& p1) -> uint32_t {
-            float x0, x1;
-            fma2(__uint_as_float(s0), __uint_as_float(s1), sl2, neg_m, x0, x1);
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-            p0 = v0 ? p0 : 0.f;
-            p1 = v1 ? p1 : 0.f;
-            return pack_bf16x2(p0, p1);
-        };
-
-        bool pend = false;  // a finished unit whose epilogue has not run yet
-        UnitInfo pend_t{};
-        float pend_m = 0.f, pend_l = 0.f;
-        int pend_idx = 0;
-        if (T::Q_TMEM && busy_from(u0) >= 0) ok = copy_q(0);
-        for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
-            const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
-            const int64_t i = t.q0 + wg * 128 + row;
-            if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
-                if (i < p.sq) {
-                    uint4* dst =
-                        reinterpret_cast<uint4*>(p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
-#pragma unroll 1
-                    for (int c = 0; c < T::DV / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                    if (p.lse) p.lse[(t.bi * p.hq + t.h) * p.sq + i] = -INFINITY;
-                }
-                continue;
-            }
-            const int64_t un = busy_from(u + ustep);
-            const int64_t lim_row = CAUSAL ? i + p.sk - p.sq : p.sk - 1;
-            const int64_t lim = lim_row < p.sk - 1 ? lim_row : p.sk - 1;  // last allowed key
-            float m_ref = -INFINITY;  // exponent reference (log2 units); moves lazily
-            float l = 0.f;            // sum of exp2(x - m_ref) over the keys seen so far
-
-            for (int j = 0; j < t.n_blocks; ++j, ++wi) {
-                // score buffer and its phase: one buffer per tile with two tiles, alternating
-                // buffers with one tile
-                const int sb = NT == 2 ? wg : (int)(wi & 1);
-                const uint32_t sph = NT == 2 ? (uint32_t)(wi & 1) : (uint32_t)(wi >> 1) & 1u;
-                const uint32_t s_col = tl + sb * BN;
-                ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), sph, wc, kErrTimeout));
-                if (!ok) break;
-                tc_fence_after_sync();
-                if (T::Q_TMEM && j == t.n_blocks - 1 && un >= 0) {
-                    // Every Q K^T of this tile in this unit is complete (its last S has landed),
-                    // so its Q columns can take the next unit's Q now, ahead of this softmax.
-                    ok = copy_q(units + 1);
-                    if (!ok) break;
-                }
-                const bool masked_block = j >= t.mask_from;
-                // keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all)
-                int64_t rel64 = lim - (int64_t)j * BN;
-                rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
-                const int rel = (int)rel64;
-
-                float bmax;
-                float rs = 0.f;  // sum of this block's p (relative to the reference after it)
-                float m_new, alpha = 1.f;
-                bool need;
-                if (NT == 1) {
-                    // ---- single pass: the whole score row stays in registers
-                    uint32_t sr[BN];
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c)
-                        tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-                    tmem_wait_ld();
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    if (masked_block) {
-#pragma unroll
-                        for (int c = 0; c < BN; ++c)
-                            mx[c & 3] = fmaxf(mx[c & 3], c <= rel ? __uint_as_float(sr[c]) : -INFINITY);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < BN; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
-                    }
-                    bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
-                    m_new = fmaxf(m_ref, m_blk);
-                    need = m_new > m_ref + 8.0f;
-                    if (need) {
-                        alpha = ex2(m_ref - m_new);
-                        m_ref = m_new;
-                        l *= alpha;
-                    }
-                    if (j > 0 && __any_sync(FULL, need)) {
-                        // O holds blocks < j: wait for the previous P V (item wi-1; bar_pv_done
-                        // is then in phase wi-1 or wi, so the parity test is unambiguous), then
-                        // scale O in place.
-                        ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(wi - 1) & 1u, wc,
-                                                        kErrTimeout));
-                        if (!ok) break;
-                        tc_fence_after_sync();
-#pragma unroll 1
-                        for (int c = 0; c < T::DV / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(tl + T::O_COL0 + c * 32, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            tmem_st32(tl + T::O_COL0 + c * 32, r);
-                        }
-                    }
-                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int h2 = 0; h2 < BN / 64; ++h2) {
-                        uint32_t pk[32];
-                        if (masked_block) {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int e = h2 * 64 + 2 * c;
-                                float p0, p1;
-                                pk[c] = p_pair(sr[e], sr[e + 1], neg_m, e <= rel, e + 1 <= rel, p0, p1);
-                                acc[(2 * c) & 3] += p0;
-                                acc[(2 * c + 1) & 3] += p1;
-                            }
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int e = h2 * 64 + 2 * c;
-                                float p0, p1;
-                                pk[c] = p_pair(sr[e], sr[e + 1], neg_m, true, true, p0, p1);
-                                acc[(2 * c) & 3] += p0;
-                                acc[(2 * c + 1) & 3] += p1;
-                            }
-                        }
-                        tmem_st32(s_col + h2 * 32, pk);
-                    }
-                    rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                } else {
-                    // ---- two passes over TMEM in 32-column chunks (max, then exp), so that few
-                    // registers are live; the next chunk's load overlaps this chunk's math.
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    uint32_t ra[32], rb[32];
-                    tmem_ld32(s_col, ra);
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t (&cur)[32] = (c & 1) ? rb : ra;
-                        uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
-                        tmem_wait_ld();
-                        if (c + 1 < BN / 32) tmem_ld32(s_col + (c + 1) * 32, nxt);
-                        if (masked_block) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                mx[e & 3] = fmaxf(mx[e & 3], c * 32 + e <= rel ? __uint_as_float(cur[e]) : -INFINITY);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(cur[e]));
-                        }
-                    }
-                    bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
-                    m_new = fmaxf(m_ref, m_blk);
-                    need = m_new > m_ref + 8.0f;
-                    if (need) {
-                        alpha = ex2(m_ref - m_new);
-                        m_ref = m_new;
-                        l *= alpha;
-                    }
-                    if (j > 0 && __any_sync(FULL, need)) {
-                        // O holds blocks < j of this tile. Its last P V (item of block j-1) was
-                        // issued before this block's Q K^T, so it is complete now that S has
-                        // landed: scale O in place.
-#pragma unroll 1
-                        for (int c = 0; c < T::DV / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            tmem_st32(tl + T::O_COL0 + wg * T::DV + c * 32, r);
-                        }
-                    }
-                    const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    tmem_ld32(s_col, ra);
-#pragma unroll
-                    for (int c = 0; c < BN / 32; ++c) {
-                        uint32_t (&cur)[32] = (c & 1) ? rb : ra;
-                        uint32_t (&nxt)[32] = (c & 1) ? ra : rb;
-                        tmem_wait_ld();
-                        if (c + 1 < BN / 32) tmem_ld32(s_col + (c + 1) * 32, nxt);
-                        uint32_t pk[16];
-                        if (masked_block) {
-#pragma unroll
-                            for (int e2 = 0; e2 < 16; ++e2) {
-                                const int e = c * 32 + 2 * e2;
-                                float p0, p1;
-                                pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, e <= rel, e + 1 <= rel, p0, p1);
-                                add2(acc[(2 * e2) & 3], acc[(2 * e2 + 1) & 3], p0, p1);
-                            }
-                        } else {
-#pragma unroll
-                            for (int e2 = 0; e2 < 16; ++e2) {
-                                float p0, p1;
-                                pk[e2] = p_pair(cur[2 * e2], cur[2 * e2 + 1], neg_m, true, true, p0, p1);
-                                add2(acc[(2 * e2) & 3], acc[(2 * e2 + 1) & 3], p0, p1);
-                            }
-                        }
-                        // P chunk c (16 columns of bf16 pairs) overwrites S columns already read
-                        tmem_st16(s_col + c * 16, pk);
-                    }
-                    rs = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-                }
-                l += rs;
-                tmem_wait_st();
-                tc_fence_before_sync();
-                mbar_arrive(bar_p_full(sb));
-                if (j == 0 && pend) {
-                    // The previous unit's epilogue, now that this unit's first P is out.
-                    pend = false;
-                    ok = epilogue(pend_t, pend_m, pend_l, pend_idx);
-                    if (!ok) break;
-                }
-            }
-            if (!ok) break;
-            pend = true;
-            pend_t = t;
-            pend_m = m_ref;
-            pend_l = l;
-            pend_idx = units;
-            ++units;
-        }
-        if (ok && pend) ok = epilogue(pend_t, pend_m, pend_l, pend_idx);
-        } else {
-        // --------------------------- softmax + epilogue warps 0-3 ---------------------------
-        const int row = threadIdx.x;  // TMEM lane
-        const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-        const float sl2 = p.scale_log2;
-        bool ok = true;
-        int64_t gi = 0;  // global item counter (score buffer gi % 2, phase (gi / 2) % 2)
+        int64_t jg = 0;  // key blocks stepped through so far (all units); item g = jg * NT + tile
         int units = 0;   // busy units whose items are done
 
         // Staged Q of busy unit number qidx, tile tt (128-byte swizzled rows, as TMA wrote them)
@@ -807,29 +543,72 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             tc_fence_after_sync();
             const int64_t i = t.q0 + tt * 128 + row;
             const bool row_valid = i < p.sq;
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            if constexpr (T::O_TMA) {
+                // This warp's 32 rows go to its own slab of the staging tile (one 32-row, 128-byte
+                // swizzled box per 64 columns), then one lane stores the slab with TMA; rows past
+                // sq are clipped by the tensor map. The slab is reused only after the previous
+                // store from it has been read out.
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
+                const int r32 = row & 31;
 #pragma unroll 1
-            for (int c = 0; c < T::DV / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
-                tmem_wait_ld();
-                if (c == T::DV / 32 - 1) {
-                    // this tile's O has been read out: the next unit's P V may overwrite it
-                    tc_fence_before_sync();
-                    mbar_arrive(bar_o_free(tt));
-                }
-                uint32_t w[16];
+                for (int c = 0; c < T::DV / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                    tmem_wait_ld();
+                    if (c == T::DV / 32 - 1) {
+                        // this tile's O has been read out: the next unit's P V may overwrite it
+                        tc_fence_before_sync();
+                        mbar_arrive(bar_o_free(tt));
+                    }
+                    uint32_t w[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
-                                       __uint_as_float(r[2 * e + 1]) * inv_l);
-                if (row_valid) {
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                           __uint_as_float(r[2 * e + 1]) * inv_l);
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        dst[c * 4 + q4] =
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int u16 = c * 4 + q4;  // 16-byte unit of the row
+                        uint8_t* slab = smem + T::O_OFF + T::o_slab(tt, u16 >> 3, w4);
+                        *reinterpret_cast<uint4*>(slab + r32 * 128 + (((u16 & 7) ^ (r32 & 7)) << 4)) =
                             make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int64_t row0 = t.q0 + tt * 128 + w4 * 32;
+                if (lane == 0 && row0 < p.sq) {
+#pragma unroll
+                    for (int bx = 0; bx < T::DV / 64; ++bx)
+                        tma_store_4d(&tmap_o, sbase + T::O_OFF + T::o_slab(tt, bx, w4), bx * 64,
+                                     (int)t.h, (int)row0, (int)t.bi);
+                    bulk_commit_group();
+                }
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(
+                    p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
+#pragma unroll 1
+                for (int c = 0; c < T::DV / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                    tmem_wait_ld();
+                    if (c == T::DV / 32 - 1) {
+                        // this tile's O has been read out: the next unit's P V may overwrite it
+                        tc_fence_before_sync();
+                        mbar_arrive(bar_o_free(tt));
+                    }
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l,
+                                           __uint_as_float(r[2 * e + 1]) * inv_l);
+                    if (row_valid) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            dst[c * 4 + q4] =
+                                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                    }
                 }
             }
             if (row_valid && p.lse)
@@ -840,18 +619,18 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 
         bool pend = false;  // a finished unit whose epilogues have not run yet
         UnitInfo pend_t{};
-        float pend_m[NT], pend_l[NT];
+        float pend_m[NTW], pend_l[NTW];
 #pragma unroll
-        for (int tt = 0; tt < NT; ++tt) pend_m[tt] = pend_l[tt] = 0.f;
+        for (int k = 0; k < NTW; ++k) pend_m[k] = pend_l[k] = 0.f;
         int pend_idx = 0;
         if (T::Q_TMEM && busy_from(u0) >= 0)
-            for (int tt = 0; tt < NT && ok; ++tt) ok = copy_q(0, tt);
+            for (int k = 0; k < NTW && ok; ++k) ok = copy_q(0, tile_of(k));
         for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
             const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
             if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt) {
-                    const int64_t i = t.q0 + tt * 128 + row;
+                for (int k = 0; k < NTW; ++k) {
+                    const int64_t i = t.q0 + tile_of(k) * 128 + row;
                     if (i < p.sq) {
                         uint4* dst = reinterpret_cast<uint4*>(
                             p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
@@ -863,24 +642,26 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 continue;
             }
             const int64_t un = busy_from(u + ustep);
-            int64_t lim[NT];  // last allowed key of this thread's row in each tile
-            float m_ref[NT];  // exponent reference (log2 units); moves lazily
-            float l[NT];      // sum of exp2(x - m_ref) over the keys seen so far
+            int64_t lim[NTW];  // last allowed key of this thread's row in each tile
+            float m_ref[NTW];  // exponent reference (log2 units); moves lazily
+            float l[NTW];      // sum of exp2(x - m_ref) over the keys seen so far
 #pragma unroll
-            for (int tt = 0; tt < NT; ++tt) {
-                const int64_t i = t.q0 + tt * 128 + row;
+            for (int k = 0; k < NTW; ++k) {
+                const int64_t i = t.q0 + tile_of(k) * 128 + row;
                 const int64_t lim_row = CAUSAL ? i + p.sk - p.sq : p.sk - 1;
-                lim[tt] = lim_row < p.sk - 1 ? lim_row : p.sk - 1;
-                m_ref[tt] = -INFINITY;
-                l[tt] = 0.f;
+                lim[k] = lim_row < p.sk - 1 ? lim_row : p.sk - 1;
+                m_ref[k] = -INFINITY;
+                l[k] = 0.f;
             }
 
-            for (int j = 0; j < t.n_blocks && ok; ++j) {
+            for (int j = 0; j < t.n_blocks && ok; ++j, ++jg) {
 #pragma unroll
-                for (int tt = 0; tt < NT; ++tt, ++gi) {
-                    const int sb = (int)(gi & 1);
+                for (int k = 0; k < NTW; ++k) {
+                    const int tt = tile_of(k);
+                    const int64_t g = jg * NT + tt;  // global item number
+                    const int sb = (int)(g & 1);     // score buffer
                     const uint32_t s_col = tl + sb * BN;
-                    ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(gi >> 1) & 1u, wc,
+                    ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(g >> 1) & 1u, wc,
                                                     kErrTimeout));
                     if (!ok) break;
                     tc_fence_after_sync();
@@ -896,42 +677,57 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                     tmem_wait_ld();
 
-                    const bool masked_block = j >= t.mask_from;
-                    // keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all)
-                    int64_t rel64 = lim[tt] - (int64_t)j * BN;
-                    rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
-                    const int rel = (int)rel64;
+                    // Keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all).
+                    // Per 32-key chunk the warp takes one of three uniform paths: every row of
+                    // the warp allows the whole chunk (nothing to do), none allows any of it
+                    // (skipped below: no max, P = 0 without exp2), or the chunk holds some row's
+                    // limit: then the disallowed scores become -inf, so the max ignores them and
+                    // their p = exp2(-inf) is exactly 0 (the scale factor is never 0: the launch
+                    // clamps it to at least 2^-100).
+                    int rel_hi = BN;  // the warp's largest rel: chunks starting above it are skipped
+                    if (j >= t.mask_from) {
+                        int64_t rel64 = lim[k] - (int64_t)j * BN;
+                        rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
+                        const int rel = (int)rel64;
+                        const int rel_lo = __reduce_min_sync(FULL, rel);
+                        rel_hi = __reduce_max_sync(FULL, rel);
+#pragma unroll
+                        for (int ch = 0; ch < BN / 32; ++ch) {
+                            if (ch * 32 + 31 <= rel_lo || ch * 32 > rel_hi) continue;
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                sr[ch * 32 + e] = ch * 32 + e <= rel ? sr[ch * 32 + e] : 0xff800000u;
+                        }
+                    }
                     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    if (masked_block) {
 #pragma unroll
-                        for (int c = 0; c < BN; ++c)
-                            mx[c & 3] = fmaxf(mx[c & 3],
-                                              c <= rel ? __uint_as_float(sr[c]) : -INFINITY);
-                    } else {
+                    for (int ch = 0; ch < BN / 32; ++ch) {
+                        if (ch * 32 > rel_hi) continue;
 #pragma unroll
-                        for (int c = 0; c < BN; ++c)
-                            mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c]));
+                        for (int c = 0; c < 16; ++c)
+                            mx[c & 3] = fmax3(mx[c & 3], __uint_as_float(sr[ch * 32 + 2 * c]),
+                                              __uint_as_float(sr[ch * 32 + 2 * c + 1]));
                     }
                     const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
                     const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
-                    const float m_new = fmaxf(m_ref[tt], m_blk);
+                    const float m_new = fmaxf(m_ref[k], m_blk);
                     // Lazy rescale: keep the old reference while the running max stays within
                     // 2^8 of it; the final O / l uses the same reference, so the result is exact.
-                    const bool need = m_new > m_ref[tt] + 8.0f;
+                    const bool need = m_new > m_ref[k] + 8.0f;
                     float alpha = 1.f;
                     if (need) {
-                        alpha = ex2(m_ref[tt] - m_new);
-                        m_ref[tt] = m_new;
-                        l[tt] *= alpha;
+                        alpha = ex2(m_ref[k] - m_new);
+                        m_ref[k] = m_new;
+                        l[k] *= alpha;
                     }
                     if (j > 0 && __any_sync(FULL, need)) {
                         // O holds blocks < j of this tile: scale it in place once its last P V
-                        // is complete. With two tiles that P V is item gi-2, issued before this
+                        // is complete. With two tiles that P V is item g-2, issued before this
                         // item's Q K^T, so it is complete now that S has landed. With one tile it
-                        // is item gi-1: wait for it (bar_pv_done is then in phase gi-1 or gi, so
-                        // the parity test on phase gi-1 is unambiguous).
+                        // is item g-1: wait for it (bar_pv_done is then in phase g-1 or g, so
+                        // the parity test on phase g-1 is unambiguous).
                         if (NT == 1) {
-                            ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(gi - 1) & 1u,
+                            ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(g - 1) & 1u,
                                                             wc, kErrTimeout));
                             if (!ok) break;
                             tc_fence_after_sync();
@@ -947,46 +743,43 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                             tmem_st32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
                         }
                     }
-                    const float neg_m = (m_ref[tt] == -INFINITY) ? 0.f : -m_ref[tt];
+                    const float neg_m = (m_ref[k] == -INFINITY) ? 0.f : -m_ref[k];
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int h2 = 0; h2 < BN / 64; ++h2) {
-                        uint32_t pk[32];
-                        if (masked_block) {
+                    for (int ch = 0; ch < BN / 32; ++ch) {
+                        uint32_t pk[16];
+                        if (ch * 32 > rel_hi) {  // no row of this warp allows any key here
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int e = h2 * 64 + 2 * c;
-                                float x0, x1;
-                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, neg_m,
-                                     x0, x1);
-                                float p0 = ex2(x0), p1 = ex2(x1);
-                                p0 = (e <= rel) ? p0 : 0.f;  // masked keys: exactly 0
-                                p1 = (e + 1 <= rel) ? p1 : 0.f;
-                                add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
-                                pk[c] = pack_bf16x2(p0, p1);
-                            }
+                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
                         } else {
 #pragma unroll
-                            for (int c = 0; c < 32; ++c) {
-                                const int e = h2 * 64 + 2 * c;
+                            for (int c = 0; c < 16; ++c) {
+                                const int e = ch * 32 + 2 * c;
                                 float x0, x1;
-                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, neg_m,
-                                     x0, x1);
-                                const float p0 = ex2(x0), p1 = ex2(x1);
+                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2,
+                                     neg_m, x0, x1);
+                                float p0, p1;
+                                if ((T::EXP_FMA_PAIRS >> (c & 7)) & 1u) {
+                                    exp2_fma_pair(x0, x1, p0, p1);
+                                } else {
+                                    p0 = ex2(x0);
+                                    p1 = ex2(x1);
+                                }
                                 add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
                                 pk[c] = pack_bf16x2(p0, p1);
                             }
                         }
-                        tmem_st32(s_col + h2 * 32, pk);
+                        // P chunk ch (16 columns of bf16 pairs) overwrites S columns already read
+                        tmem_st16(s_col + ch * 16, pk);
                     }
-                    l[tt] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                    l[k] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
                     tmem_wait_st();
                     tc_fence_before_sync();
                     mbar_arrive(bar_p_full(sb));
                     if (j == 0 && pend) {
                         // Tile tt of the previous unit, now that its successor's first P is out.
-                        ok = epilogue(pend_t, tt, pend_m[tt], pend_l[tt], pend_idx);
-                        if (tt == NT - 1) pend = false;
+                        ok = epilogue(pend_t, tt, pend_m[k], pend_l[k], pend_idx);
+                        if (k == NTW - 1) pend = false;
                         if (!ok) break;
                     }
                 }
@@ -995,17 +788,18 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             pend = true;
             pend_t = t;
 #pragma unroll
-            for (int tt = 0; tt < NT; ++tt) {
-                pend_m[tt] = m_ref[tt];
-                pend_l[tt] = l[tt];
+            for (int k = 0; k < NTW; ++k) {
+                pend_m[k] = m_ref[k];
+                pend_l[k] = l[k];
             }
             pend_idx = units;
             ++units;
         }
         if (ok && pend)
-            for (int tt = 0; tt < NT && ok; ++tt)
-                ok = epilogue(pend_t, tt, pend_m[tt], pend_l[tt], pend_idx);
-        }
+            for (int k = 0; k < NTW && ok; ++k)
+                ok = epilogue(pend_t, tile_of(k), pend_m[k], pend_l[k], pend_idx);
+        // every O store this warp issued is complete before the CTA exits
+        if (T::O_TMA && lane == 0) bulk_wait_all();
     }
 
     // ---- teardown: every tcgen05 access is complete (MMAs drained, loads waited) ----

@@ -68,7 +68,9 @@ struct WaitCtx {
     uint64_t timeout_ns;
 };
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx& w,
+// Inlined like every helper here: ptxas cannot allocate registers for a called function inside
+// code whose per-warpgroup budget setmaxnreg changes.
+__device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitCtx& w,
                                             int code)
 {
     const uint64_t t0 = global_timer_ns();
@@ -106,6 +108,59 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* desc, uint
         " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(desc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
         : "memory");
+}
+
+// Shared -> global tile store, tracked by the issuing thread's bulk-async groups. Rows outside
+// the tensor map's extent are not written.
+__device__ __forceinline__ void tma_store_4d(const void* desc, uint32_t src, int c0, int c1, int c2,
+                                             int c3)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(desc)), "r"(src), "r"(c0), "r"(c1), "r"(c2),
+                 "r"(c3)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group()
+{
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// This thread's committed bulk stores have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// This thread's committed bulk stores are complete (written to global memory).
+__device__ __forceinline__ void bulk_wait_all()
+{
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Barrier over `count` threads (a multiple of 32) with id `id` (1..15; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Per-thread register budget of the executing warpgroup (all four warps execute it).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------------------------------------
@@ -266,6 +321,34 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Division of 0 <= n < 2^31 by a divisor fixed at launch, as a multiply-high, an add and a
+// shift (Granlund and Montgomery, "Division by Invariant Integers using Multiplication", 1994:
+// the round-up multiplier m = floor(2^32 (2^l - d) / d) + 1 with l = ceil(log2 d)).
+struct FastDiv {
+    uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d)
+{
+    uint32_t l = 0;
+    while (l < 32 && ((uint64_t)1 << l) < d) ++l;
+    const uint64_t m = ((((uint64_t)1 << l) - d) << 32) / d + 1;
+    return FastDiv{d, (uint32_t)m, l};
+}
+
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, const FastDiv& f)
+{
+    return (__umulhi(n, f.m) + n) >> f.l;
+}
+
 // (x0, x1) = (a0 * b + c, a1 * b + c) with one packed fp32x2 FMA (flush-to-zero).
 __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float& x0, float& x1)
 {
@@ -289,6 +372,47 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1)
         "mov.b64 {%0, %1}, ra;\n\t}"
         : "+f"(s0), "+f"(s1)
         : "f"(a0), "f"(a1));
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe, leaving the MUFU unit (16 exp2 per clock per
+// SM) to the other pairs. Round-to-nearest splits x = j + f with |f| <= 1/2 (adding and then
+// subtracting 1.5 * 2^23 rounds to an integer, and leaves j in the low bits of the sum),
+// 2^f comes from the cubic 1 + f (c1 + f (c2 + f c3)) (a minimax fit, relative error 1.0e-4
+// in fp32; fit_exp2_poly.py derives it), and j is added to the exponent field as an integer.
+// x is clamped at -127 first: there j = -127, f = 0, 2^f = 1 exactly and the result is +0, as
+// for every smaller x (so -inf, a masked score, gives exactly 0 like ex2.approx.ftz).
+constexpr float kExp2C1 = 0.6932829022407532f;
+constexpr float kExp2C2 = 0.2422109693288803f;
+constexpr float kExp2C3 = 0.05500893294811249f;
+
+__device__ __forceinline__ uint64_t f32x2_splat(float a)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+    return r;
+}
+
+__device__ __forceinline__ void exp2_fma_pair(float x0, float x1, float& y0, float& y1)
+{
+    const uint64_t magic = f32x2_splat(12582912.0f);  // 1.5 * 2^23
+    const uint64_t c1 = f32x2_splat(kExp2C1), c2 = f32x2_splat(kExp2C2),
+                   c3 = f32x2_splat(kExp2C3), one = f32x2_splat(1.0f);
+    x0 = fmaxf(x0, -127.0f);
+    x1 = fmaxf(x1, -127.0f);
+    uint64_t x, t, r, f, q;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+    asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(magic));  // 1.5 * 2^23 + j
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(t), "l"(magic));  // j
+    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(r));      // f = x - j
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(c3), "l"(f), "l"(c2));
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(c1));
+    asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(q), "l"(f), "l"(one));
+    uint32_t t0, t1, q0, q1;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(q0), "=r"(q1) : "l"(q));
+    // the low bits of t hold j (two's complement); t << 23 keeps only j * 2^23
+    y0 = __uint_as_float((t0 << 23) + q0);
+    y1 = __uint_as_float((t1 << 23) + q1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
