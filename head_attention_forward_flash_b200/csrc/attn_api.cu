@@ -173,11 +173,12 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 // warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe>. Tensor
 // memory holds two score buffers, one O per query tile and (when it fits) each tile's Q; shared
 // memory holds the Q staging buffer and the K / V rings. The (tiles, warpgroups) choice per head
-// dim is the measured fastest on B200. d64 is bound by the exp2 rate, so 3 of every 8 score
-// pairs take the FMA-pipe exp2 there.
+// dim is the measured fastest on B200. The share of score pairs whose exp2 runs on the FMA pipe
+// is the measured best per head dim (3 of 8 at d64, 2 of 8 at d128 / d192, none at d256, which
+// is bound by the tensor core).
 using T64 = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 KB
-using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2>;   // smem 64 + 96 + 64 KB
-using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1>;   // smem 96 + 96 + 32 KB
+using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 + 96 + 64 KB
+using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
 template <class T>

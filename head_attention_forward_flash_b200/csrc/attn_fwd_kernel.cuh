@@ -186,6 +186,44 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
     return t;
 }
 
+// S = Q K^T for one query tile and one key block: DQK/16 MMAs of M128 x N=BN x K16. K (and Q
+// when staged in shared memory) are K-major 128-byte swizzled tiles in 64-column chunks, so
+// k-step kk starts (kk / 4) chunks and (kk % 4) * 32 bytes in. q is a TMEM column (Q in TMEM)
+// or a shared-memory address.
+template <class T>
+__device__ __forceinline__ void issue_qk_mmas(uint32_t d_tmem, uint32_t q, uint32_t kaddr,
+                                              uint32_t idesc)
+{
+    const uint64_t b0 = make_sdesc_sw128(kaddr, 16, 1024);
+    if constexpr (T::Q_TMEM) {
+#pragma unroll
+        for (int kk = 0; kk < T::DQK / 16; ++kk)
+            mma_ts(d_tmem, q + kk * 8,
+                   sdesc_advance(b0, (kk >> 2) * T::CHUNK_BYTES + (kk & 3) * 32), idesc,
+                   kk > 0 ? 1u : 0u);
+    } else {
+        const uint64_t a0 = make_sdesc_sw128(q, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < T::DQK / 16; ++kk)
+            mma_ss(d_tmem, sdesc_advance(a0, (kk >> 2) * T::QCHUNK_BYTES + (kk & 3) * 32),
+                   sdesc_advance(b0, (kk >> 2) * T::CHUNK_BYTES + (kk & 3) * 32), idesc,
+                   kk > 0 ? 1u : 0u);
+    }
+}
+
+// O += P V for one query tile and one key block: BN/16 MMAs of M128 x N=DV x K16 with P (bf16
+// pairs) from TMEM and V an MN-major 128-byte swizzled tile (16 keys = 2048 bytes per k-step).
+template <class T>
+__device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, uint32_t vaddr,
+                                              bool accumulate)
+{
+    const uint64_t b0 = make_sdesc_sw128(vaddr, T::CHUNK_BYTES, 1024);
+#pragma unroll
+    for (int kk = 0; kk < T::BN / 16; ++kk)
+        mma_ts(o_tmem, p_tmem + kk * 8, sdesc_advance(b0, kk * 2048), T::IDESC_PV,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
 template <class T, bool CAUSAL>
 __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -400,22 +438,10 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     }
                     kaddr = k_slots + kslot * T::K_TILE_BYTES;
                 }
-                const uint32_t d_tmem = tmem + (uint32_t)(gi & 1) * BN;
-#pragma unroll
-                for (int kk = 0; kk < T::DQK / 16; ++kk) {
-                    const uint64_t bdesc = make_sdesc_sw128(
-                        kaddr + (kk >> 2) * T::CHUNK_BYTES + (kk & 3) * 32, 16, 1024);
-                    if (T::Q_TMEM) {
-                        mma_ts(d_tmem, tmem + T::Q_COL0 + tt * (T::DQK / 2) + kk * 8, bdesc,
-                               p.idesc_qk, kk > 0 ? 1u : 0u);
-                    } else {
-                        const uint64_t adesc = make_sdesc_sw128(
-                            q_stage + tt * T::Q_TILE_BYTES + (kk >> 2) * T::QCHUNK_BYTES +
-                                (kk & 3) * 32,
-                            16, 1024);
-                        mma_ss(d_tmem, adesc, bdesc, p.idesc_qk, kk > 0 ? 1u : 0u);
-                    }
-                }
+                issue_qk_mmas<T>(tmem + (uint32_t)(gi & 1) * BN,
+                                 T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
+                                           : q_stage + tt * T::Q_TILE_BYTES,
+                                 kaddr, p.idesc_qk);
                 tc_commit(bar_s_full(gi & 1));
                 if (tt == NT - 1) tc_commit(bar_kempty(kslot));
                 if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
@@ -442,15 +468,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     }
                     vaddr = v_slots + vslot * T::V_TILE_BYTES;
                 }
-                const uint32_t p_tmem = tmem + (uint32_t)(g & 1) * BN;
-                const uint32_t o_tmem = tmem + T::O_COL0 + tt * T::DV;
-#pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t bdesc =
-                        make_sdesc_sw128(vaddr + kk * 2048, T::CHUNK_BYTES, 1024);
-                    mma_ts(o_tmem, p_tmem + kk * 8, bdesc, T::IDESC_PV,
-                           (j > 0 || kk > 0) ? 1u : 0u);
-                }
+                issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)(g & 1) * BN, vaddr,
+                                 j > 0);
                 if (NT == 1) tc_commit(bar_pv_done);
                 if (tt == NT - 1) tc_commit(bar_vempty(vslot));
                 if (last_block) tc_commit(bar_o_full(tt));

@@ -257,6 +257,18 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
     return d;
 }
 
+// The descriptor of the same layout starting `bytes` further on: only the 14-bit start field
+// (address / 16, bits 0-13) changes, and it cannot carry for addresses inside shared memory.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t d, uint32_t bytes)
+{
+    uint32_t lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(d));
+    lo += bytes >> 4;
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
 // 32 lanes x 32 columns of 32-bit words: thread t of the warp gets lane (base lane + t).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
 {
