@@ -118,6 +118,15 @@ class OracleSampler:
         return max(1, int(n * seconds / max(dt, 1e-6)))
 
 
+def varlen_first_sequence(c, inputs):
+    """A packed-sequence workload's first sequence as a dense b = 1 config and its inputs."""
+    q, k, v, cu_q, cu_k = inputs
+    n_q, n_k = int(cu_q[1]), int(cu_k[1])
+    c0 = dict(c, b=1, sq=n_q, sk=n_k, varlen=False,
+              workload=f"{c['workload']} (sequence 0: {n_q} queries)")
+    return c0, (q[:n_q].unsqueeze(0), k[:n_k].unsqueeze(0), v[:n_k].unsqueeze(0))
+
+
 def cpu_baseline(c, inputs, seconds):
     s = OracleSampler(c, inputs)
     n = s.rows_for(seconds)
@@ -231,10 +240,17 @@ def run_gpu(args):
     c = workloads.config(args.config)
     c_rank = dict(c)
     c_rank["seed"] = c["seed"] + 7919 * rank  # every rank its own independent batch
-    q_h, k_h, v_h = workloads.config_inputs(c_rank)
+    varlen = bool(c.get("varlen"))
+    if varlen:  # packed sequences: [total, h, d] tensors and int32 offsets
+        q_h, k_h, v_h, cuq_h, cuk_h = workloads.config_varlen_inputs(c_rank)
+        cu_q, cu_k = cuq_h.to(dev), cuk_h.to(dev)
+        o = torch.empty((q_h.shape[0], c["hq"], c["dv"]), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((c["hq"], q_h.shape[0]), dtype=torch.float32, device=dev)
+    else:
+        q_h, k_h, v_h = workloads.config_inputs(c_rank)
+        o = torch.empty((c["b"], c["sq"], c["hq"], c["dv"]), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((c["b"], c["hq"], c["sq"]), dtype=torch.float32, device=dev)
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    o = torch.empty((c["b"], c["sq"], c["hq"], c["dv"]), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((c["b"], c["hq"], c["sq"]), dtype=torch.float32, device=dev)
     mean = torch.empty((c["b"], c["hk"], c["dqk"]), dtype=torch.float32, device=dev)
     k_s = torch.empty_like(k) if c["kmean"] else None
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -248,7 +264,11 @@ def run_gpu(args):
             b2.k_smooth_sub(k, mean, k_s)
             kk = k_s
         ev_a0.record(stream)
-        b2.attn_fwd(q, kk, v, causal=c["causal"], scale=c["scale"], out=o, lse=lse)
+        if varlen:
+            b2.attn_fwd_varlen(q, kk, v, cu_q, cu_k, c["sq"], causal=c["causal"],
+                               scale=c["scale"], out=o, lse=lse)
+        else:
+            b2.attn_fwd(q, kk, v, causal=c["causal"], scale=c["scale"], out=o, lse=lse)
         ev_a1.record(stream)
 
     ev_a0 = torch.cuda.Event(enable_timing=True)
@@ -316,13 +336,21 @@ def run_gpu(args):
         ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps + 1)]
         ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps + 1)]
 
+        if varlen:
+            cqp, ckp = cuq_h.pin_memory(), cuk_h.pin_memory()
+
         def e2e_step():
             qd = qp.to(dev, non_blocking=True)
             kd = kp.to(dev, non_blocking=True)
             vd = vp.to(dev, non_blocking=True)
             if c["kmean"]:
                 kd = b2.k_smooth_sub(kd, b2.k_smooth_mean(kd))
-            od, ld = b2.attn_fwd(qd, kd, vd, causal=c["causal"], scale=c["scale"])
+            if varlen:
+                od, ld = b2.attn_fwd_varlen(qd, kd, vd, cqp.to(dev, non_blocking=True),
+                                            ckp.to(dev, non_blocking=True), c["sq"],
+                                            causal=c["causal"], scale=c["scale"])
+            else:
+                od, ld = b2.attn_fwd(qd, kd, vd, causal=c["causal"], scale=c["scale"])
             op.copy_(od, non_blocking=True)
             lp.copy_(ld, non_blocking=True)
 
@@ -335,13 +363,19 @@ def run_gpu(args):
         e_ms = max_over_ranks(sum(ev0[s].elapsed_time(ev1[s]) for s in range(1, e_steps + 1))
                               / e_steps)
         h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+        if varlen:
+            h2d += (cuq_h.numel() + cuk_h.numel()) * 4
         d2h = o.numel() * 2 + lse.numel() * 4
         e2e = {"value": world * fl / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(c, (q_h, k_h, v_h), args.cpu_seconds)
+        if varlen:  # the oracle on rows of the first sequence, as a dense b = 1 problem
+            c0, inputs0 = varlen_first_sequence(c, (q_h, k_h, v_h, cuq_h, cuk_h))
+            cpu = cpu_baseline(c0, inputs0, args.cpu_seconds)
+        else:
+            cpu = cpu_baseline(c, (q_h, k_h, v_h), args.cpu_seconds)
 
     if world > 1:
         dist.destroy_process_group()
@@ -360,11 +394,14 @@ def run_gpu(args):
                                  peaks.get("bf16_tflops_sustained", FALLBACK[
                                      "bf16_tflops_sustained"]),
                                  "source": peak_src},
-        "config": {"workload": c["workload"], "b": c["b"], "hq": c["hq"], "hk": c["hk"],
-                   "sq": c["sq"], "sk": c["sk"], "dqk": c["dqk"], "dv": c["dv"],
-                   "causal": c["causal"], "kmean_prepass": c["kmean"], "scale": c["scale"],
-                   "l2": "flushed before every step (256 MiB write, outside the events)",
-                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "config": dict({"workload": c["workload"], "b": c["b"], "hq": c["hq"], "hk": c["hk"],
+                        "sq": c["sq"], "sk": c["sk"], "dqk": c["dqk"], "dv": c["dv"],
+                        "causal": c["causal"], "kmean_prepass": c["kmean"], "scale": c["scale"],
+                        "l2": "flushed before every step (256 MiB write, outside the events)",
+                        "parallelism": f"replicas x{world} (independent batches, no "
+                                       f"collective)"},
+                       **({"packed_sequence_lengths": workloads.varlen_lengths(c)}
+                          if varlen else {})),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": f"attn_fwd_kernel d{c['dqk']}x{c['dv']}",
@@ -389,7 +426,11 @@ def run_reference(args):
     if rank != 0:
         return  # the oracle arm runs on rank 0 only
     c = workloads.config(args.config)
-    s = OracleSampler(c)
+    if c.get("varlen"):  # the oracle on rows of the first sequence (a dense b = 1 problem)
+        c, inputs0 = varlen_first_sequence(c, workloads.config_varlen_inputs(c))
+        s = OracleSampler(c, inputs0)
+    else:
+        s = OracleSampler(c)
     per_step = max(0.5, min(8.0, 90.0 / max(1, args.steps + args.warmup)))
     n = s.rows_for(per_step)
     for _ in range(args.warmup):

@@ -25,7 +25,7 @@ STATUS = {
     6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
     11: "ERR_SCRATCH",
 }
-EXPORTS = ("attn_fwd", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+EXPORTS = ("attn_fwd", "attn_fwd_varlen", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
            "attn_status_string", "attn_debug_status")
 
 
@@ -45,6 +45,9 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_int,
                              ctypes.c_float, vp]
     lib.attn_fwd.restype = ctypes.c_int
+    lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
+                                    i64, ctypes.c_int, ctypes.c_float, vp]
+    lib.attn_fwd_varlen.restype = ctypes.c_int
     lib.k_smooth_mean.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean.restype = ctypes.c_int
     lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
@@ -111,6 +114,48 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
                       lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
                       1 if causal else 0, float(scale), _stream_ptr(q))
     _check("attn_fwd", st)
+    return out, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, causal: bool = False,
+                    scale: float | None = None, out=None, lse=None, return_lse: bool = True):
+    """attn_fwd over packed sequences: sequence i owns query rows cu_seqlens_q[i] ..
+    cu_seqlens_q[i+1]-1 and key rows cu_seqlens_k[i] .. cu_seqlens_k[i+1]-1.
+
+    q [total_q, hq, dqk], k [total_k, hk, dqk], v [total_k, hk, dv]: contiguous bf16 CUDA
+    tensors; cu_seqlens_q / cu_seqlens_k: int32 CUDA tensors of b + 1 offsets; max_seqlen_q: at
+    least the longest query length. Returns ``(out [total_q, hq, dv] bf16, lse [hq, total_q] fp32
+    or None)``. Rows that belong to no sequence are left as allocated.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _want(t, name, 3)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        _want(t, name, 1)
+        if t.dtype != torch.int32:
+            raise TypeError(f"{name} must be int32")
+    total_q, hq, dqk = q.shape
+    total_k, hk, dqk2 = k.shape
+    total_kv, hkv, dv = v.shape
+    if dqk2 != dqk or total_kv != total_k or hkv != hk:
+        raise ValueError("inconsistent q/k/v shapes")
+    b = cu_seqlens_q.shape[0] - 1
+    if b < 0 or cu_seqlens_k.shape[0] != b + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold b + 1 offsets")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    if out is None:
+        out = torch.empty((total_q, hq, dv), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((hq, total_q), dtype=torch.float32, device=q.device)
+    st = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr() if lse is not None else None,
+                             cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), b, hq, hk, total_q,
+                             total_k, int(max_seqlen_q), dqk, dv, 1 if causal else 0,
+                             float(scale), _stream_ptr(q))
+    _check("attn_fwd_varlen", st)
     return out, lse
 
 

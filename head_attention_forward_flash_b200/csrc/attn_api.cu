@@ -95,17 +95,28 @@ int sm_count()
     return cached[dev];
 }
 
-template <class T, bool CAUSAL>
-int launch_attn(const void* q, const void* k, const void* v, void* out, float* lse, int64_t b,
-                int64_t hq, int64_t hk, int64_t sq, int64_t sk, float scale, cudaStream_t stream)
+// Problem geometry. Dense: b batches of sq queries and sk keys. Packed sequences: b sequences,
+// sq = the longest query length, the per-sequence offsets in cu_q / cu_k (device memory), and
+// the tensors' total row counts.
+struct Shape {
+    int64_t b, hq, hk, sq, sk;
+    const int* cu_q = nullptr;
+    const int* cu_k = nullptr;
+    int64_t total_q = 0, total_k = 0;
+};
+
+template <class T, bool CAUSAL, bool VARLEN>
+int launch_attn(const void* q, const void* k, const void* v, void* out, float* lse,
+                const Shape& sh, float scale, cudaStream_t stream)
 {
+    const int64_t b = sh.b, hq = sh.hq, hk = sh.hk, sq = sh.sq, sk = sh.sk;
     static bool attr_done[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
-    auto kern = attn_fwd_kernel<T, CAUSAL>;
+    auto kern = attn_fwd_kernel<T, CAUSAL, VARLEN>;
     if (!attr_done[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)T::SMEM_BYTES) != cudaSuccess) {
@@ -127,12 +138,16 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
         }
         attr_done[dev] = true;
     }
+    // packed sequences: one batch of all rows; each unit adds its sequence's first row
+    const int64_t mb = VARLEN ? 1 : b;
+    const int64_t mq = VARLEN ? sh.total_q : sq;
+    const int64_t mk = VARLEN ? sh.total_k : sk;
     CUtensorMap tq, tk, tv, to;
-    int rc = encode_bshd(&tq, q, b, sq, hq, T::DQK, T::BM);
-    if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, b, sk, hk, T::DQK, T::BN);
-    if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, b, sk, hk, T::DV, T::BN);
+    int rc = encode_bshd(&tq, q, mb, mq, hq, T::DQK, T::BM);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, mb, mk, hk, T::DQK, T::BN);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, mb, mk, hk, T::DV, T::BN);
     // O is stored per warp: boxes of 32 rows (only used when the kernel stages O for TMA)
-    if (rc == B200ATTN_OK) rc = encode_bshd(&to, out, b, sq, hq, T::DV, 32);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&to, out, mb, mq, hq, T::DV, 32);
     if (rc != B200ATTN_OK) return rc;
     int* status = status_word();
     const int n_sm = sm_count();
@@ -146,6 +161,10 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.hk = hk;
     p.sq = sq;
     p.sk = sk;
+    p.cu_q = sh.cu_q;
+    p.cu_k = sh.cu_k;
+    p.total_q = sh.total_q;
+    p.total_k = sh.total_k;
     p.group = hq / hk;
     p.n_qu = (sq + T::NT * T::BM - 1) / (T::NT * T::BM);
     p.n_units = b * hq * p.n_qu;  // below 2^31 (checked by attn_fwd)
@@ -182,12 +201,26 @@ using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 +
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
 template <class T>
-int dispatch_causal(int causal, const void* q, const void* k, const void* v, void* out,
-                    float* lse, int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk,
-                    float scale, cudaStream_t st)
+int dispatch(int causal, bool varlen, const void* q, const void* k, const void* v, void* out,
+             float* lse, const Shape& sh, float scale, cudaStream_t st)
 {
-    return causal ? launch_attn<T, true>(q, k, v, out, lse, b, hq, hk, sq, sk, scale, st)
-                  : launch_attn<T, false>(q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    if (varlen)
+        return causal ? launch_attn<T, true, true>(q, k, v, out, lse, sh, scale, st)
+                      : launch_attn<T, false, true>(q, k, v, out, lse, sh, scale, st);
+    return causal ? launch_attn<T, true, false>(q, k, v, out, lse, sh, scale, st)
+                  : launch_attn<T, false, false>(q, k, v, out, lse, sh, scale, st);
+}
+
+int dispatch_dims(int64_t dqk, int causal, bool varlen, const void* q, const void* k,
+                  const void* v, void* out, float* lse, const Shape& sh, float scale,
+                  cudaStream_t st)
+{
+    switch (dqk) {
+    case 64: return dispatch<T64>(causal, varlen, q, k, v, out, lse, sh, scale, st);
+    case 128: return dispatch<T128>(causal, varlen, q, k, v, out, lse, sh, scale, st);
+    case 192: return dispatch<T192>(causal, varlen, q, k, v, out, lse, sh, scale, st);
+    default: return dispatch<T256>(causal, varlen, q, k, v, out, lse, sh, scale, st);
+    }
 }
 
 // Rows with no key at all (sk == 0): O = 0, LSE = -inf.
@@ -243,12 +276,65 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* out, 
                                              n_l / 4);
         return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
     }
-    switch (dqk) {
-    case 64: return dispatch_causal<T64>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
-    case 128: return dispatch_causal<T128>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
-    case 192: return dispatch_causal<T192>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
-    default: return dispatch_causal<T256>(causal, q, k, v, out, lse, b, hq, hk, sq, sk, scale, st);
+    Shape sh;
+    sh.b = b;
+    sh.hq = hq;
+    sh.hk = hk;
+    sh.sq = sq;
+    sh.sk = sk;
+    return dispatch_dims(dqk, causal, false, q, k, v, out, lse, sh, scale, st);
+}
+
+extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                               const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int64_t b,
+                               int64_t hq, int64_t hk, int64_t total_q, int64_t total_k,
+                               int64_t max_sq, int64_t dqk, int64_t dv, int causal, float scale,
+                               void* stream)
+{
+    if (b < 0 || hq < 0 || hk <= 0 || total_q < 0 || total_k < 0 || max_sq < 0)
+        return B200ATTN_ERR_SHAPE;
+    if (hq % hk != 0) return B200ATTN_ERR_GQA;
+    const bool hd_ok = (dqk == 64 && dv == 64) || (dqk == 128 && dv == 128) ||
+                       (dqk == 192 && dv == 128) || (dqk == 256 && dv == 256);
+    if (!hd_ok) return B200ATTN_ERR_HEADDIM;
+    if (!std::isfinite(scale)) return B200ATTN_ERR_SCALE;
+    int64_t n_q, n_k, n_v, n_o, n_l, n_units;
+    if (!numel({total_q, hq, dqk, 2}, &n_q) || !numel({total_k, hk, dqk, 2}, &n_k) ||
+        !numel({total_k, hk, dv, 2}, &n_v) || !numel({total_q, hq, dv, 2}, &n_o) ||
+        !numel({hq, total_q, 4}, &n_l) || !numel({b, hq, (max_sq + 127) / 128}, &n_units) ||
+        n_units >= ((int64_t)1 << 31) || total_q >= ((int64_t)1 << 31) ||
+        total_k >= ((int64_t)1 << 31) || b >= ((int64_t)1 << 31))
+        return B200ATTN_ERR_RANGE;
+    if (n_o == 0 || b == 0 || max_sq == 0) return B200ATTN_OK;  // no query row to compute
+    if (!q || !out || !cu_seqlens_q || !cu_seqlens_k || (total_k > 0 && (!k || !v)))
+        return B200ATTN_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(out, 16) || (k && !aligned(k, 16)) ||
+        (v && !aligned(v, 16)) || (lse && !aligned(lse, 4)) || !aligned(cu_seqlens_q, 4) ||
+        !aligned(cu_seqlens_k, 4))
+        return B200ATTN_ERR_ALIGN;
+    if (!tma_extent_ok(1, total_q, hq, dqk) ||
+        (total_k > 0 && (!tma_extent_ok(1, total_k, hk, dqk) || !tma_extent_ok(1, total_k, hk, dv))))
+        return B200ATTN_ERR_RANGE;
+    int rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (total_k == 0) {  // no keys anywhere: every query row gets O = 0, LSE = -inf
+        fill_empty_rows<<<296, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), n_o / 2, lse,
+                                             n_l / 4);
+        return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
     }
+    Shape sh;
+    sh.b = b;
+    sh.hq = hq;
+    sh.hk = hk;
+    sh.sq = max_sq;
+    sh.sk = 0;
+    sh.cu_q = cu_seqlens_q;
+    sh.cu_k = cu_seqlens_k;
+    sh.total_q = total_q;
+    sh.total_k = total_k;
+    return dispatch_dims(dqk, causal, true, q, k, v, out, lse, sh, scale, st);
 }
 
 extern "C" const char* attn_status_string(int status)

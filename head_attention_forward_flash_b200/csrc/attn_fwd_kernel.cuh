@@ -57,7 +57,13 @@ constexpr int kErrTimeout = 10;  // B200ATTN_ERR_TIMEOUT
 struct AttnParams {
     __nv_bfloat16* o;
     float* lse;  // may be null
+    // Dense: b batches of sq queries / sk keys. Packed sequences: b sequences, sq = the longest
+    // query length (it sizes the unit grid), sk unused; sequence i owns query rows
+    // cu_q[i] .. cu_q[i+1] and key rows cu_k[i] .. cu_k[i+1] of the packed tensors.
     int64_t b, hq, hk, sq, sk;
+    const int* cu_q;
+    const int* cu_k;
+    int64_t total_q, total_k;
     int64_t group;    // hq / hk
     int64_t n_qu;     // query units per (batch, head): ceil(sq / (NT * 128))
     int64_t n_units;  // b * hq * n_qu (below 2^31)
@@ -148,14 +154,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,
     }
 }
 
-// One work unit: (batch, query head, NT query tiles starting at row q0) and its key blocks.
+// One work unit: (batch or sequence, query head, NT query tiles starting at row q0 of the
+// sequence) and its key blocks.
 struct UnitInfo {
     int64_t bi, h, g, q0;
+    int64_t sq, sk;      // this sequence's query / key lengths
+    int64_t qrow, krow;  // its first query / key row in the tensor maps' row dimension
+    int64_t obase;       // O row of its query 0: O[(obase + i) * hq + h]
+    int64_t lbase;       // LSE of its query i at lse[lbase + i]
+    int bmap;            // the tensor maps' batch coordinate
     int n_blocks;   // key blocks with at least one allowed key for some row of the unit
     int mask_from;  // blocks >= mask_from need the per-key mask (causal diagonal, ragged tail)
 };
 
-template <int BN, int NT, bool CAUSAL>
+template <int BN, int NT, bool CAUSAL, bool VARLEN>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
 {
     UnitInfo t;
@@ -168,20 +180,49 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
     t.h = h;
     t.g = fast_div(h, p.div_group);
     t.q0 = qu * (NT * 128);
-    const int64_t n_kv = (p.sk + BN - 1) / BN;
+    if (VARLEN) {
+        // offsets clamped into the packed tensors, so no row outside them is ever addressed
+        int64_t qs = __ldg(p.cu_q + bi), qe = __ldg(p.cu_q + bi + 1);
+        int64_t ks = __ldg(p.cu_k + bi), ke = __ldg(p.cu_k + bi + 1);
+        qs = qs < 0 ? 0 : (qs > p.total_q ? p.total_q : qs);
+        qe = qe < qs ? qs : (qe > p.total_q ? p.total_q : qe);
+        ks = ks < 0 ? 0 : (ks > p.total_k ? p.total_k : ks);
+        ke = ke < ks ? ks : (ke > p.total_k ? p.total_k : ke);
+        t.sq = qe - qs;
+        t.sk = ke - ks;
+        t.qrow = qs;
+        t.krow = ks;
+        t.obase = qs;
+        t.lbase = (int64_t)h * p.total_q + qs;
+        t.bmap = 0;
+    } else {
+        t.sq = p.sq;
+        t.sk = p.sk;
+        t.qrow = 0;
+        t.krow = 0;
+        t.obase = (int64_t)bi * p.sq;
+        t.lbase = ((int64_t)bi * p.hq + h) * p.sq;
+        t.bmap = (int)bi;
+    }
+    if (t.q0 >= t.sq) {  // (packed sequences) no query row of this sequence here
+        t.n_blocks = 0;
+        t.mask_from = 0;
+        return t;
+    }
+    const int64_t n_kv = (t.sk + BN - 1) / BN;
     if (CAUSAL) {
-        const int64_t last_row = (t.q0 + NT * 128 - 1 < p.sq - 1) ? t.q0 + NT * 128 - 1 : p.sq - 1;
-        const int64_t last_key = last_row + p.sk - p.sq;
+        const int64_t last_row = (t.q0 + NT * 128 - 1 < t.sq - 1) ? t.q0 + NT * 128 - 1 : t.sq - 1;
+        const int64_t last_key = last_row + t.sk - t.sq;
         int64_t nb = last_key < 0 ? 0 : last_key / BN + 1;
         nb = nb < n_kv ? nb : n_kv;
-        const int64_t first_lim = t.q0 + p.sk - p.sq + 1;  // keys < first_lim: allowed for all
+        const int64_t first_lim = t.q0 + t.sk - t.sq + 1;  // keys < first_lim: allowed for all
         int64_t full = first_lim <= 0 ? 0 : first_lim / BN;
-        full = full < p.sk / BN ? full : p.sk / BN;
+        full = full < t.sk / BN ? full : t.sk / BN;
         t.n_blocks = (int)nb;
         t.mask_from = (int)(full < nb ? full : nb);
     } else {
         t.n_blocks = (int)n_kv;
-        t.mask_from = (int)(p.sk / BN);
+        t.mask_from = (int)(t.sk / BN);
     }
     return t;
 }
@@ -224,7 +265,7 @@ __device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, 
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <class T, bool CAUSAL>
+template <class T, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -233,6 +274,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 {
     constexpr int BN = T::BN;
     constexpr int NT = T::NT;
+    // O through the staging tile and TMA stores, except for packed sequences, where a store box
+    // could reach into the next sequence's rows
+    constexpr bool OTMA = T::O_TMA && !VARLEN;
     constexpr int NK = T::NK;
     constexpr int NV = T::NV;
     constexpr uint32_t FULL = 0xffffffffu;
@@ -312,7 +356,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     // First unit of this CTA's list (from u) with at least one key block, or -1.
     auto busy_from = [&](int64_t u) -> int64_t {
         for (; u < p.n_units; u += ustep)
-            if (unit_info<BN, NT, CAUSAL>(p, u).n_blocks > 0) return u;
+            if (unit_info<BN, NT, CAUSAL, VARLEN>(p, u).n_blocks > 0) return u;
         return -1;
     };
 
@@ -328,7 +372,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int q_cnt = 0;       // Q units issued
             bool ok = true;
             auto load_q = [&](int64_t u) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
                 if (!mbar_wait(bar_q_empty, (uint32_t)(q_cnt & 1) ^ 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
@@ -337,8 +381,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 for (int tt = 0; tt < NT; ++tt)
                     for (int ch = 0; ch < T::QCH; ++ch)
                         tma_load_4d(q_stage + tt * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES, &tmap_q,
-                                    bar_q_full, ch * 64, (int)t.h, (int)(t.q0 + tt * 128),
-                                    (int)t.bi);
+                                    bar_q_full, ch * 64, (int)t.h,
+                                    (int)(t.qrow + t.q0 + tt * 128), t.bmap);
                 ++q_cnt;
             };
             auto load_k = [&](const UnitInfo& t, int j) {
@@ -352,7 +396,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 mbar_arrive_expect_tx(bar_kfull(slot), T::K_TILE_BYTES);
                 for (int ch = 0; ch < T::QCH; ++ch)
                     tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_k, bar_kfull(slot), ch * 64,
-                                (int)t.g, j * BN, (int)t.bi);
+                                (int)t.g, (int)(t.krow + (int64_t)j * BN), t.bmap);
                 ++kq;
             };
             auto load_v = [&](const UnitInfo& t, int j) {
@@ -366,7 +410,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 mbar_arrive_expect_tx(bar_vfull(slot), T::V_TILE_BYTES);
                 for (int ch = 0; ch < T::VCH; ++ch)
                     tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_v, bar_vfull(slot), ch * 64,
-                                (int)t.g, j * BN, (int)t.bi);
+                                (int)t.g, (int)(t.krow + (int64_t)j * BN), t.bmap);
                 ++vq;
             };
             bool pend = false;  // the P V step still owed for the previous item
@@ -375,7 +419,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int64_t u = busy_from(u0);
             if (u >= 0) load_q(u);
             while (u >= 0 && ok) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
                 const int64_t un = busy_from(u + ustep);
                 for (int j = 0; j < t.n_blocks && ok; ++j) {
                     for (int tt = 0; tt < NT && ok; ++tt) {
@@ -480,7 +524,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int pend_j = 0, pend_tt = 0, pend_u = 0;
             int64_t pend_g = 0;
             for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
                 if (t.n_blocks == 0) continue;
                 if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
                     if (!mbar_wait(bar_q_full, (uint32_t)(units & 1), wc, kErrTimeout)) {
@@ -561,9 +605,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 return false;
             tc_fence_after_sync();
             const int64_t i = t.q0 + tt * 128 + row;
-            const bool row_valid = i < p.sq;
+            const bool row_valid = i < t.sq;
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            if constexpr (T::O_TMA) {
+            if constexpr (OTMA) {
                 // This warp's 32 rows go to its own slab of the staging tile (one 32-row, 128-byte
                 // swizzled box per 64 columns), then one lane stores the slab with TMA; rows past
                 // sq are clipped by the tensor map. The slab is reused only after the previous
@@ -597,16 +641,16 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 const int64_t row0 = t.q0 + tt * 128 + w4 * 32;
-                if (lane == 0 && row0 < p.sq) {
+                if (lane == 0 && row0 < t.sq) {
 #pragma unroll
                     for (int bx = 0; bx < T::DV / 64; ++bx)
                         tma_store_4d(&tmap_o, sbase + T::O_OFF + T::o_slab(tt, bx, w4), bx * 64,
-                                     (int)t.h, (int)row0, (int)t.bi);
+                                     (int)t.h, (int)(t.qrow + row0), t.bmap);
                     bulk_commit_group();
                 }
             } else {
                 uint4* dst = reinterpret_cast<uint4*>(
-                    p.o + ((t.bi * p.sq + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
+                    p.o + ((t.obase + (row_valid ? i : 0)) * p.hq + t.h) * T::DV);
 #pragma unroll 1
                 for (int c = 0; c < T::DV / 32; ++c) {
                     uint32_t r[32];
@@ -631,7 +675,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
             }
             if (row_valid && p.lse)
-                p.lse[(t.bi * p.hq + t.h) * p.sq + i] =
+                p.lse[t.lbase + i] =
                     l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
             return true;
         };
@@ -645,17 +689,17 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         if (T::Q_TMEM && busy_from(u0) >= 0)
             for (int k = 0; k < NTW && ok; ++k) ok = copy_q(0, tile_of(k));
         for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
-            const UnitInfo t = unit_info<BN, NT, CAUSAL>(p, u);
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
             if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
 #pragma unroll
                 for (int k = 0; k < NTW; ++k) {
                     const int64_t i = t.q0 + tile_of(k) * 128 + row;
-                    if (i < p.sq) {
+                    if (i < t.sq) {
                         uint4* dst = reinterpret_cast<uint4*>(
-                            p.o + ((t.bi * p.sq + i) * p.hq + t.h) * T::DV);
+                            p.o + ((t.obase + i) * p.hq + t.h) * T::DV);
 #pragma unroll 1
                         for (int c = 0; c < T::DV / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                        if (p.lse) p.lse[(t.bi * p.hq + t.h) * p.sq + i] = -INFINITY;
+                        if (p.lse) p.lse[t.lbase + i] = -INFINITY;
                     }
                 }
                 continue;
@@ -667,8 +711,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k < NTW; ++k) {
                 const int64_t i = t.q0 + tile_of(k) * 128 + row;
-                const int64_t lim_row = CAUSAL ? i + p.sk - p.sq : p.sk - 1;
-                lim[k] = lim_row < p.sk - 1 ? lim_row : p.sk - 1;
+                const int64_t lim_row = CAUSAL ? i + t.sk - t.sq : t.sk - 1;
+                lim[k] = lim_row < t.sk - 1 ? lim_row : t.sk - 1;
                 m_ref[k] = -INFINITY;
                 l[k] = 0.f;
             }
@@ -818,7 +862,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             for (int k = 0; k < NTW && ok; ++k)
                 ok = epilogue(pend_t, tile_of(k), pend_m[k], pend_l[k], pend_idx);
         // every O store this warp issued is complete before the CTA exits
-        if (T::O_TMA && lane == 0) bulk_wait_all();
+        if (OTMA && lane == 0) bulk_wait_all();
     }
 
     // ---- teardown: every tcgen05 access is complete (MMAs drained, loads waited) ----

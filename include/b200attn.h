@@ -83,6 +83,40 @@ B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out
              int causal, float scale, void* stream);
 
 /*
+ * attn_fwd_varlen -- attn_fwd over b packed sequences of different lengths.
+ *
+ * Sequence i (i < b) owns query rows cu_seqlens_q[i] .. cu_seqlens_q[i+1]-1 of q / out and key
+ * rows cu_seqlens_k[i] .. cu_seqlens_k[i+1]-1 of k / v; with sq_i, sk_i its lengths, every
+ * query row r = i0 + i of it gets attn_fwd's result for its own sequence alone (same J with
+ * sq_i, sk_i in place of sq, sk -- bottom-right causal alignment per sequence; an empty J
+ * gives O = 0, LSE = -inf). This is the "varlen" layout of the shape tables of "Tune MHA config
+ * & small-head pipeline pathology" (Source of shapes; the varlen rows after Final status),
+ * which print no packing convention; this is the usual one (cumulative offsets, one entry per
+ * sequence boundary).
+ *
+ *   q        device bf16 [total_q, hq, dqk];  k: [total_k, hk, dqk];  v: [total_k, hk, dv].
+ *   out      device bf16 [total_q, hq, dv]. Rows of every sequence are written; rows that
+ *            belong to no sequence are left unchanged.
+ *   lse      device fp32 [hq, total_q] (head-major), or NULL.
+ *   cu_seqlens_q, cu_seqlens_k  device int32 [b + 1], 4-byte aligned, non-decreasing row
+ *            offsets into the packed tensors (usually 0 .. total_q / total_k; rows outside
+ *            [cu[0], cu[b]) belong to no sequence). Read by the kernel only (the host never
+ *            dereferences them). Offsets outside [0, total] are clamped into it, so no row
+ *            outside the tensors is ever addressed.
+ *   max_sq   at least the longest query length (it sizes the grid); query rows of a sequence
+ *            beyond max_sq are not computed.
+ *   b, total_q, max_sq  may be 0 (nothing is launched); total_k may be 0 (every row empty).
+ *   hk, hq, dqk, dv, causal, scale  as in attn_fwd.
+ * Errors as attn_fwd; also ERR_RANGE when total_q, total_k or b * hq * ceil(max_sq / 128)
+ * reaches 2^31. Allocates nothing. Safe to call concurrently on different streams.
+ */
+B200ATTN_API int attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
+                                 const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                                 int64_t b, int64_t hq, int64_t hk, int64_t total_q,
+                                 int64_t total_k, int64_t max_sq, int64_t dqk, int64_t dv,
+                                 int causal, float scale, void* stream);
+
+/*
  * k_smooth_mean -- fp32 channel mean of K over its sequence axis.
  *     mean[bi,g,c] = (1/sk) * sum_{s < sk} K[bi,s,g,c]
  * The per-(batch, head) moments of K over its key axis, folded per head in a fixed order, that

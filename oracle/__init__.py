@@ -118,6 +118,35 @@ def attn_full(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, nthreads=None,
     return o, lse
 
 
+def attn_varlen(q, k, v, cu_q, cu_k, hq, hk, dqk, dv, causal, scale, nthreads=None, lib=None):
+    """Packed sequences: O (fp64 [total_q, hq, dv]) and LSE (fp64 [hq, total_q]).
+
+    Sequence i is the dense problem on its own query rows cu_q[i] .. cu_q[i+1]-1 and key rows
+    cu_k[i] .. cu_k[i+1]-1 -- the "varlen" layout of the shape tables of "Tune MHA config &
+    small-head pipeline pathology" (Source of shapes; varlen rows after Final status), read as
+    independent sequences packed along the row axis. Each sequence goes to attn_full with b = 1.
+    Rows that belong to no sequence are NaN.
+    """
+    q = _u16(q).reshape(-1, hq, dqk)
+    k = _u16(k).reshape(-1, hk, dqk)
+    v = _u16(v).reshape(-1, hk, dv)
+    total_q = q.shape[0]
+    o = np.full((total_q, hq, dv), np.nan)
+    lse = np.full((hq, total_q), np.nan)
+    cu_q = [int(x) for x in cu_q]
+    cu_k = [int(x) for x in cu_k]
+    for i in range(len(cu_q) - 1):
+        qs, qe, ks, ke = cu_q[i], cu_q[i + 1], cu_k[i], cu_k[i + 1]
+        if qe <= qs:
+            continue
+        oi, li = attn_full(np.ascontiguousarray(q[qs:qe]), np.ascontiguousarray(k[ks:ke]),
+                           np.ascontiguousarray(v[ks:ke]), 1, hq, hk, qe - qs, ke - ks, dqk, dv,
+                           causal, scale, nthreads=nthreads, lib=lib)
+        o[qs:qe] = oi[0]
+        lse[:, qs:qe] = li[0]
+    return o, lse
+
+
 def k_mean(k, b, hk, sk, d, lib=None):
     """Channel mean of K over the sequence: (fp64 [b,hk,d], its fp32 rounding [b,hk,d])."""
     lib = lib or load_library()

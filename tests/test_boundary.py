@@ -77,3 +77,30 @@ def test_k_mean_rejects(fn):
     if fn == "k_smooth_sub":
         assert f(A, A, None, 1, 2, 8, 64, None) == 1
         assert f(A, A, A + 2, 1, 2, 8, 64, None) == 5
+
+
+def call_varlen(q=A, k=A, v=A, o=A, lse=A, cq=A, ck=A, b=2, hq=2, hk=1, tq=32, tk=32, max_sq=16,
+                dqk=64, dv=64, causal=0, scale=0.125):
+    return b2.lib.attn_fwd_varlen(q, k, v, o, lse, cq, ck, b, hq, hk, tq, tk, max_sq, dqk, dv,
+                                  causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b=-1), 2), (dict(tq=-1), 2), (dict(tk=-5), 2), (dict(max_sq=-1), 2), (dict(hk=0), 2),
+    (dict(hq=3, hk=2), 3), (dict(dqk=128, dv=64), 4), (dict(dqk=32, dv=32), 4),
+    (dict(scale=float("nan")), 7),
+    (dict(q=None), 1), (dict(o=None), 1), (dict(k=None), 1), (dict(v=None), 1),
+    (dict(cq=None), 1), (dict(ck=None), 1),
+    (dict(q=A + 8), 5), (dict(v=A + 2), 5), (dict(lse=A + 2), 5), (dict(cq=A + 2), 5),
+    (dict(ck=A + 1), 5),
+    (dict(tq=1 << 31), 6), (dict(tk=1 << 31), 6), (dict(b=1 << 20, hq=1 << 10, hk=1, max_sq=1 << 10), 6),
+])
+def test_attn_fwd_varlen_rejects(kw, code):
+    assert call_varlen(**kw) == code
+
+
+def test_varlen_empty_problem_is_a_no_op():
+    # no sequence, no query row or a zero longest length: nothing is computed or touched
+    assert call_varlen(b=0, q=None, k=None, v=None, o=None, lse=None, cq=None, ck=None) == 0
+    assert call_varlen(tq=0, q=None, o=None, lse=None, cq=None, ck=None) == 0
+    assert call_varlen(max_sq=0, q=None, o=None, lse=None, cq=None, ck=None) == 0

@@ -29,6 +29,11 @@ CONFIGS = {
             dqk=256, dv=256, causal=False, kmean=True),
     5: dict(workload="long_b1_h5_s65536_d128_causal", b=1, hq=5, hk=5, sq=65536, sk=65536,
             dqk=128, dv=128, causal=True, kmean=False),
+    # Packed sequences (the "varlen" layout of the pages' shape tables, e.g. 2048^2 d64 48/8
+    # varlen): b sequences whose lengths are drawn uniformly from [min_s, sq] (seed 3000 + id),
+    # each sequence's query and key lengths equal; sq / sk hold the longest possible length.
+    6: dict(workload="varlen_b8_hq48_hk8_s1024to2048_d64_causal", b=8, hq=48, hk=8, sq=2048,
+            sk=2048, min_s=1024, dqk=64, dv=64, causal=True, kmean=False, varlen=True),
 }
 
 HEAD_DIMS = ((64, 64), (128, 128), (192, 128), (256, 256))
@@ -44,9 +49,39 @@ def config(n: int) -> dict:
 
 
 def flops(c: dict) -> float:
-    """Algorithmic FLOPs of one forward pass: 2*b*hq*sq*sk*(dqk+dv), halved when causal."""
-    f = 2.0 * c["b"] * c["hq"] * c["sq"] * c["sk"] * (c["dqk"] + c["dv"])
+    """Algorithmic FLOPs of one forward pass: 2*b*hq*sq*sk*(dqk+dv), halved when causal (for
+    packed sequences, the sum of that over the sequences)."""
+    if c.get("varlen"):
+        lengths = varlen_lengths(c)
+        f = sum(2.0 * c["hq"] * n * n * (c["dqk"] + c["dv"]) for n in lengths)
+    else:
+        f = 2.0 * c["b"] * c["hq"] * c["sq"] * c["sk"] * (c["dqk"] + c["dv"])
     return f / 2.0 if c["causal"] else f
+
+
+def varlen_lengths(c: dict) -> list:
+    """The sequence lengths of a packed-sequence workload (query length = key length)."""
+    g = torch.Generator(device="cpu").manual_seed(3000 + int(c.get("id", 0)))
+    return [int(x) for x in torch.randint(c["min_s"], c["sq"] + 1, (c["b"],), generator=g)]
+
+
+def make_varlen_inputs(lengths_q, lengths_k, hq, hk, dqk, dv, seed):
+    """Packed Q [sum lengths_q, hq, dqk], K, V [sum lengths_k, hk, d] (bf16, CPU) drawn from
+    ``seed`` in the order Q, K, V, and the int32 offsets cu_q, cu_k (b + 1 entries each)."""
+    g = torch.Generator(device="cpu").manual_seed(int(seed))
+    f32 = torch.float32
+    tq, tk = int(sum(lengths_q)), int(sum(lengths_k))
+    q = torch.randn((tq, hq, dqk), generator=g, dtype=f32).to(torch.bfloat16)
+    k = torch.randn((tk, hk, dqk), generator=g, dtype=f32).to(torch.bfloat16)
+    v = torch.randn((tk, hk, dv), generator=g, dtype=f32).to(torch.bfloat16)
+    cu_q = torch.tensor([0] + list(lengths_q), dtype=torch.int64).cumsum(0).to(torch.int32)
+    cu_k = torch.tensor([0] + list(lengths_k), dtype=torch.int64).cumsum(0).to(torch.int32)
+    return q, k, v, cu_q, cu_k
+
+
+def config_varlen_inputs(c: dict):
+    lengths = varlen_lengths(c)
+    return make_varlen_inputs(lengths, lengths, c["hq"], c["hk"], c["dqk"], c["dv"], c["seed"])
 
 
 def make_inputs(b, hq, hk, sq, sk, dqk, dv, seed, kmean=False):
