@@ -51,6 +51,12 @@ def _bind(lib):
     lib.oracle_attn_full.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
                                                                _p, _p, ctypes.c_int]
     lib.oracle_attn_full.restype = ctypes.c_int
+    lib.oracle_attn_rows_ex.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
+                                        _i64, _p, _p, _i64, _p, _p, ctypes.c_int]
+    lib.oracle_attn_rows_ex.restype = ctypes.c_int
+    lib.oracle_attn_full_ex.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
+                                        _i64, _p, _p, _p, ctypes.c_int]
+    lib.oracle_attn_full_ex.restype = ctypes.c_int
     lib.oracle_k_mean.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p]
     lib.oracle_k_mean.restype = ctypes.c_int
     lib.oracle_k_sub.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i64]
@@ -89,30 +95,50 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def attn_rows(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, rows, nthreads=None, lib=None):
-    """O (fp64 [nrows, dv]) and LSE (fp64 [nrows]) for the (batch, head, query) triples in rows."""
+def _sinks(sinks, hq):
+    if sinks is None:
+        return None
+    s = np.ascontiguousarray(np.asarray(sinks, dtype=np.float64).reshape(-1))
+    if s.shape[0] != hq:
+        raise ValueError("sinks must hold one logit per query head")
+    return s
+
+
+def attn_rows(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, rows, nthreads=None, lib=None,
+              window=-1, sinks=None):
+    """O (fp64 [nrows, dv]) and LSE (fp64 [nrows]) for the (batch, head, query) triples in rows.
+
+    window >= 0 limits row i to keys j >= i + sk - sq - window; sinks (one logit per query head)
+    join each row's softmax denominator (see attn_oracle.c)."""
     lib = lib or load_library()
     q, k, v = _u16(q), _u16(k), _u16(v)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     n = rows.shape[0]
     o = np.zeros((n, dv), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    rc = lib.oracle_attn_rows(_ptr(q), _ptr(k), _ptr(v), b, hq, hk, sq, sk, dqk, dv, int(causal),
-                              float(scale), _ptr(rows), n, _ptr(o), _ptr(lse),
-                              int(nthreads or default_threads()))
+    sk_arr = _sinks(sinks, hq)
+    rc = lib.oracle_attn_rows_ex(_ptr(q), _ptr(k), _ptr(v), b, hq, hk, sq, sk, dqk, dv,
+                                 int(causal), float(scale), int(window),
+                                 _ptr(sk_arr) if sk_arr is not None else None, _ptr(rows), n,
+                                 _ptr(o), _ptr(lse), int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_attn_rows failed with code {rc}")
     return o, lse
 
 
-def attn_full(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, nthreads=None, lib=None):
-    """O (fp64 BSHD [b,sq,hq,dv]) and LSE (fp64 [b,hq,sq]) for every row."""
+def attn_full(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, nthreads=None, lib=None,
+              window=-1, sinks=None):
+    """O (fp64 BSHD [b,sq,hq,dv]) and LSE (fp64 [b,hq,sq]) for every row (window and sinks as
+    in attn_rows)."""
     lib = lib or load_library()
     q, k, v = _u16(q), _u16(k), _u16(v)
     o = np.zeros((b, sq, hq, dv), dtype=np.float64)
     lse = np.zeros((b, hq, sq), dtype=np.float64)
-    rc = lib.oracle_attn_full(_ptr(q), _ptr(k), _ptr(v), b, hq, hk, sq, sk, dqk, dv, int(causal),
-                              float(scale), _ptr(o), _ptr(lse), int(nthreads or default_threads()))
+    sk_arr = _sinks(sinks, hq)
+    rc = lib.oracle_attn_full_ex(_ptr(q), _ptr(k), _ptr(v), b, hq, hk, sq, sk, dqk, dv,
+                                 int(causal), float(scale), int(window),
+                                 _ptr(sk_arr) if sk_arr is not None else None, _ptr(o), _ptr(lse),
+                                 int(nthreads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_attn_full failed with code {rc}")
     return o, lse

@@ -19,6 +19,15 @@
  *     LSE[bi,h,i]  = m + ln(l)
  *   An empty J gives O = 0 and LSE = -inf.
  *
+ * Sliding window and attention sink (the "GPT-OSS sink+sliding-window" shapes of "Tune MHA
+ * config & small-head pipeline pathology", Source of shapes; the pages define neither, and
+ * this is the usual reading -- a left window relative to the row's diagonal key, and a
+ * per-head logit that joins the softmax denominator without a value):
+ *     J      = J  intersected with  { j >= i + sk - sq - window }     (window >= 0)
+ *     with sink sigma_h:  m = max(max_J s_j, sigma_h),
+ *                         l = sum_J exp(s_j - m) + exp(sigma_h - m),
+ *     O and LSE as above; an empty J then gives O = 0 and LSE = sigma_h.
+ *
  * K channel mean ("[HIP] Mha v4: run the K-smoothing gate as one HIP call", Summary and the
  * commit message: per-(batch*head) moments of K over its key axis, folded per head):
  *     mean[bi,g,c] = (1/sk) * sum_s K[bi,s,g,c]      (fp64 sum, rounded once to fp32)
@@ -73,6 +82,8 @@ typedef struct {
     int64_t b, hq, hk, sq, sk, dqk, dv;
     int causal;
     double scale;
+    int64_t window;       /* left window (keys before the diagonal), < 0: none */
+    const double *sinks;  /* per query head sink logit, or NULL */
     const int64_t *rows; /* nrows triples (bi, h, i), or NULL for every row in BSHD order */
     int64_t nrows;
     double *o, *lse;
@@ -86,21 +97,24 @@ static void attn_row(const attn_job *a, int64_t bi, int64_t h, int64_t i, double
 {
     int64_t group = a->hq / a->hk;
     int64_t g = h / group;
-    int64_t n = a->sk; /* keys 0 .. n-1 are allowed */
-    if (a->causal) {
-        int64_t last = i + a->sk - a->sq;
-        if (last + 1 < n) n = last + 1;
-    }
-    if (n <= 0) {
+    const int64_t diag = i + a->sk - a->sq; /* the row's diagonal key */
+    int64_t hi = a->sk - 1;                 /* allowed keys: lo .. hi */
+    if (a->causal && diag < hi) hi = diag;
+    int64_t lo = 0;
+    if (a->window >= 0 && diag - a->window > lo) lo = diag - a->window;
+    const int has_sink = a->sinks != NULL;
+    const double sink = has_sink ? a->sinks[h] : 0.0;
+    if (hi < lo) {
         for (int64_t c = 0; c < a->dv; ++c) o_row[c] = 0.0;
-        *lse_out = -INFINITY;
+        *lse_out = has_sink ? sink : -INFINITY;
         return;
     }
+    const int64_t n = hi - lo + 1;
     const uint16_t *qrow = a->q + ((bi * a->sq + i) * a->hq + h) * a->dqk;
     for (int64_t c = 0; c < a->dqk; ++c) qd[c] = bf16_value(qrow[c]);
 
     for (int64_t j = 0; j < n; ++j) {
-        const uint16_t *krow = a->k + ((bi * a->sk + j) * a->hk + g) * a->dqk;
+        const uint16_t *krow = a->k + ((bi * a->sk + lo + j) * a->hk + g) * a->dqk;
         double dot = 0.0;
         for (int64_t c = 0; c < a->dqk; ++c) dot += qd[c] * bf16_value(krow[c]);
         s[j] = a->scale * dot;
@@ -108,14 +122,16 @@ static void attn_row(const attn_job *a, int64_t bi, int64_t h, int64_t i, double
     double m = s[0];
     for (int64_t j = 1; j < n; ++j)
         if (s[j] > m) m = s[j];
+    if (has_sink && sink > m) m = sink;
     double l = 0.0;
     for (int64_t j = 0; j < n; ++j) {
         s[j] = exp(s[j] - m); /* s now holds the unnormalised weights */
         l += s[j];
     }
+    if (has_sink) l += exp(sink - m);
     for (int64_t c = 0; c < a->dv; ++c) o_row[c] = 0.0;
     for (int64_t j = 0; j < n; ++j) {
-        const uint16_t *vrow = a->v + ((bi * a->sk + j) * a->hk + g) * a->dv;
+        const uint16_t *vrow = a->v + ((bi * a->sk + lo + j) * a->hk + g) * a->dv;
         for (int64_t c = 0; c < a->dv; ++c) o_row[c] += s[j] * bf16_value(vrow[c]);
     }
     for (int64_t c = 0; c < a->dv; ++c) o_row[c] /= l;
@@ -187,17 +203,40 @@ static int run_attn(attn_job *a, int nthreads)
     return rc;
 }
 
-/* Selected rows: rows[3r..3r+2] = (bi, h, i); o is [nrows, dv], lse is [nrows]. */
+/* Selected rows with a left window (< 0: none) and per-head sinks (NULL: none):
+ * rows[3r..3r+2] = (bi, h, i); o is [nrows, dv], lse is [nrows]. */
+int oracle_attn_rows_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t b,
+                        int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                        int causal, double scale, int64_t window, const double *sinks,
+                        const int64_t *rows, int64_t nrows, double *o, double *lse, int nthreads)
+{
+    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, window, sinks, rows,
+                  nrows, o, lse};
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[3 * r] < 0 || rows[3 * r] >= b || rows[3 * r + 1] < 0 ||
+            rows[3 * r + 1] >= hq || rows[3 * r + 2] < 0 || rows[3 * r + 2] >= sq)
+            return 2;
+    return run_attn(&a, nthreads);
+}
+
+/* Selected rows, no window, no sink. */
 int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t b,
                      int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
                      int causal, double scale, const int64_t *rows, int64_t nrows, double *o,
                      double *lse, int nthreads)
 {
-    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, rows, nrows, o, lse};
-    for (int64_t r = 0; r < nrows; ++r)
-        if (rows[3 * r] < 0 || rows[3 * r] >= b || rows[3 * r + 1] < 0 ||
-            rows[3 * r + 1] >= hq || rows[3 * r + 2] < 0 || rows[3 * r + 2] >= sq)
-            return 2;
+    return oracle_attn_rows_ex(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, -1, NULL,
+                               rows, nrows, o, lse, nthreads);
+}
+
+/* Every row, with a left window (< 0: none) and per-head sinks (NULL: none). */
+int oracle_attn_full_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t b,
+                        int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                        int causal, double scale, int64_t window, const double *sinks, double *o,
+                        double *lse, int nthreads)
+{
+    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, window, sinks, NULL,
+                  b * sq * hq, o, lse};
     return run_attn(&a, nthreads);
 }
 
@@ -206,8 +245,8 @@ int oracle_attn_full(const uint16_t *q, const uint16_t *k, const uint16_t *v, in
                      int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
                      int causal, double scale, double *o, double *lse, int nthreads)
 {
-    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, NULL, b * sq * hq, o, lse};
-    return run_attn(&a, nthreads);
+    return oracle_attn_full_ex(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, -1, NULL, o,
+                               lse, nthreads);
 }
 
 /* Channel mean of K over its sequence axis: mean64/mean32 are [b,hk,d]. */

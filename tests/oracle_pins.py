@@ -291,7 +291,99 @@ def pin_rows_api(lib):
         assert np.array_equal(o_r[n], o[bi, i, h]) and lse_r[n] == lse[bi, h, i]
 
 
+def _band_keep(sq, sk, causal, window):
+    """Allowed (i, j): j <= i + sk - sq when causal, j >= i + sk - sq - window when window >= 0."""
+    i = torch.arange(sq)[:, None]
+    j = torch.arange(sk)[None, :]
+    keep = torch.ones(sq, sk, dtype=torch.bool)
+    if causal:
+        keep &= j <= i + (sk - sq)
+    if window >= 0:
+        keep &= j >= i + (sk - sq) - window
+    return keep
+
+
+def _brute_force_window_sink(q, k, v, hq, hk, sq, sk, causal, scale, window, sinks):
+    """fp64 full-matrix softmax with a band mask and an extra sink column per head (numpy),
+    written independently of the oracle: O [b,sq,hq,dv], LSE [b,hq,sq]."""
+    Q = q.double().permute(0, 2, 1, 3).numpy()
+    K = k.double().permute(0, 2, 1, 3).repeat_interleave(hq // hk, dim=1).numpy()
+    V = v.double().permute(0, 2, 1, 3).repeat_interleave(hq // hk, dim=1).numpy()
+    S = np.einsum("bhid,bhjd->bhij", Q, K) * scale
+    keep = _band_keep(sq, sk, causal, window).numpy()
+    S = np.where(keep[None, None], S, -np.inf)
+    if sinks is not None:
+        col = np.broadcast_to(np.asarray(sinks, np.float64)[None, :, None, None],
+                              S.shape[:3] + (1,))
+        S = np.concatenate([S, col], axis=-1)
+        V = np.concatenate([V, np.zeros(V.shape[:2] + (1, V.shape[3]))], axis=2)
+    m = np.max(S, axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(S - m)
+    l = np.sum(w, axis=-1, keepdims=True)
+    with np.errstate(invalid="ignore", divide="ignore"):
+        O = np.where(l > 0, np.einsum("bhij,bhjd->bhid", w, V) / np.where(l > 0, l, 1.0), 0.0)
+        L = np.where(l[..., 0] > 0, m[..., 0] + np.log(np.where(l[..., 0] > 0, l[..., 0], 1.0)),
+                     -np.inf)
+    return O.transpose(0, 2, 1, 3), L
+
+
+def pin_window_brute_force(lib):
+    """Sliding window (with and without the causal bound, windows 0 .. past sk) == the numpy
+    band-masked full softmax; sq != sk exercises the diagonal offset."""
+    b, hq, hk, sq, sk, d = 1, 4, 2, 9, 13, 64
+    q, k, v = make_inputs(b, hq, hk, sq, sk, d, d, seed=41)
+    for causal in (False, True):
+        for window in (0, 1, 3, 7, 20):
+            o, l = oracle.attn_full(bf16_bits(q), bf16_bits(k), bf16_bits(v), b, hq, hk, sq, sk,
+                                    d, d, causal, 0.2, nthreads=2, lib=lib, window=window)
+            o_ref, l_ref = _brute_force_window_sink(q, k, v, hq, hk, sq, sk, causal, 0.2, window,
+                                                    None)
+            assert np.max(np.abs(o - o_ref)) < 1e-12
+            assert np.array_equal(np.isneginf(l), np.isneginf(l_ref))
+            fin = np.isfinite(l_ref)
+            assert np.max(np.abs(l[fin] - l_ref[fin])) < 1e-12
+
+
+def pin_window_zero_is_the_diagonal(lib):
+    """Causal with window 0: every row sees only its diagonal key, so O is that key's V row
+    exactly and LSE is that key's scaled score."""
+    b, hq, hk, s, d = 1, 2, 2, 6, 64
+    q, k, v = make_inputs(b, hq, hk, s, s, d, d, seed=43)
+    o, l = oracle.attn_full(bf16_bits(q), bf16_bits(k), bf16_bits(v), b, hq, hk, s, s, d, d, True,
+                            0.3, nthreads=2, lib=lib, window=0)
+    vd, qd, kd = v.double().numpy(), q.double().numpy(), k.double().numpy()
+    for h in range(hq):
+        for i in range(s):
+            assert np.array_equal(o[0, i, h], vd[0, i, h])
+            assert abs(l[0, h, i] - 0.3 * float(np.dot(qd[0, i, h], kd[0, i, h]))) < 1e-12
+
+
+def pin_sink_closed_form(lib):
+    """A sink logit sigma joins the denominator: LSE_sink = logaddexp(LSE, sigma) and
+    O_sink = O * exp(LSE - LSE_sink), exactly; rows with no allowed key give O = 0 and
+    LSE = sigma; the numpy brute force with a sink column agrees."""
+    b, hq, hk, sq, sk, d = 2, 4, 2, 11, 7, 64  # sq > sk: causal rows 0..3 have no key
+    q, k, v = make_inputs(b, hq, hk, sq, sk, d, d, seed=47)
+    sinks = np.array([-1.5, 0.0, 2.25, 30.0])
+    for causal in (False, True):
+        o0, l0 = oracle.attn_full(bf16_bits(q), bf16_bits(k), bf16_bits(v), b, hq, hk, sq, sk, d,
+                                  d, causal, 0.125, nthreads=2, lib=lib)
+        o1, l1 = oracle.attn_full(bf16_bits(q), bf16_bits(k), bf16_bits(v), b, hq, hk, sq, sk, d,
+                                  d, causal, 0.125, nthreads=2, lib=lib, sinks=sinks)
+        expect_l = np.logaddexp(l0, sinks[None, :, None])
+        assert np.max(np.abs(l1 - expect_l)) < 1e-12
+        scale_o = np.exp(l0 - expect_l).transpose(0, 2, 1)[..., None]  # [b, sq, hq, 1]
+        assert np.max(np.abs(o1 - o0 * np.where(np.isfinite(scale_o), scale_o, 0.0))) < 1e-12
+        o_ref, l_ref = _brute_force_window_sink(q, k, v, hq, hk, sq, sk, causal, 0.125, -1, sinks)
+        assert np.max(np.abs(o1 - o_ref)) < 1e-12 and np.max(np.abs(l1 - l_ref)) < 1e-12
+        if causal:
+            assert np.all(o1[:, :4] == 0.0)
+            assert np.array_equal(l1[:, :, :4], np.broadcast_to(sinks[None, :, None], (b, hq, 4)))
+
+
 ALL_PINS = [pin_sdpa, pin_uniform_scores, pin_causal_row0_and_single_key, pin_two_keys, pin_large_scores,
             pin_gqa_replication, pin_permutation_and_independence, pin_convexity,
             pin_fully_masked_rows, pin_kmean_shift_identity, pin_k_mean, pin_bf16_rne,
-            pin_rows_api]
+            pin_rows_api, pin_window_brute_force, pin_window_zero_is_the_diagonal,
+            pin_sink_closed_form]

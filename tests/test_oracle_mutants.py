@@ -1,6 +1,7 @@
 """Mutation check of the oracle's pins: plausible mistakes planted in a copy of the oracle's
 C source (a dropped scale, a wrong GQA head map, a causal off-by-one, a transposed V stride, a
-missing normalisation, a wrong LSE, a wrong mean divisor, a wrong rounding mode) must each be
+missing normalisation, a wrong LSE, a wrong mean divisor, a wrong rounding mode, a window
+off-by-one or a dropped window, a sink left out of the denominator or of an empty row) must each be
 caught by at least one pin. The planted copies are built in a temporary directory on the CPU;
 the real oracle is untouched."""
 import os
@@ -14,9 +15,13 @@ from oracle_pins import ALL_PINS
 MUTANTS = {
     "dropped_scale": ("s[j] = a->scale * dot;", "s[j] = dot;"),
     "gqa_modulo_map": ("int64_t g = h / group;", "int64_t g = h % a->hk;"),
-    "causal_off_by_one": ("int64_t last = i + a->sk - a->sq;", "int64_t last = i + a->sk - a->sq - 1;"),
-    "causal_top_left": ("int64_t last = i + a->sk - a->sq;", "int64_t last = i;"),
-    "v_stride_dqk": ("((bi * a->sk + j) * a->hk + g) * a->dv;", "((bi * a->sk + j) * a->hk + g) * a->dqk;"),
+    "causal_off_by_one": ("const int64_t diag = i + a->sk - a->sq;", "const int64_t diag = i + a->sk - a->sq - 1;"),
+    "causal_top_left": ("const int64_t diag = i + a->sk - a->sq;", "const int64_t diag = i;"),
+    "v_stride_dqk": ("((bi * a->sk + lo + j) * a->hk + g) * a->dv;", "((bi * a->sk + lo + j) * a->hk + g) * a->dqk;"),
+    "window_off_by_one": ("diag - a->window > lo) lo = diag - a->window;", "diag - a->window > lo) lo = diag - a->window + 1;"),
+    "window_ignored": ("if (a->window >= 0 && diag", "if (0 && diag"),
+    "sink_left_out_of_sum": ("if (has_sink) l += exp(sink - m);", "if (0) l += exp(sink - m);"),
+    "empty_row_ignores_sink": ("*lse_out = has_sink ? sink : -INFINITY;", "*lse_out = -INFINITY;"),
     "no_normalisation": ("o_row[c] /= l;", "o_row[c] /= 1.0;"),
     "lse_without_max": ("*lse_out = m + log(l);", "*lse_out = log(l);"),
     "mean_divisor": ("double mean = sum / (double)sk;", "double mean = sum / (double)(sk - 1);"),
