@@ -69,8 +69,10 @@ def _row_flops(c, rows):
     """Algorithmic FLOPs of the given output rows: 2 * |allowed keys| * (dqk + dv) each."""
     total = 0
     for (_, _, i) in rows:
-        n = min(c["sk"], int(i) + c["sk"] - c["sq"] + 1) if c["causal"] else c["sk"]
-        total += 2 * max(n, 0) * (c["dqk"] + c["dv"])
+        d = int(i) + c["sk"] - c["sq"]
+        hi = min(c["sk"] - 1, d) if c["causal"] else c["sk"] - 1
+        lo = max(0, d - c["window"]) if c.get("window") is not None else 0
+        total += 2 * max(hi - lo + 1, 0) * (c["dqk"] + c["dv"])
     return float(total)
 
 
@@ -103,9 +105,12 @@ class OracleSampler:
         rows = self.rows[idx]
         c = self.c
         t0 = time.perf_counter()
+        sk_logits = workloads.sinks(c)
         self.oracle.attn_rows(self.qb, self.kb, self.vb, c["b"], c["hq"], c["hk"], c["sq"],
                               c["sk"], c["dqk"], c["dv"], c["causal"], c["scale"], rows,
-                              nthreads=self.threads)
+                              nthreads=self.threads,
+                              window=c["window"] if c.get("window") is not None else -1,
+                              sinks=sk_logits.double().numpy() if sk_logits is not None else None)
         return time.perf_counter() - t0, _row_flops(c, rows), len(rows)
 
     def rows_for(self, seconds):
@@ -253,6 +258,10 @@ def run_gpu(args):
     q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     mean = torch.empty((c["b"], c["hk"], c["dqk"]), dtype=torch.float32, device=dev)
     k_s = torch.empty_like(k) if c["kmean"] else None
+    windowed = c.get("window") is not None or bool(c.get("sinks"))
+    sk_h = workloads.sinks(c)
+    sinks_d = sk_h.to(dev) if sk_h is not None else None
+    window = c["window"] if c.get("window") is not None else -1
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 4 if c["kmean"] else 1
@@ -267,6 +276,9 @@ def run_gpu(args):
         if varlen:
             b2.attn_fwd_varlen(q, kk, v, cu_q, cu_k, c["sq"], causal=c["causal"],
                                scale=c["scale"], out=o, lse=lse)
+        elif windowed:
+            b2.attn_fwd_window_sink(q, kk, v, causal=c["causal"], window_left=window,
+                                    sinks=sinks_d, scale=c["scale"], out=o, lse=lse)
         else:
             b2.attn_fwd(q, kk, v, causal=c["causal"], scale=c["scale"], out=o, lse=lse)
         ev_a1.record(stream)
@@ -338,6 +350,7 @@ def run_gpu(args):
 
         if varlen:
             cqp, ckp = cuq_h.pin_memory(), cuk_h.pin_memory()
+        skp = sk_h.pin_memory() if sk_h is not None else None
 
         def e2e_step():
             qd = qp.to(dev, non_blocking=True)
@@ -349,6 +362,11 @@ def run_gpu(args):
                 od, ld = b2.attn_fwd_varlen(qd, kd, vd, cqp.to(dev, non_blocking=True),
                                             ckp.to(dev, non_blocking=True), c["sq"],
                                             causal=c["causal"], scale=c["scale"])
+            elif windowed:
+                od, ld = b2.attn_fwd_window_sink(
+                    qd, kd, vd, causal=c["causal"], window_left=window,
+                    sinks=skp.to(dev, non_blocking=True) if skp is not None else None,
+                    scale=c["scale"])
             else:
                 od, ld = b2.attn_fwd(qd, kd, vd, causal=c["causal"], scale=c["scale"])
             op.copy_(od, non_blocking=True)
@@ -365,6 +383,8 @@ def run_gpu(args):
         h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
         if varlen:
             h2d += (cuq_h.numel() + cuk_h.numel()) * 4
+        if sk_h is not None:
+            h2d += sk_h.numel() * 4
         d2h = o.numel() * 2 + lse.numel() * 4
         e2e = {"value": world * fl / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -401,7 +421,10 @@ def run_gpu(args):
                         "parallelism": f"replicas x{world} (independent batches, no "
                                        f"collective)"},
                        **({"packed_sequence_lengths": workloads.varlen_lengths(c)}
-                          if varlen else {})),
+                          if varlen else {}),
+                       **({"window_left": window, "sinks": bool(c.get("sinks")),
+                           "flops": "2*b*hq*(dqk+dv)*allowed (query, key) pairs"}
+                          if windowed else {})),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": f"attn_fwd_kernel d{c['dqk']}x{c['dv']}",

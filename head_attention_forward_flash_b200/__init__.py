@@ -25,7 +25,7 @@ STATUS = {
     6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
     11: "ERR_SCRATCH",
 }
-EXPORTS = ("attn_fwd", "attn_fwd_varlen", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
            "attn_status_string", "attn_debug_status")
 
 
@@ -48,6 +48,9 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
                                     i64, ctypes.c_int, ctypes.c_float, vp]
     lib.attn_fwd_varlen.restype = ctypes.c_int
+    lib.attn_fwd_window_sink.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
+                                         ctypes.c_int, i64, ctypes.c_float, vp]
+    lib.attn_fwd_window_sink.restype = ctypes.c_int
     lib.k_smooth_mean.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean.restype = ctypes.c_int
     lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
@@ -114,6 +117,40 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
                       lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
                       1 if causal else 0, float(scale), _stream_ptr(q))
     _check("attn_fwd", st)
+    return out, lse
+
+
+def attn_fwd_window_sink(q, k, v, causal: bool = False, window_left: int = -1, sinks=None,
+                         scale: float | None = None, out=None, lse=None, return_lse: bool = True):
+    """attn_fwd with a sliding window (row i keeps keys j >= i + sk - sq - window_left;
+    window_left < 0: none) and optional per-head sink logits (fp32 CUDA tensor [hq]) that join
+    every row's softmax denominator. Returns ``(out, lse)`` as attn_fwd."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _want(t, name, 4)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    b, sq, hq, dqk = q.shape
+    bk, sk, hk, dqk2 = k.shape
+    bv, skv, hkv, dv = v.shape
+    if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
+        raise ValueError("inconsistent q/k/v shapes")
+    if sinks is not None:
+        _want(sinks, "sinks", 1)
+        if sinks.dtype != torch.float32 or sinks.shape[0] != hq:
+            raise ValueError("sinks must be float32 with one logit per query head")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    if out is None:
+        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q.device)
+    st = lib.attn_fwd_window_sink(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  lse.data_ptr() if lse is not None else None,
+                                  sinks.data_ptr() if sinks is not None else None, b, hq, hk, sq,
+                                  sk, dqk, dv, 1 if causal else 0, int(window_left), float(scale),
+                                  _stream_ptr(q))
+    _check("attn_fwd_window_sink", st)
     return out, lse
 
 

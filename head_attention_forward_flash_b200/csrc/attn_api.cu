@@ -103,9 +103,11 @@ struct Shape {
     const int* cu_q = nullptr;
     const int* cu_k = nullptr;
     int64_t total_q = 0, total_k = 0;
+    int64_t window = -1;          // left window, < 0: none
+    const float* sinks = nullptr;  // per query head sink logits, or null
 };
 
-template <class T, bool CAUSAL, bool VARLEN>
+template <class T, bool CAUSAL, bool VARLEN, bool EXT>
 int launch_attn(const void* q, const void* k, const void* v, void* out, float* lse,
                 const Shape& sh, float scale, cudaStream_t stream)
 {
@@ -116,7 +118,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
-    auto kern = attn_fwd_kernel<T, CAUSAL, VARLEN>;
+    auto kern = attn_fwd_kernel<T, CAUSAL, VARLEN, EXT>;
     if (!attr_done[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)T::SMEM_BYTES) != cudaSuccess) {
@@ -165,6 +167,8 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.cu_k = sh.cu_k;
     p.total_q = sh.total_q;
     p.total_k = sh.total_k;
+    p.window = sh.window;
+    p.sinks = sh.sinks;
     p.group = hq / hk;
     p.n_qu = (sq + T::NT * T::BM - 1) / (T::NT * T::BM);
     p.n_units = b * hq * p.n_qu;  // below 2^31 (checked by attn_fwd)
@@ -200,15 +204,20 @@ using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 +
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
+// Kernel variants: dense, packed sequences, and dense with window / sinks (compiled apart so
+// that the plain paths carry none of the extra bound logic).
 template <class T>
 int dispatch(int causal, bool varlen, const void* q, const void* k, const void* v, void* out,
              float* lse, const Shape& sh, float scale, cudaStream_t st)
 {
     if (varlen)
-        return causal ? launch_attn<T, true, true>(q, k, v, out, lse, sh, scale, st)
-                      : launch_attn<T, false, true>(q, k, v, out, lse, sh, scale, st);
-    return causal ? launch_attn<T, true, false>(q, k, v, out, lse, sh, scale, st)
-                  : launch_attn<T, false, false>(q, k, v, out, lse, sh, scale, st);
+        return causal ? launch_attn<T, true, true, false>(q, k, v, out, lse, sh, scale, st)
+                      : launch_attn<T, false, true, false>(q, k, v, out, lse, sh, scale, st);
+    if (sh.window >= 0 || sh.sinks)
+        return causal ? launch_attn<T, true, false, true>(q, k, v, out, lse, sh, scale, st)
+                      : launch_attn<T, false, false, true>(q, k, v, out, lse, sh, scale, st);
+    return causal ? launch_attn<T, true, false, false>(q, k, v, out, lse, sh, scale, st)
+                  : launch_attn<T, false, false, false>(q, k, v, out, lse, sh, scale, st);
 }
 
 int dispatch_dims(int64_t dqk, int causal, bool varlen, const void* q, const void* k,
@@ -223,15 +232,17 @@ int dispatch_dims(int64_t dqk, int causal, bool varlen, const void* q, const voi
     }
 }
 
-// Rows with no key at all (sk == 0): O = 0, LSE = -inf.
-__global__ void fill_empty_rows(__nv_bfloat16* out, int64_t n_out, float* lse, int64_t n_lse)
+// Rows with no key at all (sk == 0): O = 0, LSE = -inf, or the head's sink logit when sinks
+// are given (LSE [b, hq, sq]: entry t belongs to head (t / sq) % hq).
+__global__ void fill_empty_rows(__nv_bfloat16* out, int64_t n_out, float* lse, int64_t n_lse,
+                                const float* sinks = nullptr, int64_t hq = 1, int64_t sq = 1)
 {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_out; t += stride)
         out[t] = __float2bfloat16_rn(0.f);
     if (lse)
         for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_lse; t += stride)
-            lse[t] = -INFINITY;
+            lse[t] = sinks ? sinks[(t / sq) % hq] : -INFINITY;
 }
 
 }  // namespace
@@ -282,6 +293,52 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* out, 
     sh.hk = hk;
     sh.sq = sq;
     sh.sk = sk;
+    return dispatch_dims(dqk, causal, false, q, k, v, out, lse, sh, scale, st);
+}
+
+extern "C" int attn_fwd_window_sink(const void* q, const void* k, const void* v, void* out,
+                                    float* lse, const float* sinks, int64_t b, int64_t hq,
+                                    int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                                    int causal, int64_t window_left, float scale, void* stream)
+{
+    if (b < 0 || hq < 0 || sq < 0 || sk < 0 || hk <= 0) return B200ATTN_ERR_SHAPE;
+    if (hq % hk != 0) return B200ATTN_ERR_GQA;
+    const bool hd_ok = (dqk == 64 && dv == 64) || (dqk == 128 && dv == 128) ||
+                       (dqk == 192 && dv == 128) || (dqk == 256 && dv == 256);
+    if (!hd_ok) return B200ATTN_ERR_HEADDIM;
+    if (!std::isfinite(scale)) return B200ATTN_ERR_SCALE;
+    int64_t n_q, n_k, n_v, n_o, n_l, n_units;
+    if (!numel({b, sq, hq, dqk}, &n_q) || !numel({b, sk, hk, dqk}, &n_k) ||
+        !numel({b, sk, hk, dv}, &n_v) || !numel({b, sq, hq, dv}, &n_o) ||
+        !numel({b, hq, sq}, &n_l) || !numel({n_q, 2}, &n_q) || !numel({n_k, 2}, &n_k) ||
+        !numel({n_v, 2}, &n_v) || !numel({n_o, 2}, &n_o) || !numel({n_l, 4}, &n_l) ||
+        !numel({b, hq, (sq + 127) / 128}, &n_units) || n_units >= ((int64_t)1 << 31))
+        return B200ATTN_ERR_RANGE;
+    if (n_o == 0) return B200ATTN_OK;  // b, hq or sq is zero: nothing to compute
+    if (!q || !out || (sk > 0 && (!k || !v))) return B200ATTN_ERR_NULL;
+    if (!aligned(q, 16) || !aligned(out, 16) || (k && !aligned(k, 16)) ||
+        (v && !aligned(v, 16)) || (lse && !aligned(lse, 4)) || (sinks && !aligned(sinks, 4)))
+        return B200ATTN_ERR_ALIGN;
+    if (!tma_extent_ok(b, sq, hq, dqk) ||
+        (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv))))
+        return B200ATTN_ERR_RANGE;
+    int rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (sk == 0) {
+        fill_empty_rows<<<296, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), n_o / 2, lse,
+                                             n_l / 4, sinks, hq, sq);
+        return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+    }
+    Shape sh;
+    sh.b = b;
+    sh.hq = hq;
+    sh.hk = hk;
+    sh.sq = sq;
+    sh.sk = sk;
+    sh.window = window_left < 0 ? -1 : window_left;
+    sh.sinks = sinks;
     return dispatch_dims(dqk, causal, false, q, k, v, out, lse, sh, scale, st);
 }
 

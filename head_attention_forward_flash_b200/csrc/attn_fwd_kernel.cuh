@@ -64,6 +64,10 @@ struct AttnParams {
     const int* cu_q;
     const int* cu_k;
     int64_t total_q, total_k;
+    // Sliding window: row i keeps only keys j >= i + sk - sq - window (window < 0: no window).
+    // Sinks: one logit per query head that joins every row's softmax denominator (or null).
+    int64_t window;
+    const float* sinks;
     int64_t group;    // hq / hk
     int64_t n_qu;     // query units per (batch, head): ceil(sq / (NT * 128))
     int64_t n_units;  // b * hq * n_qu (below 2^31)
@@ -163,11 +167,13 @@ struct UnitInfo {
     int64_t obase;       // O row of its query 0: O[(obase + i) * hq + h]
     int64_t lbase;       // LSE of its query i at lse[lbase + i]
     int bmap;            // the tensor maps' batch coordinate
-    int n_blocks;   // key blocks with at least one allowed key for some row of the unit
+    int j_begin;    // first key block with an allowed key for some row of the unit (window)
+    int n_blocks;   // key blocks j_begin .. n_blocks-1 are visited
+    int mask_lo;    // blocks < mask_lo need the window's lower per-key bound
     int mask_from;  // blocks >= mask_from need the per-key mask (causal diagonal, ragged tail)
 };
 
-template <int BN, int NT, bool CAUSAL, bool VARLEN>
+template <int BN, int NT, bool CAUSAL, bool VARLEN, bool EXT>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
 {
     UnitInfo t;
@@ -204,6 +210,8 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
         t.lbase = ((int64_t)bi * p.hq + h) * p.sq;
         t.bmap = (int)bi;
     }
+    t.j_begin = 0;
+    t.mask_lo = 0;
     if (t.q0 >= t.sq) {  // (packed sequences) no query row of this sequence here
         t.n_blocks = 0;
         t.mask_from = 0;
@@ -223,6 +231,15 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
     } else {
         t.n_blocks = (int)n_kv;
         t.mask_from = (int)(t.sk / BN);
+    }
+    if (EXT && p.window >= 0) {  // keys left of every row's window are never visited
+        const int64_t last_row = (t.q0 + NT * 128 - 1 < t.sq - 1) ? t.q0 + NT * 128 - 1 : t.sq - 1;
+        const int64_t lo_first = t.q0 + t.sk - t.sq - p.window;  // the unit's smallest bound
+        const int64_t lo_last = last_row + t.sk - t.sq - p.window;  // and its largest
+        int64_t jb = lo_first <= 0 ? 0 : lo_first / BN;
+        jb = jb < t.n_blocks ? jb : t.n_blocks;
+        t.j_begin = (int)jb;
+        t.mask_lo = (int)(lo_last <= 0 ? 0 : (lo_last + BN - 1) / BN);
     }
     return t;
 }
@@ -265,7 +282,8 @@ __device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, 
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <class T, bool CAUSAL, bool VARLEN>
+// EXT: the sliding window and the sinks of AttnParams are honoured (compiled out otherwise).
+template <class T, bool CAUSAL, bool VARLEN, bool EXT>
 __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
@@ -356,7 +374,10 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     // First unit of this CTA's list (from u) with at least one key block, or -1.
     auto busy_from = [&](int64_t u) -> int64_t {
         for (; u < p.n_units; u += ustep)
-            if (unit_info<BN, NT, CAUSAL, VARLEN>(p, u).n_blocks > 0) return u;
+            {
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
+                if (t.n_blocks > t.j_begin) return u;
+            }
         return -1;
     };
 
@@ -372,7 +393,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int q_cnt = 0;       // Q units issued
             bool ok = true;
             auto load_q = [&](int64_t u) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 if (!mbar_wait(bar_q_empty, (uint32_t)(q_cnt & 1) ^ 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
@@ -419,12 +440,12 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int64_t u = busy_from(u0);
             if (u >= 0) load_q(u);
             while (u >= 0 && ok) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 const int64_t un = busy_from(u + ustep);
-                for (int j = 0; j < t.n_blocks && ok; ++j) {
+                for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
                     for (int tt = 0; tt < NT && ok; ++tt) {
                         if (tt == 0) load_k(t, j);  // the Q K^T step of item (j, tt)
-                        if (ok && T::Q_TMEM && j == 0 && tt == 0 && un >= 0)
+                        if (ok && T::Q_TMEM && j == t.j_begin && tt == 0 && un >= 0)
                             load_q(un);  // the staging buffer was emptied into TMEM
                         if (ok && pend && pend_tt == 0) load_v(pend_t, pend_j);  // P V step
                         pend = true;
@@ -464,8 +485,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             uint32_t kaddr = 0, vaddr = 0;
             int kslot = 0, vslot = 0;
             // Q K^T of item gi = (block j, tile tt) of the current unit.
-            auto qk = [&](int j, int tt, bool last_item) {
-                if (T::Q_TMEM && j == 0) {  // this tile's Q of the new unit must be in TMEM
+            // (first: the unit's first visited key block)
+            auto qk = [&](bool first, int tt, bool last_item) {
+                if (T::Q_TMEM && first) {  // this tile's Q of the new unit must be in TMEM
                     if (!mbar_wait(bar_q_tmem(tt), (uint32_t)(units & 1), wc, kErrTimeout)) {
                         ok = false;
                         return;
@@ -491,12 +513,12 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
             };
             // P V of item g = (block j, tile tt) of busy unit number uidx.
-            auto pv = [&](int64_t g, int j, int tt, bool last_block, int uidx) {
+            auto pv = [&](int64_t g, bool first, int tt, bool last_block, int uidx) {
                 if (!mbar_wait(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
                 }
-                if (j == 0 && uidx > 0 &&
+                if (first && uidx > 0 &&
                     !mbar_wait(bar_o_free(tt), (uint32_t)(uidx - 1) & 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
@@ -513,7 +535,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     vaddr = v_slots + vslot * T::V_TILE_BYTES;
                 }
                 issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)(g & 1) * BN, vaddr,
-                                 j > 0);
+                                 !first);
                 if (NT == 1) tc_commit(bar_pv_done);
                 if (tt == NT - 1) tc_commit(bar_vempty(vslot));
                 if (last_block) tc_commit(bar_o_full(tt));
@@ -521,11 +543,12 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             // The P V of each item is issued after the next item's Q K^T (also across units), so
             // the tensor core computes the next S while the softmax works on this one.
             bool pend = false, pend_last = false;
-            int pend_j = 0, pend_tt = 0, pend_u = 0;
+            bool pend_first = false;
+            int pend_tt = 0, pend_u = 0;
             int64_t pend_g = 0;
             for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
-                if (t.n_blocks == 0) continue;
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
+                if (t.n_blocks <= t.j_begin) continue;
                 if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
                     if (!mbar_wait(bar_q_full, (uint32_t)(units & 1), wc, kErrTimeout)) {
                         ok = false;
@@ -533,15 +556,15 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     }
                     tc_fence_after_sync();
                 }
-                for (int j = 0; j < t.n_blocks && ok; ++j) {
+                for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
                     for (int tt = 0; tt < NT && ok; ++tt) {
                         const bool last_item = (j == t.n_blocks - 1) && (tt == NT - 1);
-                        qk(j, tt, last_item);
+                        qk(j == t.j_begin, tt, last_item);
                         if (!ok) break;
-                        if (pend) pv(pend_g, pend_j, pend_tt, pend_last, pend_u);
+                        if (pend) pv(pend_g, pend_first, pend_tt, pend_last, pend_u);
                         pend = true;
                         pend_g = gi;
-                        pend_j = j;
+                        pend_first = (j == t.j_begin);
                         pend_tt = tt;
                         pend_last = (j == t.n_blocks - 1);
                         pend_u = units;
@@ -550,7 +573,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 ++units;
             }
-            if (ok && pend) pv(pend_g, pend_j, pend_tt, pend_last, pend_u);
+            if (ok && pend) pv(pend_g, pend_first, pend_tt, pend_last, pend_u);
             tc_commit(bar_mma_done);  // drain every MMA this thread issued before teardown
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
@@ -689,8 +712,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         if (T::Q_TMEM && busy_from(u0) >= 0)
             for (int k = 0; k < NTW && ok; ++k) ok = copy_q(0, tile_of(k));
         for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
-            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN>(p, u);
-            if (t.n_blocks == 0) {  // no key for any row of this unit: O = 0, LSE = -inf
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
+            if (t.n_blocks <= t.j_begin) {  // no key for any row of this unit: O = 0, LSE = -inf
+                // (or the head's sink logit)
 #pragma unroll
                 for (int k = 0; k < NTW; ++k) {
                     const int64_t i = t.q0 + tile_of(k) * 128 + row;
@@ -699,25 +723,34 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                             p.o + ((t.obase + i) * p.hq + t.h) * T::DV);
 #pragma unroll 1
                         for (int c = 0; c < T::DV / 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
-                        if (p.lse) p.lse[t.lbase + i] = -INFINITY;
+                        if (p.lse)
+                            p.lse[t.lbase + i] =
+                                (EXT && p.sinks) ? __ldg(p.sinks + t.h) : -INFINITY;
                     }
                 }
                 continue;
             }
             const int64_t un = busy_from(u + ustep);
             int64_t lim[NTW];  // last allowed key of this thread's row in each tile
+            int64_t lol[NTW];  // first allowed key (the window's lower bound), may be negative
             float m_ref[NTW];  // exponent reference (log2 units); moves lazily
             float l[NTW];      // sum of exp2(x - m_ref) over the keys seen so far
+            // A sink logit starts every row with that logit as reference and exp2(0) = 1 in
+            // the sum: it then joins the denominator exactly, through every lazy rescale.
+            const bool has_sink = EXT && p.sinks != nullptr;
+            const float sink_l2 =
+                has_sink ? __ldg(p.sinks + t.h) * 1.4426950408889634f : -INFINITY;
 #pragma unroll
             for (int k = 0; k < NTW; ++k) {
                 const int64_t i = t.q0 + tile_of(k) * 128 + row;
                 const int64_t lim_row = CAUSAL ? i + t.sk - t.sq : t.sk - 1;
                 lim[k] = lim_row < t.sk - 1 ? lim_row : t.sk - 1;
-                m_ref[k] = -INFINITY;
-                l[k] = 0.f;
+                lol[k] = (EXT && p.window >= 0) ? i + t.sk - t.sq - p.window : (int64_t)-1 << 40;
+                m_ref[k] = sink_l2;
+                l[k] = has_sink ? 1.f : 0.f;
             }
 
-            for (int j = 0; j < t.n_blocks && ok; ++j, ++jg) {
+            for (int j = t.j_begin; j < t.n_blocks && ok; ++j, ++jg) {
 #pragma unroll
                 for (int k = 0; k < NTW; ++k) {
                     const int tt = tile_of(k);
@@ -740,32 +773,45 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                     tmem_wait_ld();
 
-                    // Keys j*BN + c with c <= rel are allowed (rel < 0: none, >= BN - 1: all).
-                    // Per 32-key chunk the warp takes one of three uniform paths: every row of
-                    // the warp allows the whole chunk (nothing to do), none allows any of it
-                    // (skipped below: no max, P = 0 without exp2), or the chunk holds some row's
-                    // limit: then the disallowed scores become -inf, so the max ignores them and
-                    // their p = exp2(-inf) is exactly 0 (the scale factor is never 0: the launch
-                    // clamps it to at least 2^-100).
-                    int rel_hi = BN;  // the warp's largest rel: chunks starting above it are skipped
-                    if (j >= t.mask_from) {
+                    // Keys j*BN + c with lor <= c <= rel are allowed. Per 32-key chunk the warp
+                    // takes one of three uniform paths: every row of the warp allows the whole
+                    // chunk (nothing to do), none allows any of it (skipped below: no max, P = 0
+                    // without exp2), or the chunk holds some row's bound: then the disallowed
+                    // scores become -inf, so the max ignores them and their p = exp2(-inf) is
+                    // exactly 0 (the scale factor is never 0: the launch clamps it to at least
+                    // 2^-100).
+                    uint32_t skip = 0;  // bit ch: no row of this warp allows a key of chunk ch
+                    if ((EXT && j < t.mask_lo) || j >= t.mask_from) {
                         int64_t rel64 = lim[k] - (int64_t)j * BN;
                         rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
+                        int lor = 0;  // no lower bound without a window
+                        if (EXT) {
+                            int64_t lor64 = lol[k] - (int64_t)j * BN;
+                            lor = (int)(lor64 < 0 ? 0 : (lor64 > BN ? BN : lor64));
+                        }
                         const int rel = (int)rel64;
                         const int rel_lo = __reduce_min_sync(FULL, rel);
-                        rel_hi = __reduce_max_sync(FULL, rel);
+                        const int rel_hi = __reduce_max_sync(FULL, rel);
+                        const int lor_lo = EXT ? __reduce_min_sync(FULL, lor) : 0;
+                        const int lor_hi = EXT ? __reduce_max_sync(FULL, lor) : 0;
 #pragma unroll
                         for (int ch = 0; ch < BN / 32; ++ch) {
-                            if (ch * 32 + 31 <= rel_lo || ch * 32 > rel_hi) continue;
+                            if (ch * 32 > rel_hi || ch * 32 + 31 < lor_lo) {
+                                skip |= 1u << ch;
+                                continue;
+                            }
+                            if (ch * 32 + 31 <= rel_lo && ch * 32 >= lor_hi) continue;
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                sr[ch * 32 + e] = ch * 32 + e <= rel ? sr[ch * 32 + e] : 0xff800000u;
+                            for (int e = 0; e < 32; ++e) {
+                                const int c = ch * 32 + e;
+                                sr[c] = (c <= rel && c >= lor) ? sr[c] : 0xff800000u;
+                            }
                         }
                     }
                     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                     for (int ch = 0; ch < BN / 32; ++ch) {
-                        if (ch * 32 > rel_hi) continue;
+                        if ((skip >> ch) & 1u) continue;
 #pragma unroll
                         for (int c = 0; c < 16; ++c)
                             mx[c & 3] = fmax3(mx[c & 3], __uint_as_float(sr[ch * 32 + 2 * c]),
@@ -783,7 +829,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         m_ref[k] = m_new;
                         l[k] *= alpha;
                     }
-                    if (j > 0 && __any_sync(FULL, need)) {
+                    if (j > t.j_begin && __any_sync(FULL, need)) {
                         // O holds blocks < j of this tile: scale it in place once its last P V
                         // is complete. With two tiles that P V is item g-2, issued before this
                         // item's Q K^T, so it is complete now that S has landed. With one tile it
@@ -811,7 +857,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll
                     for (int ch = 0; ch < BN / 32; ++ch) {
                         uint32_t pk[16];
-                        if (ch * 32 > rel_hi) {  // no row of this warp allows any key here
+                        if ((skip >> ch) & 1u) {  // no row of this warp allows any key here
 #pragma unroll
                             for (int c = 0; c < 16; ++c) pk[c] = 0u;
                         } else {
@@ -839,7 +885,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     tmem_wait_st();
                     tc_fence_before_sync();
                     mbar_arrive(bar_p_full(sb));
-                    if (j == 0 && pend) {
+                    if (j == t.j_begin && pend) {
                         // Tile tt of the previous unit, now that its successor's first P is out.
                         ok = epilogue(pend_t, tt, pend_m[k], pend_l[k], pend_idx);
                         if (k == NTW - 1) pend = false;

@@ -83,6 +83,28 @@ B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out
              int causal, float scale, void* stream);
 
 /*
+ * attn_fwd_window_sink -- attn_fwd with a sliding window and per-head attention sinks.
+ *
+ * As attn_fwd, with two changes to each row's softmax (the "GPT-OSS sink+sliding-window" shapes
+ * named in "Tune MHA config & small-head pipeline pathology", Source of shapes; the pages define
+ * neither, and this is the usual reading):
+ *     window   J additionally keeps only keys j >= i + sk - sq - window_left (the row's
+ *              diagonal key and the window_left keys before it); window_left < 0: no window.
+ *     sinks    fp32 [hq] logits (in the units of scale * <q, k>), or NULL. sigma_h joins the
+ *              denominator without a value:  m = max(max_J s_j, sigma_h),
+ *              O = sum_J exp(s_j - m) V_j / (exp(sigma_h - m) + sum_J exp(s_j - m)),
+ *              LSE = log(exp(sigma_h) + sum_J exp(s_j)); an empty J gives O = 0, LSE = sigma_h.
+ * Key blocks left of every row's window are never loaded or multiplied.
+ *
+ *   sinks    device fp32, 4-byte aligned, or NULL. Read only.
+ *   other arguments, layouts, errors, allocation and concurrency as in attn_fwd.
+ */
+B200ATTN_API int attn_fwd_window_sink(const void* q, const void* k, const void* v, void* out,
+                                      float* lse, const float* sinks, int64_t b, int64_t hq,
+                                      int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                                      int causal, int64_t window_left, float scale, void* stream);
+
+/*
  * attn_fwd_varlen -- attn_fwd over b packed sequences of different lengths.
  *
  * Sequence i (i < b) owns query rows cu_seqlens_q[i] .. cu_seqlens_q[i+1]-1 of q / out and key

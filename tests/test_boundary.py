@@ -104,3 +104,25 @@ def test_varlen_empty_problem_is_a_no_op():
     assert call_varlen(b=0, q=None, k=None, v=None, o=None, lse=None, cq=None, ck=None) == 0
     assert call_varlen(tq=0, q=None, o=None, lse=None, cq=None, ck=None) == 0
     assert call_varlen(max_sq=0, q=None, o=None, lse=None, cq=None, ck=None) == 0
+
+
+def call_ws(q=A, k=A, v=A, o=A, lse=A, sinks=A, b=1, hq=2, hk=1, sq=16, sk=16, dqk=64, dv=64,
+            causal=1, window=8, scale=0.125):
+    return b2.lib.attn_fwd_window_sink(q, k, v, o, lse, sinks, b, hq, hk, sq, sk, dqk, dv, causal,
+                                       window, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b=-1), 2), (dict(sk=-1), 2), (dict(hk=0), 2), (dict(hq=3, hk=2), 3),
+    (dict(dqk=96, dv=96), 4), (dict(scale=float("inf")), 7),
+    (dict(q=None), 1), (dict(k=None), 1), (dict(o=None), 1),
+    (dict(q=A + 8), 5), (dict(sinks=A + 2), 5), (dict(lse=A + 1), 5),
+    (dict(sq=1 << 31), 6),
+])
+def test_attn_fwd_window_sink_rejects(kw, code):
+    assert call_ws(**kw) == code
+
+
+def test_window_sink_empty_problem_is_a_no_op():
+    assert call_ws(b=0, q=None, k=None, v=None, o=None, lse=None, sinks=None) == 0
+    assert call_ws(sq=0, q=None, o=None, lse=None) == 0

@@ -34,6 +34,11 @@ CONFIGS = {
     # each sequence's query and key lengths equal; sq / sk hold the longest possible length.
     6: dict(workload="varlen_b8_hq48_hk8_s1024to2048_d64_causal", b=8, hq=48, hk=8, sq=2048,
             sk=2048, min_s=1024, dqk=64, dv=64, causal=True, kmean=False, varlen=True),
+    # Sliding window + attention sinks (the "GPT-OSS sink+sliding-window" shapes of the pages'
+    # shape sources): 64:8 heads of d64, a 128-key window, one sink logit per head drawn
+    # 1.5 * N(0,1) with seed 4000 + id.
+    7: dict(workload="swa_sink_b1_hq64_hk8_s8192_d64_causal_w128", b=1, hq=64, hk=8, sq=8192,
+            sk=8192, dqk=64, dv=64, causal=True, kmean=False, window=128, sinks=True),
 }
 
 HEAD_DIMS = ((64, 64), (128, 128), (192, 128), (256, 256))
@@ -50,13 +55,36 @@ def config(n: int) -> dict:
 
 def flops(c: dict) -> float:
     """Algorithmic FLOPs of one forward pass: 2*b*hq*sq*sk*(dqk+dv), halved when causal (for
-    packed sequences, the sum of that over the sequences)."""
+    packed sequences, the sum of that over the sequences; with a sliding window, 2*b*hq*(dqk+dv)
+    times the exact number of allowed (query, key) pairs)."""
+    if c.get("window") is not None:
+        return 2.0 * c["b"] * c["hq"] * (c["dqk"] + c["dv"]) * allowed_pairs(c)
     if c.get("varlen"):
         lengths = varlen_lengths(c)
         f = sum(2.0 * c["hq"] * n * n * (c["dqk"] + c["dv"]) for n in lengths)
     else:
         f = 2.0 * c["b"] * c["hq"] * c["sq"] * c["sk"] * (c["dqk"] + c["dv"])
     return f / 2.0 if c["causal"] else f
+
+
+def allowed_pairs(c: dict) -> int:
+    """Allowed (query, key) pairs of one (batch, head): key j <= i + sk - sq when causal and
+    j >= i + sk - sq - window."""
+    total = 0
+    for i in range(c["sq"]):
+        d = i + c["sk"] - c["sq"]
+        hi = min(c["sk"] - 1, d) if c["causal"] else c["sk"] - 1
+        lo = max(0, d - c["window"]) if c.get("window") is not None else 0
+        total += max(0, hi - lo + 1)
+    return total
+
+
+def sinks(c: dict):
+    """The per-head sink logits of a workload with sinks (fp32 [hq]), else None."""
+    if not c.get("sinks"):
+        return None
+    g = torch.Generator(device="cpu").manual_seed(4000 + int(c.get("id", 0)))
+    return (1.5 * torch.randn(c["hq"], generator=g)).float()
 
 
 def varlen_lengths(c: dict) -> list:
