@@ -175,6 +175,24 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.div_nqu = make_fastdiv((uint32_t)p.n_qu);
     p.div_hq = make_fastdiv((uint32_t)hq);
     p.div_group = make_fastdiv((uint32_t)p.group);
+    p.div_bh = make_fastdiv((uint32_t)(b * hq > 0 ? b * hq : 1));
+    // Unit order (measured on B200 at 8x48:8 2048^2 d64, 128 heads 8192^2 d192/128 and 5 heads
+    // 65536^2 d128, all causal). Causal units differ in cost, so CTAs take them in snake order
+    // (odd rounds reversed), which evens out the per-CTA totals; where every head's K/V fits in
+    // L2 or the kv heads are few, in weight-major order (all heads' heaviest units first), which
+    // evens them out best; where many heads' K/V far exceed L2, head-major, so that the CTAs
+    // working at the same time share a few heads' K/V. Equal-cost units (no causal mask, or a
+    // window band) take plain round robin, and so do packed sequences, whose unit costs depend
+    // on lengths the host does not see (measured: weight-major order was slower there).
+    {
+        const double kv_bytes = (double)(b * sk) * (double)hk * (double)(T::DQK + T::DV) * 2.0;
+        if (!CAUSAL || VARLEN || (EXT && sh.window >= 0))
+            p.order = 0;
+        else if (b * hk <= 16 || kv_bytes <= 64.0e6)
+            p.order = 2;
+        else
+            p.order = 1;
+    }
     // The MMA applies the sign of the scale (negate-A bit of the instruction descriptor), so
     // the softmax only ever sees a non-negative factor. It is kept at 2^-100 or more, so that a
     // masked score of -inf always maps to exp2(-inf) = 0. For |scale| below that (scale 0

@@ -72,6 +72,12 @@ struct AttnParams {
     int64_t n_qu;     // query units per (batch, head): ceil(sq / (NT * 128))
     int64_t n_units;  // b * hq * n_qu (below 2^31)
     FastDiv div_nqu, div_hq, div_group;  // by n_qu, hq and group
+    // Order in which CTAs take units. Round r gives CTA c the position
+    // r * grid + (r odd and order != 0 ? grid - 1 - c : c); position -> unit is the identity
+    // (head-major, heaviest unit of a head first) for order 0 / 1, and for order 2 the
+    // weight-major order (the k-th heaviest unit of every head, then the (k+1)-th ...).
+    int order;
+    FastDiv div_bh;  // by b * hq
     float scale_log2; // |scale| * log2(e); the sign of scale is applied by the MMA (negate A)
     uint32_t idesc_qk;
     int* status;      // device error word
@@ -368,17 +374,28 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_holder;
     const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
-    const int64_t u0 = blockIdx.x;
-    const int64_t ustep = gridDim.x;
-
-    // First unit of this CTA's list (from u) with at least one key block, or -1.
-    auto busy_from = [&](int64_t u) -> int64_t {
-        for (; u < p.n_units; u += ustep)
-            {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
-                if (t.n_blocks > t.j_begin) return u;
-            }
-        return -1;
+    // The unit this CTA takes in round r, or -1 when round r is past the last unit (and so is
+    // every later round). Every unit is taken by exactly one (CTA, round).
+    auto unit_of = [&](int64_t r) -> int64_t {
+        const int64_t g = gridDim.x;
+        const int64_t c = blockIdx.x;
+        const int64_t pos = r * g + ((p.order != 0 && (r & 1)) ? g - 1 - c : c);
+        if (pos >= p.n_units) return -1;
+        if (p.order == 2) {
+            const uint32_t k = fast_div((uint32_t)pos, p.div_bh);  // rank within its head
+            const uint32_t bh = (uint32_t)pos - k * p.div_bh.d;
+            return (int64_t)bh * p.div_nqu.d + k;
+        }
+        return pos;
+    };
+    // First round from r whose unit has at least one key block, or -1.
+    auto busy_from = [&](int64_t r) -> int64_t {
+        for (;; ++r) {
+            const int64_t u = unit_of(r);
+            if (u < 0) return -1;
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
+            if (t.n_blocks > t.j_begin) return r;
+        }
     };
 
     if constexpr (T::NSM == 2) {
@@ -437,11 +454,12 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             bool pend = false;  // the P V step still owed for the previous item
             UnitInfo pend_t{};
             int pend_j = 0, pend_tt = 0;
-            int64_t u = busy_from(u0);
-            if (u >= 0) load_q(u);
-            while (u >= 0 && ok) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
-                const int64_t un = busy_from(u + ustep);
+            int64_t r = busy_from(0);
+            if (r >= 0) load_q(unit_of(r));
+            while (r >= 0 && ok) {
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, unit_of(r));
+                const int64_t rn = busy_from(r + 1);
+                const int64_t un = rn >= 0 ? unit_of(rn) : -1;
                 for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
                     for (int tt = 0; tt < NT && ok; ++tt) {
                         if (tt == 0) load_k(t, j);  // the Q K^T step of item (j, tt)
@@ -457,7 +475,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 // With Q read from shared memory, the next unit's Q can only replace this one
                 // after the unit's last Q K^T (the MMA warp commits bar_q_empty then).
                 if (ok && !T::Q_TMEM && un >= 0) load_q(un);
-                u = un;
+                r = rn;
             }
             if (ok && pend && pend_tt == 0) load_v(pend_t, pend_j);
             // Nothing may be in flight when the CTA exits: wait for the last load of each slot
@@ -546,7 +564,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             bool pend_first = false;
             int pend_tt = 0, pend_u = 0;
             int64_t pend_g = 0;
-            for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
+            for (int64_t r = 0; ok; ++r) {
+                const int64_t u = unit_of(r);
+                if (u < 0) break;
                 const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 if (t.n_blocks <= t.j_begin) continue;
                 if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
@@ -709,9 +729,11 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll
         for (int k = 0; k < NTW; ++k) pend_m[k] = pend_l[k] = 0.f;
         int pend_idx = 0;
-        if (T::Q_TMEM && busy_from(u0) >= 0)
+        if (T::Q_TMEM && busy_from(0) >= 0)
             for (int k = 0; k < NTW && ok; ++k) ok = copy_q(0, tile_of(k));
-        for (int64_t u = u0; u < p.n_units && ok; u += ustep) {
+        for (int64_t r = 0; ok; ++r) {
+            const int64_t u = unit_of(r);
+            if (u < 0) break;
             const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
             if (t.n_blocks <= t.j_begin) {  // no key for any row of this unit: O = 0, LSE = -inf
                 // (or the head's sink logit)
@@ -730,7 +752,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 continue;
             }
-            const int64_t un = busy_from(u + ustep);
+            const int64_t rn = busy_from(r + 1);
+            const int64_t un = rn >= 0 ? unit_of(rn) : -1;
             int64_t lim[NTW];  // last allowed key of this thread's row in each tile
             int64_t lol[NTW];  // first allowed key (the window's lower bound), may be negative
             float m_ref[NTW];  // exponent reference (log2 units); moves lazily
