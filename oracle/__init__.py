@@ -59,6 +59,8 @@ def _bind(lib):
     lib.oracle_attn_full_ex.restype = ctypes.c_int
     lib.oracle_k_mean.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p]
     lib.oracle_k_mean.restype = ctypes.c_int
+    lib.oracle_k_gate.argtypes = [_p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _p, _p, _p]
+    lib.oracle_k_gate.restype = ctypes.c_int
     lib.oracle_k_sub.argtypes = [_p, _p, _p, _i64, _i64, _i64, _i64]
     lib.oracle_k_sub.restype = ctypes.c_int
     lib.oracle_bf16_rne.argtypes = [ctypes.c_double]
@@ -183,6 +185,23 @@ def k_mean(k, b, hk, sk, d, lib=None):
     if rc != 0:
         raise ValueError(f"oracle_k_mean failed with code {rc}")
     return m64, m32
+
+
+def k_gate(k, b, hk, sk, d, threshold, lib=None):
+    """K-smoothing gate over the strided key sample (see attn_oracle.c): returns (mean fp64
+    [b,hk,d], its fp32 rounding, ratio fp64 [b,hk], gate int32 [b,hk]); mean is the sampled
+    channel mean where the gate is on, else 0."""
+    lib = lib or load_library()
+    k = _u16(k)
+    m64 = np.zeros((b, hk, d), dtype=np.float64)
+    m32 = np.zeros((b, hk, d), dtype=np.float32)
+    r = np.zeros((b, hk), dtype=np.float64)
+    gate = np.zeros((b, hk), dtype=np.int32)
+    rc = lib.oracle_k_gate(_ptr(k), b, hk, sk, d, float(threshold), _ptr(m64), _ptr(m32), _ptr(r),
+                           _ptr(gate))
+    if rc != 0:
+        raise ValueError(f"oracle_k_gate failed with code {rc}")
+    return m64, m32, r, gate
 
 
 def k_sub(k, mean32, b, hk, sk, d, lib=None):

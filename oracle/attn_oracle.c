@@ -268,6 +268,54 @@ int oracle_k_mean(const uint16_t *k, int64_t b, int64_t hk, int64_t sk, int64_t 
 }
 
 /* K' = bf16_rne(K - mean), with the fp32 mean broadcast over the sequence axis. */
+/* K-smoothing gate. The pages run it as "per-(batch*head, chunk) moments over the same
+ * strided sample, then a per-head fold and gate" with a threshold and a stride they do not
+ * print ("[HIP] Mha v4: run the K-smoothing gate as one HIP call", commit message; "below 2048
+ * keys a full ... copy of K"). Reading:
+ *   sample   keys s = 0, stride, 2*stride, ... < sk with stride = ceil(sk / 2048) (every key
+ *            when sk <= 2048); n = the number of sampled keys
+ *   moments  mu_c = (1/n) sum_s K[bi,s,g,c],   e_c = (1/n) sum_s K[bi,s,g,c]^2
+ *   ratio    r = sum_c mu_c^2 / sum_c e_c        (the share of K's energy in its channel mean;
+ *            0 when K is all zero)
+ *   gate     r >= threshold
+ *   output   mean = gate ? mu (rounded to fp32) : 0, per (bi, g, c)
+ * Everything in double precision; mean32 is the fp32 rounding of the output mean. */
+int oracle_k_gate(const uint16_t *k, int64_t b, int64_t hk, int64_t sk, int64_t d,
+                  double threshold, double *mean64, float *mean32, double *ratio, int *gate)
+{
+    if (sk <= 0 || d <= 0) return 1;
+    const int64_t stride = (sk + 2047) / 2048;
+    const int64_t n = (sk + stride - 1) / stride;
+    double *mu = (double *)malloc(sizeof(double) * (size_t)d);
+    if (!mu) return 1;
+    for (int64_t bi = 0; bi < b; ++bi)
+        for (int64_t g = 0; g < hk; ++g) {
+            double num = 0.0, den = 0.0;
+            for (int64_t c = 0; c < d; ++c) {
+                double sum = 0.0, sq = 0.0;
+                for (int64_t t = 0; t < n; ++t) {
+                    const double x = bf16_value(k[((bi * sk + t * stride) * hk + g) * d + c]);
+                    sum += x;
+                    sq += x * x;
+                }
+                mu[c] = sum / (double)n;
+                num += mu[c] * mu[c];
+                den += sq / (double)n;
+            }
+            const double r = den > 0.0 ? num / den : 0.0;
+            const int on = r >= threshold;
+            if (ratio) ratio[bi * hk + g] = r;
+            if (gate) gate[bi * hk + g] = on;
+            for (int64_t c = 0; c < d; ++c) {
+                const int64_t idx = (bi * hk + g) * d + c;
+                if (mean64) mean64[idx] = on ? mu[c] : 0.0;
+                if (mean32) mean32[idx] = on ? (float)mu[c] : 0.0f;
+            }
+        }
+    free(mu);
+    return 0;
+}
+
 int oracle_k_sub(const uint16_t *k, const float *mean32, uint16_t *kout, int64_t b, int64_t hk,
                  int64_t sk, int64_t d)
 {

@@ -382,8 +382,51 @@ def pin_sink_closed_form(lib):
             assert np.array_equal(l1[:, :, :4], np.broadcast_to(sinks[None, :, None], (b, hq, 4)))
 
 
+def pin_k_gate(lib):
+    """K-smoothing gate: constant key rows put all of K's energy in the mean (ratio 1, gate on
+    at a threshold of exactly 1, output = that row); rows in +/- pairs have zero mean (ratio 0,
+    output 0); two alternating values a, b in one channel give the closed form
+    r = (a + b)^2 / (2 (a^2 + b^2)); at 4096 keys every 2nd key is sampled (changing an
+    unsampled key changes nothing, a sampled one changes the mean); with threshold 0 the output
+    is numpy's fp64 mean over all keys (sk <= 2048)."""
+    b, hk, d = 1, 2, 64
+    g = torch.Generator().manual_seed(51)
+    row = torch.randn(hk, d, generator=g).to(torch.bfloat16)
+    const = row.expand(b, 100, hk, d).contiguous()
+    m64, m32, r, gate = oracle.k_gate(bf16_bits(const), b, hk, 100, d, 1.0, lib=lib)
+    assert np.all(r == 1.0) and np.all(gate == 1)
+    assert np.array_equal(m32, row.float().numpy()[None])
+    _, _, _, gate = oracle.k_gate(bf16_bits(const), b, hk, 100, d, 1.0 + 1e-12, lib=lib)
+    assert np.all(gate == 0)
+    pm = torch.stack([row, -row], dim=0).repeat(50, 1, 1)[None].contiguous()  # [1,100,hk,d]
+    m64, m32, r, gate = oracle.k_gate(bf16_bits(pm), b, hk, 100, d, 1e-9, lib=lib)
+    assert np.all(r == 0.0) and np.all(gate == 0) and np.all(m64 == 0.0)
+    a_, b_ = 3.0, -0.5
+    two = torch.zeros(b, 64, hk, d)
+    two[:, 0::2, :, 0] = a_
+    two[:, 1::2, :, 0] = b_
+    _, _, r, _ = oracle.k_gate(bf16_bits(two.to(torch.bfloat16)), b, hk, 64, d, 0.5, lib=lib)
+    assert np.allclose(r, (a_ + b_) ** 2 / (2 * (a_ ** 2 + b_ ** 2)), rtol=0, atol=1e-15)
+    sk = 4096
+    big = torch.randn(b, sk, hk, d, generator=g).to(torch.bfloat16)
+    m_ref, _, r_ref, _ = oracle.k_gate(bf16_bits(big), b, hk, sk, d, 0.0, lib=lib)
+    unsampled = big.clone()
+    unsampled[:, 3] += 5.0
+    m_u, _, r_u, _ = oracle.k_gate(bf16_bits(unsampled), b, hk, sk, d, 0.0, lib=lib)
+    assert np.array_equal(m_u, m_ref) and np.array_equal(r_u, r_ref)
+    sampled = big.clone()
+    sampled[:, 2] += 5.0
+    m_s, _, _, _ = oracle.k_gate(bf16_bits(sampled), b, hk, sk, d, 0.0, lib=lib)
+    assert not np.array_equal(m_s, m_ref)
+    assert np.allclose(m_ref, big[:, 0::2].double().numpy().mean(axis=1), rtol=0, atol=1e-14)
+    small = big[:, :1500].contiguous()
+    m_a, _, _, gate = oracle.k_gate(bf16_bits(small), b, hk, 1500, d, 0.0, lib=lib)
+    assert np.all(gate == 1)
+    assert np.allclose(m_a, small.double().numpy().mean(axis=1), rtol=0, atol=1e-14)
+
+
 ALL_PINS = [pin_sdpa, pin_uniform_scores, pin_causal_row0_and_single_key, pin_two_keys, pin_large_scores,
             pin_gqa_replication, pin_permutation_and_independence, pin_convexity,
             pin_fully_masked_rows, pin_kmean_shift_identity, pin_k_mean, pin_bf16_rne,
             pin_rows_api, pin_window_brute_force, pin_window_zero_is_the_diagonal,
-            pin_sink_closed_form]
+            pin_sink_closed_form, pin_k_gate]

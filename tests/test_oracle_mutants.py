@@ -1,7 +1,8 @@
 """Mutation check of the oracle's pins: plausible mistakes planted in a copy of the oracle's
 C source (a dropped scale, a wrong GQA head map, a causal off-by-one, a transposed V stride, a
 missing normalisation, a wrong LSE, a wrong mean divisor, a wrong rounding mode, a window
-off-by-one or a dropped window, a sink left out of the denominator or of an empty row) must each be
+off-by-one or a dropped window, a sink left out of the denominator or of an empty row, a gate
+sample stride off by one, a strict gate threshold, an unsquared gate mean) must each be
 caught by at least one pin. The planted copies are built in a temporary directory on the CPU;
 the real oracle is untouched."""
 import os
@@ -22,6 +23,9 @@ MUTANTS = {
     "window_ignored": ("if (a->window >= 0 && diag", "if (0 && diag"),
     "sink_left_out_of_sum": ("if (has_sink) l += exp(sink - m);", "if (0) l += exp(sink - m);"),
     "empty_row_ignores_sink": ("*lse_out = has_sink ? sink : -INFINITY;", "*lse_out = -INFINITY;"),
+    "gate_stride_off_by_one": ("const int64_t stride = (sk + 2047) / 2048;", "const int64_t stride = sk / 2048 + 1;"),
+    "gate_strict_threshold": ("const int on = r >= threshold;", "const int on = r > threshold;"),
+    "gate_mean_not_squared": ("num += mu[c] * mu[c];", "num += fabs(mu[c]);"),
     "no_normalisation": ("o_row[c] /= l;", "o_row[c] /= 1.0;"),
     "lse_without_max": ("*lse_out = m + log(l);", "*lse_out = log(l);"),
     "mean_divisor": ("double mean = sum / (double)sk;", "double mean = sum / (double)(sk - 1);"),
