@@ -338,6 +338,27 @@ def run_gpu(args):
     srt = sorted(attn_ms)
     lo, hi = int(0.1 * len(srt)), max(int(0.9 * len(srt)), int(0.1 * len(srt)) + 1)
 
+    # the K-smoothing gate on the same K (K-mean workload): its own event-timed calls
+    kgate = None
+    if c["kmean"]:
+        ge0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        ge1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+        for _ in range(3):
+            b2.k_smooth_gate(k, 0.25)
+        for s_ in range(10):
+            flush.zero_()
+            ge0[s_].record(stream)
+            b2.k_smooth_gate(k, 0.25)
+            ge1[s_].record(stream)
+        torch.cuda.synchronize()
+        g_us = 1e3 * statistics.median(ge0[s_].elapsed_time(ge1[s_]) for s_ in range(10))
+        stride = (c["sk"] + 2047) // 2048
+        n_samp = (c["sk"] + stride - 1) // stride
+        g_bytes = c["b"] * n_samp * c["hk"] * c["dqk"] * 2
+        kgate = {"us_median": g_us, "sampled_bytes": g_bytes,
+                 "gbs": g_bytes / (g_us * 1e-6) / 1e9, "threshold": 0.25,
+                 "launches": 2, "note": "k_smooth_gate alone, L2 flushed before each call"}
+
     # end to end through the public API with host buffers (pinned), copies inside the timing
     e2e = None
     if not args.no_e2e:
@@ -437,6 +458,8 @@ def run_gpu(args):
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
+    if kgate is not None:
+        line["k_smooth_gate"] = kgate
     print(json.dumps(line), flush=True)
 
 

@@ -25,7 +25,7 @@ STATUS = {
     6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
     11: "ERR_SCRATCH",
 }
-EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
            "attn_status_string", "attn_debug_status")
 
 
@@ -55,6 +55,8 @@ def _load() -> ctypes.CDLL:
     lib.k_smooth_mean.restype = ctypes.c_int
     lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean_noalloc.restype = ctypes.c_int
+    lib.k_smooth_gate.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, vp]
+    lib.k_smooth_gate.restype = ctypes.c_int
     lib.k_smooth_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_sub.restype = ctypes.c_int
     lib.attn_status_string.argtypes = [ctypes.c_int]
@@ -222,6 +224,29 @@ def k_smooth_mean_noalloc(k, mean):
     _check("k_smooth_mean_noalloc", lib.k_smooth_mean_noalloc(k.data_ptr(), mean.data_ptr(), b, hk,
                                                               sk, d, _stream_ptr(k)))
     return mean
+
+
+def k_smooth_gate(k, threshold: float, mean=None, gate=None, ratio=None, return_ratio=True):
+    """The K-smoothing gate over a strided sample of keys. k [b, sk, hk, d] bf16.
+
+    Returns ``(mean [b, hk, d] fp32 -- the sampled channel mean where the gate is on, else 0 --,
+    gate [b, hk] int32, ratio [b, hk] fp32 or None)``; pass ``mean`` to k_smooth_sub."""
+    import torch
+    _want(k, "k", 4)
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
+    b, sk, hk, d = k.shape
+    if mean is None:
+        mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    if gate is None:
+        gate = torch.empty((b, hk), dtype=torch.int32, device=k.device)
+    if return_ratio and ratio is None:
+        ratio = torch.empty((b, hk), dtype=torch.float32, device=k.device)
+    st = lib.k_smooth_gate(k.data_ptr(), mean.data_ptr(), gate.data_ptr(),
+                           ratio.data_ptr() if ratio is not None else None, b, hk, sk, d,
+                           float(threshold), _stream_ptr(k))
+    _check("k_smooth_gate", st)
+    return mean, gate, ratio
 
 
 def k_smooth_sub(k, mean, out=None):

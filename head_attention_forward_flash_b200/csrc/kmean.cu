@@ -7,6 +7,7 @@
 // each channel in a fixed order, so the result is bit-identical from run to run (the two
 // deterministic kernels behind one host call of "[HIP] Mha v4: run the K-smoothing gate as one
 // HIP call", Summary and commit message).
+#include <cmath>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -86,6 +87,114 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
         for (int q = 0; q < kThreads / 32; ++q) t += red[q][lane];
         mean[bi * cols + col] = __fdiv_rn(t, sk_f);
+    }
+}
+
+// Gate moments over the sampled keys s = t * stride (t < n_samp):
+// partial[bi][chunk][0][col] = sum of K, partial[bi][chunk][1][col] = sum of K^2 over the chunk's
+// sampled rows (K^2 of a bf16 value is exact in fp32).
+__global__ void __launch_bounds__(kThreads)
+    k_gate_partial(const uint4* __restrict__ k, float* __restrict__ partial, int64_t sk,
+                   int64_t cols, int64_t stride, int64_t n_samp, int64_t per_chunk, int nchunks)
+{
+    const int64_t bi = blockIdx.z;
+    const int chunk = blockIdx.y;
+    const int64_t g8 = (int64_t)blockIdx.x * kThreads + threadIdx.x;  // 8-channel group
+    const int64_t c8 = cols / 8;
+    if (g8 >= c8) return;
+    const int64_t t0 = (int64_t)chunk * per_chunk;
+    int64_t t1 = t0 + per_chunk;
+    t1 = t1 < n_samp ? t1 : n_samp;
+    float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float sq[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4* src = k + (bi * sk) * c8 + g8;
+    const int64_t step = stride * c8;
+    auto add = [&](const uint4& x) {
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+            sum[2 * q] += lo;
+            sum[2 * q + 1] += hi;
+            sq[2 * q] = fmaf(lo, lo, sq[2 * q]);
+            sq[2 * q + 1] = fmaf(hi, hi, sq[2 * q + 1]);
+        }
+    };
+    int64_t t = t0;
+    for (; t + 4 <= t1; t += 4) {  // four independent 16-byte loads in flight, added in row order
+        const uint4 x0 = __ldg(src + (t + 0) * step);
+        const uint4 x1 = __ldg(src + (t + 1) * step);
+        const uint4 x2 = __ldg(src + (t + 2) * step);
+        const uint4 x3 = __ldg(src + (t + 3) * step);
+        add(x0);
+        add(x1);
+        add(x2);
+        add(x3);
+    }
+    for (; t < t1; ++t) add(__ldg(src + t * step));
+    float* dst = partial + ((bi * nchunks + chunk) * 2) * cols + g8 * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        dst[e] = sum[e];
+        dst[cols + e] = sq[e];
+    }
+}
+
+// Per (bi, g), 1024 threads: chunk group grp = threadIdx.x / d of channel c = threadIdx.x % d
+// sums the partials of chunks grp, grp + G, grp + 2G, ... (G = 1024 / d groups); the G group
+// sums are added in group order, giving mu_c and e_c (mean and mean square over the sample);
+// then sum mu_c^2 and sum e_c over the d channels by a fixed tree in shared memory; ratio =
+// first / second (0 for an all-zero K); gate = ratio >= threshold; mean = mu where the gate is
+// on, else 0. Every order is fixed, so the result does not depend on timing.
+constexpr int kFoldThreads = 1024;
+__global__ void __launch_bounds__(kFoldThreads)
+    k_gate_fold(const float* __restrict__ partial, float* __restrict__ mean,
+                int* __restrict__ gate, float* __restrict__ ratio, int64_t hk, int64_t d,
+                int nchunks, float n_f, float threshold)
+{
+    __shared__ float gs[kFoldThreads], gq[kFoldThreads];
+    __shared__ float num[256], den[256];
+    const int64_t bg = blockIdx.x;  // bi * hk + g
+    const int64_t bi = bg / hk, g = bg - bi * hk;
+    const int groups = kFoldThreads / (int)d;
+    const int c = threadIdx.x % (int)d;
+    const int grp = threadIdx.x / (int)d;
+    const int64_t cols = hk * d;
+    const int64_t col = g * d + c;
+    float gsum = 0.f, gsq = 0.f;
+    for (int ch = grp; ch < nchunks; ch += groups) {
+        const float* src = partial + ((bi * nchunks + ch) * 2) * cols;
+        gsum += src[col];
+        gsq += src[cols + col];
+    }
+    gs[threadIdx.x] = gsum;
+    gq[threadIdx.x] = gsq;
+    __syncthreads();
+    if (grp != 0) return;
+    float sum = 0.f, sq = 0.f;
+    for (int q = 0; q < groups; ++q) {
+        sum += gs[q * (int)d + c];
+        sq += gq[q * (int)d + c];
+    }
+    const float mu = __fdiv_rn(sum, n_f);
+    num[c] = mu * mu;
+    den[c] = __fdiv_rn(sq, n_f);
+    // only the d threads of group 0 remain: a barrier over exactly those warps (d is a multiple
+    // of 32), id 1
+    asm volatile("bar.sync 1, %0;" ::"r"((int)d) : "memory");
+    for (int w = (int)d / 2; w > 0; w >>= 1) {
+        if (c < w) {
+            num[c] += num[c + w];
+            den[c] += den[c + w];
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"((int)d) : "memory");
+    }
+    const float r = den[0] > 0.f ? __fdiv_rn(num[0], den[0]) : 0.f;
+    const bool on = r >= threshold;
+    mean[bg * d + c] = on ? mu : 0.f;
+    if (c == 0) {
+        gate[bg] = on ? 1 : 0;
+        if (ratio) ratio[bg] = r;
     }
 }
 
@@ -264,6 +373,53 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     k_mean_fold<<<dim3((unsigned)((cols + 31) / 32), (unsigned)b), kThreads, 0, st>>>(
         partial, mean, cols, (int)nchunks, (float)sk);
     return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+extern "C" int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* ratio, int64_t b,
+                             int64_t hk, int64_t sk, int64_t d, float threshold, void* stream)
+{
+    int64_t cols = 0;
+    int rc = check_kmean_args(k, mean, b, hk, sk, d, &cols);
+    if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
+    if (!gate) return B200ATTN_ERR_NULL;
+    if (!aligned(gate, 4) || (ratio && !aligned(ratio, 4))) return B200ATTN_ERR_ALIGN;
+    if (!std::isfinite(threshold)) return B200ATTN_ERR_SCALE;
+    int64_t n_bg;
+    if (!numel({b, hk}, &n_bg) || n_bg >= ((int64_t)1 << 31)) return B200ATTN_ERR_RANGE;
+    rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    const int64_t stride = (sk + 2047) / 2048;  // every key up to 2048, else a strided sample
+    const int64_t n_samp = (sk + stride - 1) / stride;
+    const int64_t col_ctas = (cols + kColsPerCta - 1) / kColsPerCta;
+    int64_t nchunks = (kTargetCtas + col_ctas * b - 1) / (col_ctas * b);
+    const int64_t max_chunks = (n_samp + kMinRowsPerChunk - 1) / kMinRowsPerChunk;
+    if (nchunks > max_chunks) nchunks = max_chunks;
+    if (nchunks > 1024) nchunks = 1024;
+    if (nchunks < 1) nchunks = 1;
+    const int64_t per_chunk = (n_samp + nchunks - 1) / nchunks;
+    nchunks = (n_samp + per_chunk - 1) / per_chunk;
+
+    float* partial = nullptr;
+    cudaMemPool_t pool = scratch_pool();
+    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&partial),
+                                         (size_t)(b * nchunks * 2 * cols) * sizeof(float), pool,
+                                         st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    dim3 g1((unsigned)col_ctas, (unsigned)nchunks, (unsigned)b);
+    k_gate_partial<<<g1, kThreads, 0, st>>>(static_cast<const uint4*>(k), partial, sk, cols,
+                                            stride, n_samp, per_chunk, (int)nchunks);
+    k_gate_fold<<<(unsigned)n_bg, kFoldThreads, 0, st>>>(partial, mean, gate, ratio, hk, d,
+                                                         (int)nchunks, (float)n_samp, threshold);
+    const bool launched = cudaGetLastError() == cudaSuccess;
+    if (cudaFreeAsync(partial, st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    return launched ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }
 
 extern "C" int k_smooth_sub(const void* k, const float* mean, void* k_out, int64_t b, int64_t hk,

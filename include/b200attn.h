@@ -183,6 +183,35 @@ B200ATTN_API int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, in
                                        int64_t sk, int64_t d, void* stream);
 
 /*
+ * k_smooth_gate -- the K-smoothing gate: sampled channel mean of K and a per-head decision.
+ *
+ * "[HIP] Mha v4: run the K-smoothing gate as one HIP call" (Summary, commit message) runs the
+ * gate as per-(batch*head, chunk) moments over a strided sample of the keys, then a per-head
+ * fold and the gate, as two deterministic kernels behind one call; it prints neither the stride
+ * nor the threshold. Reading:
+ *     sample   keys s = 0, stride, 2*stride, ... < sk, stride = ceil(sk / 2048) (every key when
+ *              sk <= 2048); n sampled keys
+ *     mu[bi,g,c] = (1/n) sum_s K[bi,s,g,c],   e[bi,g,c] = (1/n) sum_s K[bi,s,g,c]^2
+ *     ratio[bi,g] = sum_c mu^2 / sum_c e   (the share of K's energy in its channel mean; 0 when
+ *                                           the sampled K is all zero)
+ *     gate[bi,g] = ratio >= threshold
+ *     mean[bi,g,c] = gate ? mu : 0   (fp32; feed it to k_smooth_sub: where the gate is off,
+ *                                     K' = K)
+ * All sums in fp32 in a fixed order: the outputs are bit-identical from run to run.
+ *
+ *   k          device bf16 [b, sk, hk, d], 16-byte aligned. Read only.
+ *   mean       device fp32 [b, hk, d], 16-byte aligned. Fully written.
+ *   gate       device int32 [b, hk] (0 / 1), 4-byte aligned. Fully written.
+ *   ratio      device fp32 [b, hk], 4-byte aligned, or NULL. Fully written when given.
+ *   threshold  finite (NaN / inf -> ERR_SCALE).
+ *   b, hk, sk, d  as in k_smooth_mean (sk > 0, d in {64, 128, 256}).
+ * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`
+ * (as k_smooth_mean). Safe to call concurrently on different streams.
+ */
+B200ATTN_API int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* ratio, int64_t b,
+                               int64_t hk, int64_t sk, int64_t d, float threshold, void* stream);
+
+/*
  * k_smooth_sub -- subtract the channel mean from K: k_out = bf16_rne(float(K) - mean),
  * with mean[bi,g,c] broadcast over the sequence axis. This makes the smoothed K that the
  * attention pass then reads ("mean subtracted before attention"). k_out must not overlap k.

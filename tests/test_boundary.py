@@ -126,3 +126,16 @@ def test_attn_fwd_window_sink_rejects(kw, code):
 def test_window_sink_empty_problem_is_a_no_op():
     assert call_ws(b=0, q=None, k=None, v=None, o=None, lse=None, sinks=None) == 0
     assert call_ws(sq=0, q=None, o=None, lse=None) == 0
+
+
+def test_k_smooth_gate_rejects():
+    f = b2.lib.k_smooth_gate
+
+    def c(k=A, m=A, g=A, r=A, b=1, hk=2, sk=8, d=64, t=0.25):
+        return f(k, m, g, r, b, hk, sk, d, t, None)
+
+    assert c(d=96) == 4 and c(sk=0) == 2 and c(b=-1) == 2
+    assert c(k=None) == 1 and c(m=None) == 1 and c(g=None) == 1
+    assert c(k=A + 8) == 5 and c(m=A + 4) == 5 and c(g=A + 2) == 5 and c(r=A + 1) == 5
+    assert c(t=float("nan")) == 7 and c(t=float("inf")) == 7
+    assert c(b=0) == 0 and c(hk=0) == 0
