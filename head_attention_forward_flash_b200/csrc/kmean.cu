@@ -162,6 +162,7 @@ __global__ void __launch_bounds__(kFoldThreads)
     const int64_t cols = hk * d;
     const int64_t col = g * d + c;
     float gsum = 0.f, gsq = 0.f;
+#pragma unroll 4
     for (int ch = grp; ch < nchunks; ch += groups) {
         const float* src = partial + ((bi * nchunks + ch) * 2) * cols;
         gsum += src[col];
@@ -394,7 +395,8 @@ extern "C" int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* r
     const int64_t n_samp = (sk + stride - 1) / stride;
     const int64_t col_ctas = (cols + kColsPerCta - 1) / kColsPerCta;
     int64_t nchunks = (kTargetCtas + col_ctas * b - 1) / (col_ctas * b);
-    const int64_t max_chunks = (n_samp + kMinRowsPerChunk - 1) / kMinRowsPerChunk;
+    // at least 32 sampled rows per chunk: fewer partials for the per-head fold to read
+    const int64_t max_chunks = (n_samp + 31) / 32;
     if (nchunks > max_chunks) nchunks = max_chunks;
     if (nchunks > 1024) nchunks = 1024;
     if (nchunks < 1) nchunks = 1;
