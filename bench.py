@@ -213,6 +213,31 @@ def attn_source_hash():
 
 
 # ---------------------------------------------------------------------------------------------
+# multi-rank plumbing (replicas: every rank runs its own batch; ranks meet only for the barrier
+# and the max-over-ranks time)
+# ---------------------------------------------------------------------------------------------
+def rank_seed(seed: int, rank: int) -> int:
+    """Every rank draws its own independent batch."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' x (the slowest rank sets the job's time)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, flops_per_step: float, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------------
 def run_gpu(args):
@@ -233,18 +258,12 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     import head_attention_forward_flash_b200 as b2
 
     c = workloads.config(args.config)
     c_rank = dict(c)
-    c_rank["seed"] = c["seed"] + 7919 * rank  # every rank its own independent batch
+    c_rank["seed"] = rank_seed(c["seed"], rank)
     varlen = bool(c.get("varlen"))
     if varlen:  # packed sequences: [total, h, d] tensors and int32 offsets
         q_h, k_h, v_h, cuq_h, cuk_h = workloads.config_varlen_inputs(c_rank)
@@ -320,9 +339,9 @@ def run_gpu(args):
         raise RuntimeError(f"a kernel reported status {status} in the timed region")
 
     ms_local = sum(step_ms) / len(step_ms)
-    ms = max_over_ranks(ms_local)
+    ms = max_over_ranks(ms_local, world, dev)
     fl = workloads.flops(c)
-    value = world * fl / (ms * 1e-3) / 1e12
+    value = job_value(world, fl, ms)
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     achieved = fl / (attn_avg_ms * 1e-3) / 1e12
     peaks, peak_src = measured_peaks()
@@ -400,14 +419,14 @@ def run_gpu(args):
             ev1[s].record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(sum(ev0[s].elapsed_time(ev1[s]) for s in range(1, e_steps + 1))
-                              / e_steps)
+                              / e_steps, world, dev)
         h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
         if varlen:
             h2d += (cuq_h.numel() + cuk_h.numel()) * 4
         if sk_h is not None:
             h2d += sk_h.numel() * 4
         d2h = o.numel() * 2 + lse.numel() * 4
-        e2e = {"value": world * fl / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_value(world, fl, e_ms), "unit": "TFLOP/s",
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     cpu = None
