@@ -26,7 +26,7 @@ STATUS = {
     11: "ERR_SCRATCH",
 }
 EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
-           "attn_status_string", "attn_debug_status")
+           "attn_status_string", "attn_debug_status", "attn_debug_starve")
 
 
 class B200AttnError(RuntimeError):
@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_debug_status.argtypes = [vp]
     lib.attn_debug_status.restype = ctypes.c_int
+    lib.attn_debug_starve.argtypes = [i64]
+    lib.attn_debug_starve.restype = ctypes.c_int
     return lib
 
 
@@ -271,3 +273,9 @@ def attn_debug_status(stream=None) -> int:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream().cuda_stream
     return int(lib.attn_debug_status(s))
+
+
+def attn_debug_starve(timeout_us: int = 20000) -> None:
+    """Failure test: the next attention launch loads nothing and every wait gives up after
+    ``timeout_us``; attn_debug_status() then reports the timeout (status 10)."""
+    _check("attn_debug_starve", lib.attn_debug_starve(int(timeout_us)))

@@ -1,4 +1,5 @@
-// attn_api.cu -- C-ABI entry points attn_fwd, attn_status_string and attn_debug_status:
+// attn_api.cu -- C-ABI entry points attn_fwd, attn_fwd_varlen, attn_fwd_window_sink,
+// attn_status_string, attn_debug_status and attn_debug_starve:
 // argument checks, TMA descriptor encoding, head-dim dispatch and the kernel launch.
 #include <cmath>
 #include <cstring>
@@ -14,6 +15,10 @@ namespace b200 {
 
 // Device error word written by kernels whose bounded waits give up.
 __device__ int g_attn_status;
+
+// Failure test armed by attn_debug_starve: the wait limit of the next attention launch, or 0.
+std::mutex g_starve_mu;
+unsigned long long g_starve_timeout_ns = 0;
 
 namespace {
 
@@ -203,6 +208,16 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.idesc_qk = T::IDESC_QK | (scale < 0.f ? (1u << 13) : 0u);
     p.status = status;
     p.timeout_ns = 4000000000ull;  // 4 s: far above any legitimate wait
+    p.starve = 0;
+    {
+        // a pending failure test (attn_debug_starve) applies to this one launch
+        std::lock_guard<std::mutex> lk(g_starve_mu);
+        if (g_starve_timeout_ns > 0) {
+            p.starve = 1;
+            p.timeout_ns = g_starve_timeout_ns;
+            g_starve_timeout_ns = 0;
+        }
+    }
 
     const int64_t grid = p.n_units < n_sm ? p.n_units : n_sm;  // persistent: one CTA per SM
     kern<<<(unsigned)grid, T::NUM_THREADS, T::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
@@ -432,6 +447,14 @@ extern "C" const char* attn_status_string(int status)
         return "b*hk*d exceeds the fixed scratch of k_smooth_mean_noalloc (2^20 floats)";
     default: return "unknown status";
     }
+}
+
+extern "C" int attn_debug_starve(int64_t timeout_us)
+{
+    if (timeout_us < 1 || timeout_us > 1000000) return B200ATTN_ERR_RANGE;
+    std::lock_guard<std::mutex> lk(g_starve_mu);
+    g_starve_timeout_ns = (unsigned long long)timeout_us * 1000ull;
+    return B200ATTN_OK;
 }
 
 extern "C" int attn_debug_status(void* stream)

@@ -82,6 +82,7 @@ struct AttnParams {
     uint32_t idesc_qk;
     int* status;      // device error word
     unsigned long long timeout_ns;
+    int starve;       // failure test: the TMA producer loads nothing (see attn_debug_starve)
 };
 
 template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_,
@@ -405,7 +406,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         // ------------------------------ TMA producer ------------------------------
         // Walks the MMA warp's item sequence and issues each load at the point the MMA warp
         // will first need it (K_j at the Q K^T of item (j, 0), V_j at the P V of item (j, 0)).
-        if (lane == 0) {
+        // Failure test (p.starve): no tile is ever loaded, so every other role's first wait runs
+        // out; they all leave through the bounded abort and drain path.
+        if (lane == 0 && !p.starve) {
             int kq = 0, vq = 0;  // K / V items issued
             int q_cnt = 0;       // Q units issued
             bool ok = true;

@@ -233,6 +233,18 @@ B200ATTN_API const char* attn_status_string(int status);
  */
 B200ATTN_API int attn_debug_status(void* stream);
 
+/*
+ * attn_debug_starve -- failure test of the bounded waits (no counterpart on the pages; their
+ * stalls were found by timing only). Arms the next attention launch of this process (any entry
+ * point, any stream) so that its TMA producer loads nothing and every wait of the other roles is
+ * limited to timeout_us: they all give up, leave through the abort path (in-flight work drained,
+ * tensor memory freed), the launch completes, and attn_debug_status then reports
+ * B200ATTN_ERR_TIMEOUT. The device and its context stay usable; the launch's outputs are
+ * undefined. No fault, trap or hang is involved.
+ *   timeout_us  1 .. 1000000 (else B200ATTN_ERR_RANGE).
+ */
+B200ATTN_API int attn_debug_starve(int64_t timeout_us);
+
 #ifdef __cplusplus
 }
 #endif

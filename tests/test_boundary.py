@@ -139,3 +139,7 @@ def test_k_smooth_gate_rejects():
     assert c(k=A + 8) == 5 and c(m=A + 4) == 5 and c(g=A + 2) == 5 and c(r=A + 1) == 5
     assert c(t=float("nan")) == 7 and c(t=float("inf")) == 7
     assert c(b=0) == 0 and c(hk=0) == 0
+
+
+def test_debug_starve_range():
+    assert b2.lib.attn_debug_starve(0) == 6 and b2.lib.attn_debug_starve(2_000_000) == 6
