@@ -229,23 +229,22 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 // warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe>. Tensor
 // memory holds two score buffers, one O per query tile and (when it fits) each tile's Q; shared
 // memory holds the Q staging buffer and the K / V rings. The (tiles, warpgroups) choice per head
-// dim is the measured fastest on B200. The share of score pairs whose exp2 runs on the FMA pipe
-// is the measured best per head dim (3 of 8 at d64, 2 of 8 at d128 / d192, none at d256, which
-// is bound by the tensor core).
-using T64 = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 KB
+// dim is the measured fastest on B200 (d64: two tiles and two warpgroups, except for packed
+// sequences). The share of score pairs whose exp2 runs on the FMA pipe is the measured best per
+// head dim (3 of 8 at d64, 2 of 8 at d128 / d192, none at d256, which is bound by the tensor
+// core).
+using T64 = AttnTraits<64, 64, 128, 2, 2, true, 5, 5, 0x92u>;   // smem 32 + 80 + 80 (+32) KB
+using T64V = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 (+16) KB
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
 
-// Kernel variants: dense, packed sequences, and dense with window / sinks (compiled apart so
-// that the plain paths carry none of the extra bound logic).
+// Kernel variants: dense, dense with window / sinks (compiled apart so that the plain path
+// carries none of the extra bound logic), and packed sequences.
 template <class T>
-int dispatch(int causal, bool varlen, const void* q, const void* k, const void* v, void* out,
-             float* lse, const Shape& sh, float scale, cudaStream_t st)
+int dispatch_dense(int causal, const void* q, const void* k, const void* v, void* out,
+                   float* lse, const Shape& sh, float scale, cudaStream_t st)
 {
-    if (varlen)
-        return causal ? launch_attn<T, true, true, false>(q, k, v, out, lse, sh, scale, st)
-                      : launch_attn<T, false, true, false>(q, k, v, out, lse, sh, scale, st);
     if (sh.window >= 0 || sh.sinks)
         return causal ? launch_attn<T, true, false, true>(q, k, v, out, lse, sh, scale, st)
                       : launch_attn<T, false, false, true>(q, k, v, out, lse, sh, scale, st);
@@ -253,15 +252,33 @@ int dispatch(int causal, bool varlen, const void* q, const void* k, const void* 
                   : launch_attn<T, false, false, false>(q, k, v, out, lse, sh, scale, st);
 }
 
+template <class T>
+int dispatch_varlen(int causal, const void* q, const void* k, const void* v, void* out,
+                    float* lse, const Shape& sh, float scale, cudaStream_t st)
+{
+    return causal ? launch_attn<T, true, true, false>(q, k, v, out, lse, sh, scale, st)
+                  : launch_attn<T, false, true, false>(q, k, v, out, lse, sh, scale, st);
+}
+
+// d64 packed sequences use the one-warpgroup layout (measured faster there: 310 vs 278 TFLOP/s
+// on 8 sequences of 1024-2048; the two-tile layout is faster for dense and windowed d64).
 int dispatch_dims(int64_t dqk, int causal, bool varlen, const void* q, const void* k,
                   const void* v, void* out, float* lse, const Shape& sh, float scale,
                   cudaStream_t st)
 {
+    if (varlen) {
+        switch (dqk) {
+        case 64: return dispatch_varlen<T64V>(causal, q, k, v, out, lse, sh, scale, st);
+        case 128: return dispatch_varlen<T128>(causal, q, k, v, out, lse, sh, scale, st);
+        case 192: return dispatch_varlen<T192>(causal, q, k, v, out, lse, sh, scale, st);
+        default: return dispatch_varlen<T256>(causal, q, k, v, out, lse, sh, scale, st);
+        }
+    }
     switch (dqk) {
-    case 64: return dispatch<T64>(causal, varlen, q, k, v, out, lse, sh, scale, st);
-    case 128: return dispatch<T128>(causal, varlen, q, k, v, out, lse, sh, scale, st);
-    case 192: return dispatch<T192>(causal, varlen, q, k, v, out, lse, sh, scale, st);
-    default: return dispatch<T256>(causal, varlen, q, k, v, out, lse, sh, scale, st);
+    case 64: return dispatch_dense<T64>(causal, q, k, v, out, lse, sh, scale, st);
+    case 128: return dispatch_dense<T128>(causal, q, k, v, out, lse, sh, scale, st);
+    case 192: return dispatch_dense<T192>(causal, q, k, v, out, lse, sh, scale, st);
+    default: return dispatch_dense<T256>(causal, q, k, v, out, lse, sh, scale, st);
     }
 }
 
