@@ -202,13 +202,19 @@ class ClockSampler:
 
 
 def attn_source_hash():
-    """Hash of the attention kernel's sources (profiled traffic is valid only for these)."""
+    """Hash of the attention kernel's sources with comments and blank space removed (profiled
+    traffic is valid only for this code; editing a comment does not change it)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "head_attention_forward_flash_b200", "csrc")
     for f in ("attn_fwd_kernel.cuh", "sm100_ptx.cuh", "attn_api.cu"):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(d, f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)   # block comments
+        src = re.sub(r"//[^\n]*", " ", src)                # line comments
+        src = re.sub(r"\s+", " ", src)
+        h.update(src.encode())
     return h.hexdigest()[:16]
 
 

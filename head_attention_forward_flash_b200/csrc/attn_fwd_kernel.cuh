@@ -5,36 +5,40 @@
 // forward of "Tune MHA config & small-head pipeline pathology" (Motivation; shapes in "Source of
 // shapes"), re-designed for the 5th-generation tensor core.
 //
-// Work unit: NT consecutive 128-row query tiles (NT = 2, or 1 for d256) of one (batch, query
-// head). Every K/V tile brought into shared memory serves all NT query tiles, which halves the
-// L2 -> SM traffic per FLOP and doubles the time each K/V slot can hide load latency. Persistent
-// kernel: one CTA per SM walks its units head-major (CTAs working at the same time share K/V
-// in L2), the units that see the most keys (causal) first within a head. The pipeline does not
-// drain between units.
+// Work unit: NT consecutive 128-row query tiles (NT = 1 or 2, per head dim and layout) of one
+// (batch or packed sequence, query head). Every K/V tile brought into shared memory serves all
+// NT query tiles, which halves the L2 -> SM traffic per FLOP when NT = 2. Persistent kernel: one
+// CTA per SM takes units in rounds, in the order AttnParams::order selects (round robin, snake,
+// or weight-major snake); within a head the units that see the most keys (causal) come first.
+// The pipeline does not drain between units.
 //
 // Items: the pipeline steps through "items" (key block j, query tile t) in the order
 // (0,0) (0,1) (1,0) (1,1) ... for NT = 2, or (0) (1) (2) ... for NT = 1. Item g uses score buffer
 // g % 2, so one item's Q K^T runs on the tensor core while the previous item's softmax runs.
 //
-// Roles (NSM softmax warpgroups + 2 warps): NSM = 1 (192 threads) or NSM = NT = 2 (320 threads).
-//   softmax + epilogue warps: thread r owns row r (= TMEM lane r) of a query tile. Turns each
-//              score block S into P (online softmax: exp2 with the scale folded into one FMA,
-//              lazy rescaling of O; the FMA and the row-sum adds run as packed fp32x2
-//              instructions, two scores each), and writes each tile's finished O rows (divided by the row
-//              sums) and LSE right after handing over that tile's first P of the next unit. When
-//              Q lives in TMEM they also copy each tile's Q from the shared-memory staging buffer
-//              into TMEM once the tile's last Q K^T of the current unit has landed.
-//              NSM = 1: warps 0-3 take every item in order and keep the whole score row in
-//              registers (at most two warps per SM sub-partition allow up to 255 registers).
-//              NSM = 2: warps 4t..4t+3 own query tile t, so the two tiles' softmax run side by
-//              side; within the 10-warp register budget each thread reads its score row from
-//              TMEM twice (max, then exp) in 32-column chunks.
+// Roles: NSM softmax warpgroups, then the MMA warp and the TMA warp. NSM = 1: 192 threads.
+// NSM = 2: 384 threads (a third warpgroup holds the MMA and TMA warps and two idle warps, so
+// that setmaxnreg can move registers from it to the softmax warpgroups).
+//   softmax + epilogue warps: thread r owns row r (= TMEM lane r) of a query tile and keeps its
+//              whole score row of the current item in registers. Turns each score block S into
+//              P (online softmax: exp2 with the scale folded into one packed fp32x2 FMA, part of
+//              the exp2 on the FMA pipe, lazy rescaling of O, row sums as packed fp32x2 adds),
+//              and writes each tile's finished O rows (divided by the row sums) and LSE right
+//              after handing over that tile's first P of the next unit. When Q lives in TMEM they
+//              also copy each tile's Q from the shared-memory staging buffer into TMEM once the
+//              tile's last Q K^T of the current unit has landed.
+//              NSM = 1: warps 0-3 take every item in order. NSM = 2: warps 4t..4t+3 own query
+//              tile t, so the two tiles' softmax run side by side.
 //   warp 4*NSM   MMA issuer (one thread): S = Q K^T and O += P V. A operand: Q from TMEM or
 //              shared memory, then P from TMEM; B operand: K, V from shared memory; fp32
 //              accumulators in TMEM.
 //   warp 4*NSM+1 TMA producer (one thread): each unit's Q into the staging buffer, and K, V
 //              tiles through two rings of shared-memory slots, in the order the MMA warp takes
 //              them.
+//
+// Template flags: CAUSAL; VARLEN (packed sequences: per-unit offsets from cu_seqlens); EXT
+// (sliding window and sinks: a first key block per unit, a lower per-key bound, and each row's
+// reference and sum started at the head's sink logit).
 //
 // Tensor memory (128 lanes x 512 columns of 32 bit): S0 | S1 (BN columns each; P in bf16 pairs
 // overwrites the first BN/2 columns of its own S buffer) | O for each query tile (DV fp32
