@@ -6,7 +6,8 @@
  *     keeps a caller pointer after the call returns.
  *   - Tensors are contiguous, BSHD, row-major (last dimension fastest):
  *       Q [b, sq, hq, dqk], K [b, sk, hk, dqk], V [b, sk, hk, dv], O [b, sq, hq, dv]  (bf16)
- *       LSE [b, hq, sq] (fp32, natural log), K mean [b, hk, d] (fp32).
+ *       LSE [b, hq, sq] (fp32, natural log), K mean [b, hk, d] (fp32);
+ *     attn_fwd_varlen packs sequences along the row axis instead ([total, h, d], LSE [hq, total]).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
  *     enqueued asynchronously on it; the call does not synchronise.
  *   - Return value: B200ATTN_OK (0) on success, otherwise one of the status codes below.
