@@ -8,6 +8,9 @@ The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, one left-to-right loop
 its header for the definition it follows). This module compiles it with gcc, loads it with
 ctypes and marshals numpy arrays of raw bf16 bit patterns (uint16) in and fp64 results out.
 
+The FP8 (E4M3) recipe -- codes, the per-head quantiser and attention on decoded inputs -- is in
+``oracle.fp8`` (numpy, on top of the fp64-input entry points of ``attn_oracle.c``).
+
 Parity status: every function here is pinned by ``tests/test_oracle.py`` against torch's fp64
 scaled-dot-product attention and logsumexp, numpy's fp64 mean, torch's fp32->bf16 cast, closed
 forms and invariants; none is "parity unpinned".
@@ -57,6 +60,12 @@ def _bind(lib):
     lib.oracle_attn_full_ex.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
                                         _i64, _p, _p, _p, ctypes.c_int]
     lib.oracle_attn_full_ex.restype = ctypes.c_int
+    lib.oracle_attn_full_f64.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
+                                                                   _p, _p, ctypes.c_int]
+    lib.oracle_attn_full_f64.restype = ctypes.c_int
+    lib.oracle_attn_rows_f64.argtypes = [_p, _p, _p] + [_i64] * 7 + [ctypes.c_int, ctypes.c_double,
+                                                                   _p, _i64, _p, _p, ctypes.c_int]
+    lib.oracle_attn_rows_f64.restype = ctypes.c_int
     lib.oracle_k_mean.argtypes = [_p, _i64, _i64, _i64, _i64, _p, _p]
     lib.oracle_k_mean.restype = ctypes.c_int
     lib.oracle_k_gate.argtypes = [_p, _i64, _i64, _i64, _i64, ctypes.c_double, _p, _p, _p, _p]

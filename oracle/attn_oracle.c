@@ -35,6 +35,8 @@
  *
  * Inputs are exchanged as raw bf16 bit patterns (uint16), BSHD and contiguous:
  *   Q [b,sq,hq,dqk], K [b,sk,hk,dqk], V [b,sk,hk,dv], O [b,sq,hq,dv], LSE [b,hq,sq].
+ * The *_f64 entry points take the same layouts as fp64 values instead (used for the FP8
+ * recipe, whose inputs are E4M3 codes times per-head scales, decoded by the Python side).
  * Every sum is a plain left-to-right loop in double precision.
  */
 #include <math.h>
@@ -79,6 +81,7 @@ uint16_t oracle_bf16_rne(double x)
 
 typedef struct {
     const uint16_t *q, *k, *v;
+    const double *qf, *kf, *vf; /* fp64 inputs instead of q, k, v when non-NULL */
     int64_t b, hq, hk, sq, sk, dqk, dv;
     int causal;
     double scale;
@@ -90,6 +93,12 @@ typedef struct {
     int64_t next; /* guarded by lock */
     pthread_mutex_t lock;
 } attn_job;
+
+/* Input element idx of one of the three tensors: bf16 bits or an fp64 value. */
+static double in_val(const uint16_t *bits, const double *vals, int64_t idx)
+{
+    return vals ? vals[idx] : bf16_value(bits[idx]);
+}
 
 /* One output row, straight from the definition above. s holds sk doubles, qd holds dqk. */
 static void attn_row(const attn_job *a, int64_t bi, int64_t h, int64_t i, double *s, double *qd,
@@ -110,13 +119,13 @@ static void attn_row(const attn_job *a, int64_t bi, int64_t h, int64_t i, double
         return;
     }
     const int64_t n = hi - lo + 1;
-    const uint16_t *qrow = a->q + ((bi * a->sq + i) * a->hq + h) * a->dqk;
-    for (int64_t c = 0; c < a->dqk; ++c) qd[c] = bf16_value(qrow[c]);
+    const int64_t qoff = ((bi * a->sq + i) * a->hq + h) * a->dqk;
+    for (int64_t c = 0; c < a->dqk; ++c) qd[c] = in_val(a->q, a->qf, qoff + c);
 
     for (int64_t j = 0; j < n; ++j) {
-        const uint16_t *krow = a->k + ((bi * a->sk + lo + j) * a->hk + g) * a->dqk;
+        const int64_t koff = ((bi * a->sk + lo + j) * a->hk + g) * a->dqk;
         double dot = 0.0;
-        for (int64_t c = 0; c < a->dqk; ++c) dot += qd[c] * bf16_value(krow[c]);
+        for (int64_t c = 0; c < a->dqk; ++c) dot += qd[c] * in_val(a->k, a->kf, koff + c);
         s[j] = a->scale * dot;
     }
     double m = s[0];
@@ -131,8 +140,8 @@ static void attn_row(const attn_job *a, int64_t bi, int64_t h, int64_t i, double
     if (has_sink) l += exp(sink - m);
     for (int64_t c = 0; c < a->dv; ++c) o_row[c] = 0.0;
     for (int64_t j = 0; j < n; ++j) {
-        const uint16_t *vrow = a->v + ((bi * a->sk + lo + j) * a->hk + g) * a->dv;
-        for (int64_t c = 0; c < a->dv; ++c) o_row[c] += s[j] * bf16_value(vrow[c]);
+        const int64_t voff = ((bi * a->sk + lo + j) * a->hk + g) * a->dv;
+        for (int64_t c = 0; c < a->dv; ++c) o_row[c] += s[j] * in_val(a->v, a->vf, voff + c);
     }
     for (int64_t c = 0; c < a->dv; ++c) o_row[c] /= l;
     *lse_out = m + log(l);
@@ -210,8 +219,8 @@ int oracle_attn_rows_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int causal, double scale, int64_t window, const double *sinks,
                         const int64_t *rows, int64_t nrows, double *o, double *lse, int nthreads)
 {
-    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, window, sinks, rows,
-                  nrows, o, lse};
+    attn_job a = {q, k, v, NULL, NULL, NULL, b, hq, hk, sq, sk, dqk, dv, causal, scale, window,
+                  sinks, rows, nrows, o, lse};
     for (int64_t r = 0; r < nrows; ++r)
         if (rows[3 * r] < 0 || rows[3 * r] >= b || rows[3 * r + 1] < 0 ||
             rows[3 * r + 1] >= hq || rows[3 * r + 2] < 0 || rows[3 * r + 2] >= sq)
@@ -235,8 +244,33 @@ int oracle_attn_full_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int causal, double scale, int64_t window, const double *sinks, double *o,
                         double *lse, int nthreads)
 {
-    attn_job a = {q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, window, sinks, NULL,
-                  b * sq * hq, o, lse};
+    attn_job a = {q, k, v, NULL, NULL, NULL, b, hq, hk, sq, sk, dqk, dv, causal, scale, window,
+                  sinks, NULL, b * sq * hq, o, lse};
+    return run_attn(&a, nthreads);
+}
+
+/* Every row from fp64 inputs (no window, no sink). */
+int oracle_attn_full_f64(const double *q, const double *k, const double *v, int64_t b,
+                         int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                         int causal, double scale, double *o, double *lse, int nthreads)
+{
+    attn_job a = {NULL, NULL, NULL, q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, -1, NULL,
+                  NULL, b * sq * hq, o, lse};
+    return run_attn(&a, nthreads);
+}
+
+/* Selected rows from fp64 inputs (no window, no sink). */
+int oracle_attn_rows_f64(const double *q, const double *k, const double *v, int64_t b,
+                         int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
+                         int causal, double scale, const int64_t *rows, int64_t nrows, double *o,
+                         double *lse, int nthreads)
+{
+    attn_job a = {NULL, NULL, NULL, q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, -1, NULL,
+                  rows, nrows, o, lse};
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[3 * r] < 0 || rows[3 * r] >= b || rows[3 * r + 1] < 0 ||
+            rows[3 * r + 1] >= hq || rows[3 * r + 2] < 0 || rows[3 * r + 2] >= sq)
+            return 2;
     return run_attn(&a, nthreads);
 }
 
