@@ -9,7 +9,8 @@ importing this package fails loudly when the library is missing.
 
 Raw C entry points, with the header's names and argument order, are exposed through ``lib``
 (a ``ctypes.CDLL``): ``lib.attn_fwd``, ``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``,
-``lib.k_smooth_sub``, ``lib.attn_status_string``, ``lib.attn_debug_status``.
+``lib.k_smooth_sub``, ``lib.fp8_quantize``, ``lib.attn_fwd_fp8``, ``lib.attn_status_string``,
+``lib.attn_debug_status``.
 """
 from __future__ import annotations
 
@@ -25,7 +26,8 @@ STATUS = {
     6: "ERR_RANGE", 7: "ERR_SCALE", 8: "ERR_ARCH", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
     11: "ERR_SCRATCH",
 }
-EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "attn_fwd_fp8", "fp8_quantize",
+           "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
            "attn_status_string", "attn_debug_status", "attn_debug_starve")
 
 
@@ -51,6 +53,11 @@ def _load() -> ctypes.CDLL:
     lib.attn_fwd_window_sink.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
                                          ctypes.c_int, i64, ctypes.c_float, vp]
     lib.attn_fwd_window_sink.restype = ctypes.c_int
+    lib.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64,
+                                 ctypes.c_int, ctypes.c_float, vp]
+    lib.attn_fwd_fp8.restype = ctypes.c_int
+    lib.fp8_quantize.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.fp8_quantize.restype = ctypes.c_int
     lib.k_smooth_mean.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean.restype = ctypes.c_int
     lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
@@ -197,6 +204,69 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, caus
                              total_k, int(max_seqlen_q), dqk, dv, 1 if causal else 0,
                              float(scale), _stream_ptr(q))
     _check("attn_fwd_varlen", st)
+    return out, lse
+
+
+def _codes(t, name, dims):
+    import torch
+    _want(t, name, dims)
+    if t.dtype not in (torch.uint8, torch.float8_e4m3fn):
+        raise TypeError(f"{name} must hold E4M3 codes (uint8 or float8_e4m3fn)")
+
+
+def fp8_quantize(x, mean=None, out=None, descale=None):
+    """E4M3 codes of a bf16 BSHD tensor x [b, s, h, d] with one fp32 descale per (batch, head)
+    (amax / 448); ``mean`` ([b, h, d] fp32, e.g. from k_smooth_mean or k_smooth_gate) is
+    subtracted first. Returns ``(codes [b, s, h, d] uint8, descale [b, h] fp32)``."""
+    import torch
+    _want(x, "x", 4)
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    b, s, h, d = x.shape
+    if mean is not None:
+        _want(mean, "mean", 3)
+        if mean.dtype != torch.float32 or tuple(mean.shape) != (b, h, d):
+            raise ValueError("mean must be float32 [b, h, d]")
+    if out is None:
+        out = torch.empty((b, s, h, d), dtype=torch.uint8, device=x.device)
+    if descale is None:
+        descale = torch.empty((b, h), dtype=torch.float32, device=x.device)
+    _check("fp8_quantize", lib.fp8_quantize(x.data_ptr(),
+                                            mean.data_ptr() if mean is not None else None,
+                                            out.data_ptr(), descale.data_ptr(), b, s, h, d,
+                                            _stream_ptr(x)))
+    return out, descale
+
+
+def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal: bool = False,
+                 scale: float | None = None, out=None, lse=None, return_lse: bool = True):
+    """attn_fwd on E4M3 inputs: q8 [b, sq, hq, 128], k8 [b, sk, hk, 128], v8 [b, sk, hk, 128]
+    (uint8 or float8_e4m3fn CUDA tensors) with fp32 descales q_descale [b, hq], k_descale and
+    v_descale [b, hk]. Returns ``(out [b, sq, hq, 128] bf16, lse [b, hq, sq] fp32 or None)``."""
+    import torch
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _codes(t, name, 4)
+    b, sq, hq, dqk = q8.shape
+    bk, sk, hk, dqk2 = k8.shape
+    bv, skv, hkv, dv = v8.shape
+    if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
+        raise ValueError("inconsistent q/k/v shapes")
+    for name, t, n in (("q_descale", q_descale, hq), ("k_descale", k_descale, hk),
+                       ("v_descale", v_descale, hk)):
+        _want(t, name, 2)
+        if t.dtype != torch.float32 or tuple(t.shape) != (b, n):
+            raise ValueError(f"{name} must be float32 [b, {n}]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    if out is None:
+        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q8.device)
+    if return_lse and lse is None:
+        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q8.device)
+    st = lib.attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_descale.data_ptr(),
+                          k_descale.data_ptr(), v_descale.data_ptr(), out.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
+                          1 if causal else 0, float(scale), _stream_ptr(q8))
+    _check("attn_fwd_fp8", st)
     return out, lse
 
 

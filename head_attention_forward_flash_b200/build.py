@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libb200attn.so")
-SOURCES = ["attn_api.cu", "kmean.cu"]
+SOURCES = ["attn_api.cu", "kmean.cu", "fp8_quant.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,5 +1,5 @@
 // attn_api.cu -- C-ABI entry points attn_fwd, attn_fwd_varlen, attn_fwd_window_sink,
-// attn_status_string, attn_debug_status and attn_debug_starve:
+// attn_fwd_fp8, attn_status_string, attn_debug_status and attn_debug_starve:
 // argument checks, TMA descriptor encoding, head-dim dispatch and the kernel launch.
 #include <cmath>
 #include <cstring>
@@ -55,19 +55,21 @@ int* status_word()
     return addr[dev];
 }
 
-// 4-D bf16 tensor map over a BSHD tensor [b, s, h, d] (innermost first: d, h, s, b), box
-// {64 channels, 1 head, box_rows rows, 1 batch}, 128-byte swizzle, zero fill out of bounds.
+// 4-D tensor map over a BSHD tensor [b, s, h, d] (innermost first: d, h, s, b) of bf16
+// (eb = 2) or 8-bit codes (eb = 1), box {128 bytes of channels, 1 head, box_rows rows, 1 batch},
+// 128-byte swizzle, zero fill out of bounds.
 int encode_bshd(CUtensorMap* map, const void* base, int64_t b, int64_t s, int64_t h, int64_t d,
-                int box_rows)
+                int box_rows, int eb = 2)
 {
     auto fn = encode_fn();
     if (!fn) return B200ATTN_ERR_CUDA;
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)h, (cuuint64_t)s, (cuuint64_t)b};
-    const cuuint64_t strides[3] = {(cuuint64_t)(d * 2), (cuuint64_t)(h * d * 2),
-                                   (cuuint64_t)(s * h * d * 2)};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+    const cuuint64_t strides[3] = {(cuuint64_t)(d * eb), (cuuint64_t)(h * d * eb),
+                                   (cuuint64_t)(s * h * d * eb)};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+    CUresult r = fn(map, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                    4, const_cast<void*>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? B200ATTN_OK : B200ATTN_ERR_CUDA;
@@ -110,6 +112,10 @@ struct Shape {
     int64_t total_q = 0, total_k = 0;
     int64_t window = -1;          // left window, < 0: none
     const float* sinks = nullptr;  // per query head sink logits, or null
+    // E4M3 inputs: per (batch, head) descales of Q [b, hq], K and V [b, hk]
+    const float* q_descale = nullptr;
+    const float* k_descale = nullptr;
+    const float* v_descale = nullptr;
 };
 
 template <class T, bool CAUSAL, bool VARLEN, bool EXT>
@@ -150,9 +156,9 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     const int64_t mq = VARLEN ? sh.total_q : sq;
     const int64_t mk = VARLEN ? sh.total_k : sk;
     CUtensorMap tq, tk, tv, to;
-    int rc = encode_bshd(&tq, q, mb, mq, hq, T::DQK, T::BM);
-    if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, mb, mk, hk, T::DQK, T::BN);
-    if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, mb, mk, hk, T::DV, T::BN);
+    int rc = encode_bshd(&tq, q, mb, mq, hq, T::DQK, T::BM, T::EB);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tk, k, mb, mk, hk, T::DQK, T::BN, T::EB);
+    if (rc == B200ATTN_OK) rc = encode_bshd(&tv, v, mb, mk, hk, T::DV, T::BN, T::EB);
     // O is stored per warp: boxes of 32 rows (only used when the kernel stages O for TMA)
     if (rc == B200ATTN_OK) rc = encode_bshd(&to, out, mb, mq, hq, T::DV, 32);
     if (rc != B200ATTN_OK) return rc;
@@ -174,6 +180,9 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     p.total_k = sh.total_k;
     p.window = sh.window;
     p.sinks = sh.sinks;
+    p.q_descale = sh.q_descale;
+    p.k_descale = sh.k_descale;
+    p.v_descale = sh.v_descale;
     p.group = hq / hk;
     p.n_qu = (sq + T::NT * T::BM - 1) / (T::NT * T::BM);
     p.n_units = b * hq * p.n_qu;  // below 2^31 (checked by attn_fwd)
@@ -190,7 +199,8 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     // window band) take plain round robin, and so do packed sequences, whose unit costs depend
     // on lengths the host does not see (measured: weight-major order was slower there).
     {
-        const double kv_bytes = (double)(b * sk) * (double)hk * (double)(T::DQK + T::DV) * 2.0;
+        const double kv_bytes =
+            (double)(b * sk) * (double)hk * (double)(T::DQK + T::DV) * (double)T::EB;
         if (!CAUSAL || VARLEN || (EXT && sh.window >= 0))
             p.order = 0;
         else if (b * hk <= 16 || kv_bytes <= 64.0e6)
@@ -238,6 +248,9 @@ using T64V = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
+// E4M3 inputs, (128, 128): the d128 layout with half-size tiles, so four K and four V slots fit
+// next to the Q staging buffer and the O staging tile.
+using T128F8 = AttnTraits<128, 128, 128, 2, 2, false, 4, 4, 0x11u, true>;  // 32 + 64 + 64 (+64) KB
 
 // Kernel variants: dense, dense with window / sinks (compiled apart so that the plain path
 // carries none of the extra bound logic), and packed sequences.
@@ -442,6 +455,53 @@ extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void
     sh.total_q = total_q;
     sh.total_k = total_k;
     return dispatch_dims(dqk, causal, true, q, k, v, out, lse, sh, scale, st);
+}
+
+extern "C" int attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_descale,
+                            const float* k_descale, const float* v_descale, void* out, float* lse,
+                            int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk,
+                            int64_t dv, int causal, float scale, void* stream)
+{
+    if (b < 0 || hq < 0 || sq < 0 || sk < 0 || hk <= 0) return B200ATTN_ERR_SHAPE;
+    if (hq % hk != 0) return B200ATTN_ERR_GQA;
+    if (!(dqk == 128 && dv == 128)) return B200ATTN_ERR_HEADDIM;
+    if (!std::isfinite(scale)) return B200ATTN_ERR_SCALE;
+    int64_t n_q, n_k, n_v, n_o, n_l, n_units;
+    if (!numel({b, sq, hq, dqk}, &n_q) || !numel({b, sk, hk, dqk}, &n_k) ||
+        !numel({b, sk, hk, dv}, &n_v) || !numel({b, sq, hq, dv, 2}, &n_o) ||
+        !numel({b, hq, sq, 4}, &n_l) || !numel({b, hq, (sq + 127) / 128}, &n_units) ||
+        n_units >= ((int64_t)1 << 31))
+        return B200ATTN_ERR_RANGE;
+    if (n_o == 0) return B200ATTN_OK;  // b, hq or sq is zero: nothing to compute
+    if (!q8 || !out || !q_descale || (sk > 0 && (!k8 || !v8 || !k_descale || !v_descale)))
+        return B200ATTN_ERR_NULL;
+    if (!aligned(q8, 16) || !aligned(out, 16) || (k8 && !aligned(k8, 16)) ||
+        (v8 && !aligned(v8, 16)) || (lse && !aligned(lse, 4)) || !aligned(q_descale, 4) ||
+        (k_descale && !aligned(k_descale, 4)) || (v_descale && !aligned(v_descale, 4)))
+        return B200ATTN_ERR_ALIGN;
+    if (!tma_extent_ok(b, sq, hq, dqk) ||
+        (sk > 0 && (!tma_extent_ok(b, sk, hk, dqk) || !tma_extent_ok(b, sk, hk, dv))))
+        return B200ATTN_ERR_RANGE;
+    int rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (sk == 0) {
+        fill_empty_rows<<<296, 256, 0, st>>>(static_cast<__nv_bfloat16*>(out), n_o / 2, lse,
+                                             n_l / 4);
+        return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+    }
+    Shape sh;
+    sh.b = b;
+    sh.hq = hq;
+    sh.hk = hk;
+    sh.sq = sq;
+    sh.sk = sk;
+    sh.q_descale = q_descale;
+    sh.k_descale = k_descale;
+    sh.v_descale = v_descale;
+    return causal ? launch_attn<T128F8, true, false, false>(q8, k8, v8, out, lse, sh, scale, st)
+                  : launch_attn<T128F8, false, false, false>(q8, k8, v8, out, lse, sh, scale, st);
 }
 
 extern "C" const char* attn_status_string(int status)

@@ -87,10 +87,14 @@ struct AttnParams {
     int* status;      // device error word
     unsigned long long timeout_ns;
     int starve;       // failure test: the TMA producer loads nothing (see attn_debug_starve)
+    // E4M3 inputs: fp32 descales per (batch, head) of Q [b, hq], K and V [b, hk] (else null)
+    const float* q_descale;
+    const float* k_descale;
+    const float* v_descale;
 };
 
 template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_,
-          uint32_t EXP_FMA_PAIRS_ = 0>
+          uint32_t EXP_FMA_PAIRS_ = 0, bool FP8_ = false>
 struct AttnTraits {
     static constexpr int DQK = DQK_;
     static constexpr int DV = DV_;
@@ -101,14 +105,21 @@ struct AttnTraits {
     static constexpr bool Q_TMEM = Q_TMEM_; // Q as the TMEM A operand (else from shared memory)
     static constexpr int NK = NK_;          // K slots
     static constexpr int NV = NV_;          // V slots
-    static constexpr int QCH = DQK / 64;    // 128-byte (64-element) column chunks of a Q/K row
-    static constexpr int VCH = DV / 64;
-    static constexpr uint32_t CHUNK_BYTES = BN * 128;   // one 64-column TMA box of K or V
-    static constexpr uint32_t QCHUNK_BYTES = BM * 128;  // one 64-column TMA box of Q
-    static constexpr uint32_t Q_TILE_BYTES = BM * DQK * 2;
+    // E4M3 Q, K, V (kind::f8f6f4 MMAs, P in E4M3) instead of bf16 (kind::f16, P in bf16)
+    static constexpr bool FP8 = FP8_;
+    static constexpr int EB = FP8 ? 1 : 2;    // bytes per input element
+    static constexpr int CE = 128 / EB;       // elements per 128-byte swizzled row chunk
+    static constexpr int KSTEP = 32 / EB;     // K per MMA instruction: 32 bytes of a row
+    static constexpr int QCH = DQK * EB / 128;  // 128-byte column chunks of a Q/K row
+    static constexpr int VCH = DV * EB / 128;
+    static constexpr uint32_t CHUNK_BYTES = BN * 128;   // one column chunk (TMA box) of K or V
+    static constexpr uint32_t QCHUNK_BYTES = BM * 128;  // one column chunk (TMA box) of Q
+    static constexpr uint32_t Q_TILE_BYTES = BM * DQK * EB;
     static constexpr uint32_t Q_BYTES = NT * Q_TILE_BYTES;
-    static constexpr uint32_t K_TILE_BYTES = BN * DQK * 2;
-    static constexpr uint32_t V_TILE_BYTES = BN * DV * 2;
+    static constexpr uint32_t K_TILE_BYTES = BN * DQK * EB;
+    static constexpr uint32_t V_TILE_BYTES = BN * DV * EB;
+    static_assert(!FP8 || (!Q_TMEM && (DQK * EB) % 128 == 0 && (DV * EB) % 128 == 0),
+                  "E4M3 inputs: Q from shared memory, whole 128-byte row chunks");
     // tensor memory columns
     static constexpr uint32_t O_COL0 = 2 * BN;
     static constexpr uint32_t Q_COL0 = 2 * BN + NT * DV;
@@ -151,8 +162,10 @@ struct AttnTraits {
     // Score pairs whose exp2 runs on the FMA pipe (exp2_fma_pair) rather than the MUFU unit: bit
     // k set = pairs with index k mod 8 in each row, in the one-warpgroup softmax.
     static constexpr uint32_t EXP_FMA_PAIRS = EXP_FMA_PAIRS_;
-    static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, BN, false, false);
-    static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, DV, false, true);
+    static constexpr uint32_t IDESC_QK =
+        FP8 ? make_idesc_e4m3(128, BN, false, false) : make_idesc_bf16(128, BN, false, false);
+    static constexpr uint32_t IDESC_PV =
+        FP8 ? make_idesc_e4m3(128, DV, false, true) : make_idesc_bf16(128, DV, false, true);
 };
 
 // Wait bounded only by time (used to drain in-flight copies / MMAs before exit, also after an
@@ -255,10 +268,27 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
     return t;
 }
 
-// S = Q K^T for one query tile and one key block: DQK/16 MMAs of M128 x N=BN x K16. K (and Q
-// when staged in shared memory) are K-major 128-byte swizzled tiles in 64-column chunks, so
-// k-step kk starts (kk / 4) chunks and (kk % 4) * 32 bytes in. q is a TMEM column (Q in TMEM)
-// or a shared-memory address.
+// The MMA forms of the traits' input type.
+template <class T>
+__device__ __forceinline__ void mma_ss_t(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc)
+{
+    if constexpr (T::FP8) mma_ss_f8(d, a, b, idesc, acc);
+    else mma_ss(d, a, b, idesc, acc);
+}
+
+template <class T>
+__device__ __forceinline__ void mma_ts_t(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc)
+{
+    if constexpr (T::FP8) mma_ts_f8(d, a, b, idesc, acc);
+    else mma_ts(d, a, b, idesc, acc);
+}
+
+// S = Q K^T for one query tile and one key block: one MMA of M128 x N=BN x K=KSTEP per 32
+// bytes of a row (DQK/16 for bf16, DQK/32 for E4M3). K (and Q when staged in shared memory)
+// are K-major 128-byte swizzled tiles in 128-byte column chunks, so k-step kk starts (kk / 4)
+// chunks and (kk % 4) * 32 bytes in. q is a TMEM column (Q in TMEM) or a shared-memory address.
 template <class T>
 __device__ __forceinline__ void issue_qk_mmas(uint32_t d_tmem, uint32_t q, uint32_t kaddr,
                                               uint32_t idesc)
@@ -273,24 +303,25 @@ __device__ __forceinline__ void issue_qk_mmas(uint32_t d_tmem, uint32_t q, uint3
     } else {
         const uint64_t a0 = make_sdesc_sw128(q, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < T::DQK / 16; ++kk)
-            mma_ss(d_tmem, sdesc_advance(a0, (kk >> 2) * T::QCHUNK_BYTES + (kk & 3) * 32),
+        for (int kk = 0; kk < T::DQK * T::EB / 32; ++kk)
+            mma_ss_t<T>(d_tmem, sdesc_advance(a0, (kk >> 2) * T::QCHUNK_BYTES + (kk & 3) * 32),
                    sdesc_advance(b0, (kk >> 2) * T::CHUNK_BYTES + (kk & 3) * 32), idesc,
                    kk > 0 ? 1u : 0u);
     }
 }
 
-// O += P V for one query tile and one key block: BN/16 MMAs of M128 x N=DV x K16 with P (bf16
-// pairs) from TMEM and V an MN-major 128-byte swizzled tile (16 keys = 2048 bytes per k-step).
+// O += P V for one query tile and one key block: BN/KSTEP MMAs of M128 x N=DV x K=KSTEP with P
+// from TMEM (8 columns = 32 bytes per k-step: 16 bf16 or 32 E4M3 weights of a row) and V an
+// MN-major 128-byte swizzled tile (KSTEP keys = KSTEP * 128 bytes per k-step).
 template <class T>
 __device__ __forceinline__ void issue_pv_mmas(uint32_t o_tmem, uint32_t p_tmem, uint32_t vaddr,
                                               bool accumulate)
 {
     const uint64_t b0 = make_sdesc_sw128(vaddr, T::CHUNK_BYTES, 1024);
 #pragma unroll
-    for (int kk = 0; kk < T::BN / 16; ++kk)
-        mma_ts(o_tmem, p_tmem + kk * 8, sdesc_advance(b0, kk * 2048), T::IDESC_PV,
-               (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < T::BN / T::KSTEP; ++kk)
+        mma_ts_t<T>(o_tmem, p_tmem + kk * 8, sdesc_advance(b0, kk * T::KSTEP * 128), T::IDESC_PV,
+                    (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // EXT: the sliding window and the sinks of AttnParams are honoured (compiled out otherwise).
@@ -426,7 +457,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 for (int tt = 0; tt < NT; ++tt)
                     for (int ch = 0; ch < T::QCH; ++ch)
                         tma_load_4d(q_stage + tt * T::Q_TILE_BYTES + ch * T::QCHUNK_BYTES, &tmap_q,
-                                    bar_q_full, ch * 64, (int)t.h,
+                                    bar_q_full, ch * T::CE, (int)t.h,
                                     (int)(t.qrow + t.q0 + tt * 128), t.bmap);
                 ++q_cnt;
             };
@@ -440,7 +471,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 const uint32_t dst = k_slots + slot * T::K_TILE_BYTES;
                 mbar_arrive_expect_tx(bar_kfull(slot), T::K_TILE_BYTES);
                 for (int ch = 0; ch < T::QCH; ++ch)
-                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_k, bar_kfull(slot), ch * 64,
+                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_k, bar_kfull(slot), ch * T::CE,
                                 (int)t.g, (int)(t.krow + (int64_t)j * BN), t.bmap);
                 ++kq;
             };
@@ -454,7 +485,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 const uint32_t dst = v_slots + slot * T::V_TILE_BYTES;
                 mbar_arrive_expect_tx(bar_vfull(slot), T::V_TILE_BYTES);
                 for (int ch = 0; ch < T::VCH; ++ch)
-                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_v, bar_vfull(slot), ch * 64,
+                    tma_load_4d(dst + ch * T::CHUNK_BYTES, &tmap_v, bar_vfull(slot), ch * T::CE,
                                 (int)t.g, (int)(t.krow + (int64_t)j * BN), t.bmap);
                 ++vq;
             };
@@ -615,7 +646,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         const int w4 = warp & 3;                  // TMEM lanes 32*w4 .. 32*w4+31
         const int row = threadIdx.x & 127;        // TMEM lane = row of the query tile
         const uint32_t tl = tmem + ((uint32_t)(w4 * 32) << 16);
-        const float sl2 = p.scale_log2;
+        float sl2 = p.scale_log2;  // per unit with E4M3 inputs (times the Q and K descales)
         auto tile_of = [&](int k) { return T::NSM == 1 ? k : wg; };
         bool ok = true;
         int64_t jg = 0;  // key blocks stepped through so far (all units); item g = jg * NT + tile
@@ -656,7 +687,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             tc_fence_after_sync();
             const int64_t i = t.q0 + tt * 128 + row;
             const bool row_valid = i < t.sq;
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            // E4M3 inputs: the V descale joins the final division
+            const float vds = T::FP8 ? __ldg(p.v_descale + t.bi * p.hk + t.g) : 1.f;
+            const float inv_l = l > 0.f ? vds / l : 0.f;
             if constexpr (OTMA) {
                 // This warp's 32 rows go to its own slab of the staging tile (one 32-row, 128-byte
                 // swizzled box per 64 columns), then one lane stores the slab with TMA; rows past
@@ -761,6 +794,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             }
             const int64_t rn = busy_from(r + 1);
             const int64_t un = rn >= 0 ? unit_of(rn) : -1;
+            if constexpr (T::FP8) {
+                // S holds sums of code products; the descales fold into the exp2 factor, kept at
+                // 2^-100 or more as on the host (a NaN product also becomes 2^-100)
+                const float f = p.scale_log2 * __ldg(p.q_descale + t.bi * p.hq + t.h) *
+                                __ldg(p.k_descale + t.bi * p.hk + t.g);
+                sl2 = f > 0x1p-100f ? f : 0x1p-100f;
+            }
             int64_t lim[NTW];  // last allowed key of this thread's row in each tile
             int64_t lol[NTW];  // first allowed key (the window's lower bound), may be negative
             float m_ref[NTW];  // exponent reference (log2 units); moves lazily
@@ -905,11 +945,19 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                                     p1 = ex2(x1);
                                 }
                                 add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
-                                pk[c] = pack_bf16x2(p0, p1);
+                                if constexpr (T::FP8) {  // four E4M3 weights per column
+                                    const uint32_t h2 = pack_e4m3x2(p0, p1);
+                                    if (c & 1) pk[c >> 1] |= h2 << 16;
+                                    else pk[c >> 1] = h2;
+                                } else {
+                                    pk[c] = pack_bf16x2(p0, p1);
+                                }
                             }
                         }
-                        // P chunk ch (16 columns of bf16 pairs) overwrites S columns already read
-                        tmem_st16(s_col + ch * 16, pk);
+                        // P chunk ch (16 columns of bf16 pairs, or 8 of E4M3 quads) overwrites S
+                        // columns already read
+                        if constexpr (T::FP8) tmem_st8(s_col + ch * 8, pk);
+                        else tmem_st16(s_col + ch * 16, pk);
                     }
                     l[k] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
                     tmem_wait_st();

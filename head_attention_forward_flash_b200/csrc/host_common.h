@@ -51,4 +51,33 @@ inline int check_arch()
     return ok ? B200ATTN_OK : B200ATTN_ERR_ARCH;
 }
 
+// Stream-ordered pool for the pre-passes' partial results (k_smooth_mean, k_smooth_gate,
+// fp8_quantize), one per device. Its release threshold is
+// "never", so memory freed at the end of a call stays in the pool for the next call instead of
+// being returned to the driver (and mapped again) around every synchronisation.
+inline cudaMemPool_t scratch_pool()
+{
+    static cudaMemPool_t pools[64] = {nullptr};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (pools[dev] == nullptr) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        uint64_t keep = UINT64_MAX;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        pools[dev] = pool;
+    }
+    return pools[dev];
+}
+
 }  // namespace b200

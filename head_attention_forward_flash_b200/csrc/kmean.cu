@@ -233,34 +233,6 @@ __global__ void __launch_bounds__(kThreads)
 constexpr int64_t kNoAllocScratchFloats = (int64_t)1 << 20;
 __device__ __align__(256) float g_kmean_scratch[kNoAllocScratchFloats];
 
-// Stream-ordered pool for k_smooth_mean's partial sums, one per device. Its release threshold is
-// "never", so memory freed at the end of a call stays in the pool for the next call instead of
-// being returned to the driver (and mapped again) around every synchronisation.
-cudaMemPool_t scratch_pool()
-{
-    static cudaMemPool_t pools[64] = {nullptr};
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-        cudaGetLastError();
-        return nullptr;
-    }
-    if (pools[dev] == nullptr) {
-        cudaMemPoolProps props = {};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = dev;
-        cudaMemPool_t pool = nullptr;
-        if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        uint64_t keep = UINT64_MAX;
-        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-        pools[dev] = pool;
-    }
-    return pools[dev];
-}
-
 int check_kmean_args(const void* k, const void* mean, int64_t b, int64_t hk, int64_t sk,
                      int64_t d, int64_t* cols_out)
 {

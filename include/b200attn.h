@@ -224,6 +224,58 @@ B200ATTN_API int k_smooth_gate(const void* k, float* mean, int32_t* gate, float*
 B200ATTN_API int k_smooth_sub(const void* k, const float* mean, void* k_out, int64_t b, int64_t hk,
                  int64_t sk, int64_t d, void* stream);
 
+/*
+ * fp8_quantize -- E4M3 codes of a bf16 BSHD tensor with one fp32 scale per (batch, head), for the
+ * FP8 attention recipe ("[HIP] Mha v4: run the K-smoothing gate as one HIP call", Summary: the
+ * quantized recipes apply the K-smoothing gate before quantizing K; "Tune MHA config &
+ * small-head pipeline pathology", the FP8 rows after Final status). The pages give neither the
+ * quantisation nor the scale layout. Reading (per-head amax scaling, OCP E4M3):
+ *     x'      = mean ? fp32(x - mean[bi,hh,c]) : x          (one fp32 subtraction, RNE)
+ *     amax    = max |x'| over the head's [s, d] slice
+ *     descale[bi,hh] = amax > 0 ? fp32(amax / 448) : 1
+ *     code    = E4M3_satfinite_rne(fp32(x' * f)),  f = amax > 0 ? min(fp32(448 / amax), FLT_MAX) : 1
+ * E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits, subnormals, no infinities, largest
+ * finite 448; ties round to the even code; magnitudes past 448 saturate. The codes are exact
+ * (bit-identical to any correct implementation of these steps) and deterministic.
+ *
+ *   x         device bf16 [b, s, h, d], 16-byte aligned, finite. Read only.
+ *   mean      device fp32 [b, h, d], 16-byte aligned (K smoothing: the output of k_smooth_mean or
+ *             k_smooth_gate), or NULL.
+ *   x8        device uint8 [b, s, h, d], 16-byte aligned. Fully written. Must not overlap x.
+ *   descale   device fp32 [b, h], 4-byte aligned. Fully written.
+ *   b, h      >= 0 (0: nothing to do);  s >= 0 (0: every descale is 1);  d in {64, 128, 256}.
+ * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`.
+ * Two kernels (per-chunk amax, then fold and convert). Safe on concurrent streams.
+ */
+B200ATTN_API int fp8_quantize(const void* x, const float* mean, void* x8, float* descale,
+                              int64_t b, int64_t s, int64_t h, int64_t d, void* stream);
+
+/*
+ * attn_fwd_fp8 -- attn_fwd on E4M3 inputs with per-(batch, head) descales (the FP8 recipe; see
+ * fp8_quantize for the format and the scale reading).
+ *
+ * Computes attn_fwd's O and LSE for the decoded inputs
+ *     Q = code * q_descale[bi,h],  K = code * k_descale[bi,g],  V = code * v_descale[bi,g].
+ * Q K^T and P V run as E4M3 tensor-core products with fp32 accumulation. The descales of Q and
+ * K fold into the exp2 factor, and that of V into the final division. The softmax weights P
+ * are rounded to E4M3 for the P V product; the row sums keep the unrounded weights. Per output
+ * element this moves O by at most (2^-4 sum_j w_j |V_jc| + 2^-10 sum_j |V_jc|) / sum_j w_j
+ * (w_j = exp(s_j - max s)) beyond attn_fwd's own rounding. LSE is as in attn_fwd.
+ *
+ *   q8       device uint8 [b, sq, hq, dqk];  k8: [b, sk, hk, dqk];  v8: [b, sk, hk, dv];
+ *            16-byte aligned, E4M3 codes (no NaN codes). Read only.
+ *   q_descale  device fp32 [b, hq];  k_descale, v_descale: [b, hk]; 4-byte aligned, positive
+ *            and finite (the product scale * q_descale * k_descale is kept at 2^-100 or more).
+ *   out, lse as in attn_fwd (O in bf16).
+ *   dqk, dv  (128, 128) only (else B200ATTN_ERR_HEADDIM).
+ *   other arguments, errors, allocation and concurrency as in attn_fwd.
+ */
+B200ATTN_API int attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                              const float* q_descale, const float* k_descale,
+                              const float* v_descale, void* out, float* lse, int64_t b,
+                              int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk,
+                              int64_t dv, int causal, float scale, void* stream);
+
 /* Static description of a status code (never NULL). */
 B200ATTN_API const char* attn_status_string(int status);
 

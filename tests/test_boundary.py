@@ -143,3 +143,41 @@ def test_k_smooth_gate_rejects():
 
 def test_debug_starve_range():
     assert b2.lib.attn_debug_starve(0) == 6 and b2.lib.attn_debug_starve(2_000_000) == 6
+
+
+def call_fp8(q=A, k=A, v=A, dq=A, dk=A, dv_=A, o=A, lse=A, b=1, hq=2, hk=1, sq=16, sk=16,
+             dqk=128, dv=128, causal=1, scale=0.125):
+    return b2.lib.attn_fwd_fp8(q, k, v, dq, dk, dv_, o, lse, b, hq, hk, sq, sk, dqk, dv, causal,
+                               scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(b=-1), 2), (dict(sk=-1), 2), (dict(hk=0), 2), (dict(hq=3, hk=2), 3),
+    (dict(dqk=64, dv=64), 4), (dict(dqk=192, dv=128), 4), (dict(dqk=256, dv=256), 4),
+    (dict(scale=float("nan")), 7),
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(o=None), 1),
+    (dict(dq=None), 1), (dict(dk=None), 1), (dict(dv_=None), 1),
+    (dict(q=A + 8), 5), (dict(k=A + 1), 5), (dict(o=A + 2), 5), (dict(dq=A + 2), 5),
+    (dict(dv_=A + 1), 5), (dict(lse=A + 3), 5),
+    (dict(sq=1 << 31), 6), (dict(b=1 << 40, hq=1 << 40, hk=1), 6),
+])
+def test_attn_fwd_fp8_rejects(kw, code):
+    assert call_fp8(**kw) == code
+
+
+def test_fp8_empty_problem_is_a_no_op():
+    assert call_fp8(b=0, q=None, k=None, v=None, dq=None, dk=None, dv_=None, o=None, lse=None) == 0
+    assert call_fp8(sq=0, q=None, o=None, lse=None) == 0
+
+
+def test_fp8_quantize_rejects():
+    f = b2.lib.fp8_quantize
+
+    def c(x=A, m=A, x8=A, ds=A, b=1, s=8, h=2, d=128):
+        return f(x, m, x8, ds, b, s, h, d, None)
+
+    assert c(d=96) == 4 and c(d=32) == 4 and c(b=-1) == 2 and c(s=-1) == 2 and c(h=-1) == 2
+    assert c(x=None) == 1 and c(x8=None) == 1 and c(ds=None) == 1
+    assert c(x=A + 8) == 5 and c(x8=A + 4) == 5 and c(m=A + 4) == 5 and c(ds=A + 2) == 5
+    assert c(b=1 << 40, s=1 << 30) == 6
+    assert c(b=0) == 0 and c(h=0) == 0

@@ -17,7 +17,7 @@ import math
 
 import torch
 
-# The five workloads (sizes as the pages' benchmarks and the quantised-attention table give them).
+# The workloads (sizes as the pages' benchmarks and the quantised-attention table give them).
 CONFIGS = {
     1: dict(workload="mha_b1_h2_s128_d64", b=1, hq=2, hk=2, sq=128, sk=128, dqk=64, dv=64,
             causal=False, kmean=False),
@@ -39,6 +39,11 @@ CONFIGS = {
     # 1.5 * N(0,1) with seed 4000 + id.
     7: dict(workload="swa_sink_b1_hq64_hk8_s8192_d64_causal_w128", b=1, hq=64, hk=8, sq=8192,
             sk=8192, dqk=64, dv=64, causal=True, kmean=False, window=128, sinks=True),
+    # The FP8 recipe on the pages' long FP8 shape (hd128, b1 h5 s65536; causal as the bf16 one):
+    # the same N(0,1) draws, quantised to E4M3 with one scale per (batch, head) after the
+    # K-smoothing gate.
+    8: dict(workload="fp8_long_b1_h5_s65536_d128_causal", b=1, hq=5, hk=5, sq=65536, sk=65536,
+            dqk=128, dv=128, causal=True, kmean=False, fp8=True),
 }
 
 HEAD_DIMS = ((64, 64), (128, 128), (192, 128), (256, 256))
