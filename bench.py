@@ -3,7 +3,8 @@
 python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl reference]
 
 One step = one pass of the hot path over one batch of synthetic input: attn_fwd (plus, for the
-K-mean workload, k_smooth_mean and k_smooth_sub before it). Inputs are seeded N(0,1) bf16 tensors
+K-mean workload, k_smooth_mean and k_smooth_sub before it; for the FP8 workload, the K-smoothing
+gate, fp8_quantize of Q, K (smoothed) and V, then attn_fwd_fp8). Inputs are seeded N(0,1) bf16 tensors
 of the workload's shape, resident in HBM before timing starts. Each step is timed with CUDA
 events on the launching stream; the L2 cache is flushed (a 256 MiB write) before every step,
 outside the events. Under torchrun every rank runs its own independent batch (weak scaling, no
@@ -36,6 +37,8 @@ import workloads  # noqa: E402
 DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PROFILED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+GATE_THRESHOLD = 0.25  # K-smoothing gate threshold of the FP8 recipe and the gate timing
+FP8_OVER_BF16 = 2.0    # nominal dense E4M3 / BF16 tensor throughput on B200 (4.5 / 2.25 PFLOP/s)
 
 
 def measured_peaks():
@@ -84,6 +87,20 @@ class OracleSampler:
         self.oracle = oracle
         self.c = c
         q, k, v = inputs if inputs is not None else workloads.config_inputs(c)
+        self.fp8 = bool(c.get("fp8"))
+        if self.fp8:
+            # the FP8 recipe's inputs, made by the oracle once (gate, smoothing, quantisation)
+            # and decoded once; the timed part is the attention on them
+            from oracle import fp8 as ofp8
+            self.ofp8 = ofp8
+            b, hq, hk, sq, sk, d = c["b"], c["hq"], c["hk"], c["sq"], c["sk"], c["dqk"]
+            _, m32, _, _ = oracle.k_gate(workloads.bf16_bits(k), b, hk, sk, d, GATE_THRESHOLD)
+            q8, dq = ofp8.quantize(workloads.bf16_bits(q), b, sq, hq, d)
+            k8, dk = ofp8.quantize(workloads.bf16_bits(k), b, sk, hk, d, mean32=m32)
+            v8, dv = ofp8.quantize(workloads.bf16_bits(v), b, sk, hk, c["dv"])
+            self.qf = ofp8.dequantize(q8, dq, b, sq, hq, d)
+            self.kf = ofp8.dequantize(k8, dk, b, sk, hk, d)
+            self.vf = ofp8.dequantize(v8, dv, b, sk, hk, c["dv"])
         if c["kmean"]:
             _, m32 = oracle.k_mean(workloads.bf16_bits(k), c["b"], c["hk"], c["sk"], c["dqk"])
             self.kb = oracle.k_sub(workloads.bf16_bits(k), m32, c["b"], c["hk"], c["sk"], c["dqk"])
@@ -105,6 +122,11 @@ class OracleSampler:
         rows = self.rows[idx]
         c = self.c
         t0 = time.perf_counter()
+        if self.fp8:
+            self.ofp8.attn_rows_decoded(self.qf, self.kf, self.vf, c["b"], c["hq"], c["hk"],
+                                        c["sq"], c["sk"], c["dqk"], c["dv"], c["causal"],
+                                        c["scale"], rows, nthreads=self.threads)
+            return time.perf_counter() - t0, _row_flops(c, rows), len(rows)
         sk_logits = workloads.sinks(c)
         self.oracle.attn_rows(self.qb, self.kb, self.vb, c["b"], c["hq"], c["hk"], c["sq"],
                               c["sk"], c["dqk"], c["dv"], c["causal"], c["scale"], rows,
@@ -138,7 +160,8 @@ def cpu_baseline(c, inputs, seconds):
     dt, fl, nr = s.run(n)
     return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": s.threads, "kind": "oracle",
             "sample": f"{nr} seeded output rows (all heads/batches, {c['workload']}), "
-                      f"{fl / 1e9:.2f} GFLOP in {dt:.1f} s, fp64 plain C oracle"}
+                      f"{fl / 1e9:.2f} GFLOP in {dt:.1f} s, fp64 plain C oracle"
+                      + (" on the oracle's decoded E4M3 recipe inputs" if s.fp8 else "")}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -284,15 +307,34 @@ def run_gpu(args):
     mean = torch.empty((c["b"], c["hk"], c["dqk"]), dtype=torch.float32, device=dev)
     k_s = torch.empty_like(k) if c["kmean"] else None
     windowed = c.get("window") is not None or bool(c.get("sinks"))
+    fp8 = bool(c.get("fp8"))
+    if fp8:  # the recipe's E4M3 buffers and per-(batch, head) descales
+        q8 = torch.empty(q.shape, dtype=torch.uint8, device=dev)
+        k8 = torch.empty(k.shape, dtype=torch.uint8, device=dev)
+        v8 = torch.empty(v.shape, dtype=torch.uint8, device=dev)
+        dq = torch.empty((c["b"], c["hq"]), dtype=torch.float32, device=dev)
+        dk = torch.empty((c["b"], c["hk"]), dtype=torch.float32, device=dev)
+        dv = torch.empty((c["b"], c["hk"]), dtype=torch.float32, device=dev)
+        gate = torch.empty((c["b"], c["hk"]), dtype=torch.int32, device=dev)
     sk_h = workloads.sinks(c)
     sinks_d = sk_h.to(dev) if sk_h is not None else None
     window = c["window"] if c.get("window") is not None else -1
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 4 if c["kmean"] else 1
+    launches_per_step = 4 if c["kmean"] else (9 if fp8 else 1)
 
     def step():
         kk = k
+        if fp8:
+            b2.k_smooth_gate(k, GATE_THRESHOLD, mean=mean, gate=gate, return_ratio=False)
+            b2.fp8_quantize(q, out=q8, descale=dq)
+            b2.fp8_quantize(k, mean=mean, out=k8, descale=dk)
+            b2.fp8_quantize(v, out=v8, descale=dv)
+            ev_a0.record(stream)
+            b2.attn_fwd_fp8(q8, k8, v8, dq, dk, dv, causal=c["causal"], scale=c["scale"], out=o,
+                            lse=lse)
+            ev_a1.record(stream)
+            return
         if c["kmean"]:
             b2.k_smooth_mean(k, mean)
             b2.k_smooth_sub(k, mean, k_s)
@@ -352,6 +394,11 @@ def run_gpu(args):
     achieved = fl / (attn_avg_ms * 1e-3) / 1e12
     peaks, peak_src = measured_peaks()
     peak = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    peak_note = f"{peak_src} cuBLAS bf16 burst (kernel timed alone)"
+    if fp8:  # a contraction takes its own dtype's peak
+        peak *= FP8_OVER_BF16
+        peak_note = (f"{peak_src} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal E4M3 / BF16 "
+                     f"dense ratio; kernel timed alone)")
     traffic = None
     try:
         with open(PROFILED_TRAFFIC_FILE) as f:
@@ -365,15 +412,15 @@ def run_gpu(args):
 
     # the K-smoothing gate on the same K (K-mean workload): its own event-timed calls
     kgate = None
-    if c["kmean"]:
+    if c["kmean"] or fp8:
         ge0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
         ge1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
         for _ in range(3):
-            b2.k_smooth_gate(k, 0.25)
+            b2.k_smooth_gate(k, GATE_THRESHOLD)
         for s_ in range(10):
             flush.zero_()
             ge0[s_].record(stream)
-            b2.k_smooth_gate(k, 0.25)
+            b2.k_smooth_gate(k, GATE_THRESHOLD)
             ge1[s_].record(stream)
         torch.cuda.synchronize()
         g_us = 1e3 * statistics.median(ge0[s_].elapsed_time(ge1[s_]) for s_ in range(10))
@@ -381,7 +428,7 @@ def run_gpu(args):
         n_samp = (c["sk"] + stride - 1) // stride
         g_bytes = c["b"] * n_samp * c["hk"] * c["dqk"] * 2
         kgate = {"us_median": g_us, "sampled_bytes": g_bytes,
-                 "gbs": g_bytes / (g_us * 1e-6) / 1e9, "threshold": 0.25,
+                 "gbs": g_bytes / (g_us * 1e-6) / 1e9, "threshold": GATE_THRESHOLD,
                  "launches": 2, "note": "k_smooth_gate alone, L2 flushed before each call"}
 
     # end to end through the public API with host buffers (pinned), copies inside the timing
@@ -402,6 +449,16 @@ def run_gpu(args):
             qd = qp.to(dev, non_blocking=True)
             kd = kp.to(dev, non_blocking=True)
             vd = vp.to(dev, non_blocking=True)
+            if fp8:
+                m_, _, _ = b2.k_smooth_gate(kd, GATE_THRESHOLD, return_ratio=False)
+                q8d, dqd = b2.fp8_quantize(qd)
+                k8d, dkd = b2.fp8_quantize(kd, mean=m_)
+                v8d, dvd = b2.fp8_quantize(vd)
+                od, ld = b2.attn_fwd_fp8(q8d, k8d, v8d, dqd, dkd, dvd, causal=c["causal"],
+                                         scale=c["scale"])
+                op.copy_(od, non_blocking=True)
+                lp.copy_(ld, non_blocking=True)
+                return
             if c["kmean"]:
                 kd = b2.k_smooth_sub(kd, b2.k_smooth_mean(kd))
             if varlen:
@@ -451,7 +508,8 @@ def run_gpu(args):
         "metric": "attention fwd TFLOP/s (causal-halved) and % of B200 dense BF16 peak",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "vs_baseline": None, "dtype": "e4m3 (fp32 accumulate)" if fp8 else "bf16",
+        "data": "synthetic (seeded N(0,1) bf16)" + (", quantised on the GPU each step" if fp8 else ""),
         "pct_of_dense_bf16_peak": {"value": 100.0 * value / world / DATASHEET_BF16_TFLOPS,
                                    "peak_tflops": DATASHEET_BF16_TFLOPS,
                                    "peak_source": "B200 datasheet dense BF16"},
@@ -470,11 +528,16 @@ def run_gpu(args):
                           if varlen else {}),
                        **({"window_left": window, "sinks": bool(c.get("sinks")),
                            "flops": "2*b*hq*(dqk+dv)*allowed (query, key) pairs"}
-                          if windowed else {})),
+                          if windowed else {}),
+                       **({"recipe": "k_smooth_gate (threshold "
+                                     f"{GATE_THRESHOLD:g}) + fp8_quantize Q, K - mean, V + "
+                                     "attn_fwd_fp8, all inside the step",
+                           "scales": "one fp32 descale per (batch, head) per tensor"}
+                          if fp8 else {})),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": f"attn_fwd_kernel d{c['dqk']}x{c['dv']}",
-                     "peak_source": f"{peak_src} cuBLAS bf16 burst (kernel timed alone)"},
+                     "kernel": f"attn_fwd_kernel d{c['dqk']}x{c['dv']}" + (" e4m3" if fp8 else ""),
+                     "peak_source": peak_note},
         "dispatch_us": {"median": 1e3 * statistics.median(attn_ms),
                         "trimmed_mean_80": 1e3 * sum(srt[lo:hi]) / max(1, hi - lo),
                         "max": 1e3 * max(attn_ms), "min": 1e3 * min(attn_ms)},
@@ -514,7 +577,8 @@ def run_reference(args):
     value = sum(fls) / sum(times) / 1e12
     ms = 1e3 * sum(times) / len(times)
     sample = (f"{n} seeded output rows per step of {c['workload']} (all heads/batches), "
-              f"fp64 plain C oracle")
+              f"fp64 plain C oracle"
+              + (" on the oracle's decoded E4M3 recipe inputs" if s.fp8 else ""))
     line = {
         "impl": "reference",
         "metric": "attention fwd TFLOP/s (causal-halved) and % of B200 dense BF16 peak",

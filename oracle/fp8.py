@@ -135,10 +135,18 @@ def attn_rows(q8, k8, v8, q_descale, k_descale, v_descale, b, hq, hk, sq, sk, dq
               scale, rows, nthreads=None, lib=None):
     """O (fp64 [nrows, dv]) and LSE (fp64 [nrows]) for the (batch, head, query) triples in
     rows, on the decoded, descaled E4M3 inputs."""
-    lib = lib or load_library()
     q = _f64(dequantize(q8, q_descale, b, sq, hq, dqk))
     k = _f64(dequantize(k8, k_descale, b, sk, hk, dqk))
     v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))
+    return attn_rows_decoded(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, rows,
+                             nthreads=nthreads, lib=lib)
+
+
+def attn_rows_decoded(q, k, v, b, hq, hk, sq, sk, dqk, dv, causal, scale, rows, nthreads=None,
+                      lib=None):
+    """attn_rows on inputs already decoded by dequantize (fp64 BSHD arrays)."""
+    lib = lib or load_library()
+    q, k, v = _f64(q), _f64(k), _f64(v)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     n = rows.shape[0]
     o = np.zeros((n, dv), dtype=np.float64)
