@@ -30,8 +30,8 @@ MUTANTS = {
     "mean_added": ("x = np.subtract(x, m, dtype=np.float32)", "x = np.add(x, m, dtype=np.float32)"),
     "v_descale_dropped": ("v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))\n    o = np.zeros((b, sq",
                           "v = _f64(dequantize(v8, np.ones_like(v_descale), b, sk, hk, dv))\n    o = np.zeros((b, sq"),
-    "k_descale_from_q": ("k = _f64(dequantize(k8, k_descale, b, sk, hk, dqk))\n    v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))\n    rows",
-                         "k = _f64(dequantize(k8, q_descale[:, :hk], b, sk, hk, dqk))\n    v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))\n    rows"),
+    "k_descale_from_q": ("k = _f64(dequantize(k8, k_descale, b, sk, hk, dqk))\n    v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))\n    return attn_rows_decoded",
+                         "k = _f64(dequantize(k8, q_descale[:, :hk], b, sk, hk, dqk))\n    v = _f64(dequantize(v8, v_descale, b, sk, hk, dv))\n    return attn_rows_decoded"),
 }
 
 
