@@ -149,3 +149,14 @@ def test_recipe_on_gpu_against_bf16(b2):
     err_gpu = float(np.max(np.abs(og.float().cpu().double().numpy() - o_bf)))
     err_or = float(np.max(np.abs(o_or - o_bf)))
     assert err_gpu <= err_or + 2e-2, (err_gpu, err_or)
+
+
+def test_attention_no_keys(b2):
+    # sk = 0: every row is empty (O = 0, LSE = -inf); K and V have no rows
+    q8 = torch.zeros((1, 40, 2, 128), dtype=torch.uint8, device="cuda")
+    k8 = torch.empty((1, 0, 1, 128), dtype=torch.uint8, device="cuda")
+    dq = torch.ones((1, 2), dtype=torch.float32, device="cuda")
+    dk = torch.ones((1, 1), dtype=torch.float32, device="cuda")
+    o, lse = b2.attn_fwd_fp8(q8, k8, k8, dq, dk, dk, causal=False)
+    torch.cuda.synchronize()
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
