@@ -38,10 +38,13 @@
 //
 // Template flags: CAUSAL; VARLEN (packed sequences: per-unit offsets from cu_seqlens); EXT
 // (sliding window and sinks: a first key block per unit, a lower per-key bound, and each row's
-// reference and sum started at the head's sink logit).
+// reference and sum started at the head's sink logit). Traits flag FP8: E4M3 Q, K, V with
+// kind::f8f6f4 MMAs (K = 32 per instruction, the same 32 bytes of a row as bf16's K = 16), P
+// rounded to E4M3 four per TMEM column, and per-(batch, head) descales folded into the exp2
+// factor (Q, K) and the final division (V).
 //
 // Tensor memory (128 lanes x 512 columns of 32 bit): S0 | S1 (BN columns each; P in bf16 pairs
-// overwrites the first BN/2 columns of its own S buffer) | O for each query tile (DV fp32
+// overwrites the first BN/2 columns of its own S buffer, E4M3 quads the first BN/4) | O for each query tile (DV fp32
 // columns each) | Q for each query tile when it lives in TMEM (DQK/2 columns of bf16 pairs).
 //
 // Every mbarrier wait is bounded in time; a wait that gives up sets the device error word and a

@@ -1,4 +1,5 @@
-"""Writes tests/golden/mha_b1_h2_s128_d64_rows.json from the CPU oracle alone.
+"""Writes tests/golden/mha_b1_h2_s128_d64_rows.json and tests/golden/fp8_b1_h2_s128_d128.json
+from the CPU oracle alone.
 
 The workload is the smallest benchmark shape (b=1, hq=hk=2, sq=sk=128, dqk=dv=64,
 non-causal, scale 1/sqrt(64), inputs iid N(0,1) cast to bf16 from seed 1001), the
@@ -38,5 +39,47 @@ def main():
         json.dump(out, f, indent=1)
 
 
+FP8_SEED = 1801
+FP8_ROWS = [(0, 0, 0), (0, 1, 5), (0, 0, 64), (0, 1, 127)]
+FP8_CHANNELS = [0, 7, 64, 127]
+
+
+def main_fp8():
+    """The FP8 recipe on a small causal shape (b=1, hq=hk=2, sq=sk=128, d=128, seed 1801, the
+    K-mean recipe's K with per-channel offsets, smoothed by the oracle's own mean): descales,
+    a digest and a sample of the E4M3 codes, and sampled O / LSE values of the attention on them.
+    The format (E4M3) and the recipe (smoothing before K is quantised) follow "[HIP] Mha v4: run
+    the K-smoothing gate as one HIP call" (Summary, Performance); the scale layout is this
+    build's reading. The pages print no values."""
+    import hashlib
+    from oracle import fp8
+    from workloads import make_inputs
+
+    b, h, s, d = 1, 2, 128, 128
+    q, k, v = make_inputs(b, h, h, s, s, d, d, seed=FP8_SEED, kmean=True)
+    m32 = oracle.k_mean(bf16_bits(k), b, h, s, d)[1]
+    q8, dq = fp8.quantize(bf16_bits(q), b, s, h, d)
+    k8, dk = fp8.quantize(bf16_bits(k), b, s, h, d, mean32=m32)
+    v8, dv = fp8.quantize(bf16_bits(v), b, s, h, d)
+    scale = 1.0 / d ** 0.5
+    o, lse = fp8.attn_rows(q8, k8, v8, dq, dk, dv, b, h, h, s, s, d, d, True, scale, FP8_ROWS,
+                           nthreads=1)
+    out = {
+        "shape": [b, h, s, d], "seed": FP8_SEED, "causal": True, "scale": scale,
+        "source": "CPU oracle (oracle/fp8.py on oracle/attn_oracle.c), written by "
+                  "tests/golden/make_golden.py",
+        "descale": {"q": dq.ravel().tolist(), "k": dk.ravel().tolist(), "v": dv.ravel().tolist()},
+        "codes_sha256": {n: hashlib.sha256(a.tobytes()).hexdigest()
+                         for n, a in (("q", q8), ("k", k8), ("v", v8))},
+        "k_codes_row0_head0": k8[0, 0, 0, :16].tolist(),
+        "rows": [list(r) for r in FP8_ROWS], "channels": FP8_CHANNELS,
+        "o": [[float(o[n, ch]) for ch in FP8_CHANNELS] for n in range(len(FP8_ROWS))],
+        "lse": [float(x) for x in lse],
+    }
+    with open(os.path.join(HERE, "fp8_b1_h2_s128_d128.json"), "w") as f:
+        json.dump(out, f, indent=1)
+
+
 if __name__ == "__main__":
     main()
+    main_fp8()
