@@ -39,14 +39,16 @@ __device__ __forceinline__ void load_group(const uint4* src, const float* m, flo
     }
 }
 
-// Thread layout shared by both passes: group gi = t % G of the row, row offset t / G, with
-// G = d / 8 groups per row and R = 256 / G rows per step.
+// Problem geometry of both passes. Grid: x = (batch, head) slice bh = bi * h + hh, y = row
+// chunk. Thread t of a CTA takes 16-byte group gi = t % G of a row and rows t / G, t / G + R,
+// ... of its chunk, with G = d / 8 groups per row and R = 256 / G rows per step.
 struct QGeom {
     int64_t s, h, d8;  // rows, heads, 16-byte groups per row
     int64_t rows_per_chunk;
-    int nch;
+    int nch;           // row chunks per head slice
 };
 
+// The 8 mean values of group gi of head slice bh (mean is [b, h, d] fp32).
 __device__ __forceinline__ void head_mean(const float* mean, int64_t bh, int64_t d8, int gi,
                                           float (&mv)[8])
 {
@@ -56,6 +58,7 @@ __device__ __forceinline__ void head_mean(const float* mean, int64_t bh, int64_t
     mv[4] = c.x; mv[5] = c.y; mv[6] = c.z; mv[7] = c.w;
 }
 
+// Max over the CTA's 256 threads (non-negative inputs); the result is valid in warp 0.
 __device__ __forceinline__ float block_max(float v, float* red)
 {
 #pragma unroll
