@@ -7,7 +7,9 @@
  *   - Tensors are contiguous, BSHD, row-major (last dimension fastest):
  *       Q [b, sq, hq, dqk], K [b, sk, hk, dqk], V [b, sk, hk, dv], O [b, sq, hq, dv]  (bf16)
  *       LSE [b, hq, sq] (fp32, natural log), K mean [b, hk, d] (fp32);
- *     attn_fwd_varlen packs sequences along the row axis instead ([total, h, d], LSE [hq, total]).
+ *     attn_fwd_varlen packs sequences along the row axis instead ([total, h, d], LSE [hq, total]);
+ *     the FP8 recipe takes the same BSHD shapes as E4M3 codes (uint8) with fp32 descales
+ *     [b, h] (fp8_quantize, attn_fwd_fp8).
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Work is
  *     enqueued asynchronously on it; the call does not synchronise.
  *   - Return value: B200ATTN_OK (0) on success, otherwise one of the status codes below.
@@ -41,10 +43,12 @@ enum b200attn_status {
     B200ATTN_ERR_NULL = 1,     /* a required pointer is NULL for a non-empty tensor */
     B200ATTN_ERR_SHAPE = 2,    /* a size is negative, or hk <= 0 / sk < 0 */
     B200ATTN_ERR_GQA = 3,      /* hq is not a multiple of hk */
-    B200ATTN_ERR_HEADDIM = 4,  /* (dqk, dv) not in {(64,64),(128,128),(192,128),(256,256)};
-                                  for the K mean, d not in {64, 128, 256} */
+    B200ATTN_ERR_HEADDIM = 4,  /* (dqk, dv) not in {(64,64),(128,128),(192,128),(256,256)}
+                                  ((128,128) only for attn_fwd_fp8); for the K mean and
+                                  fp8_quantize, d not in {64, 128, 256} */
     B200ATTN_ERR_ALIGN = 5,    /* a pointer below its required alignment: 16 bytes for bf16
-                                  tensors and the K mean, 4 bytes for LSE */
+                                  and E4M3 tensors and the K mean, 4 bytes for LSE, sinks
+                                  and descales */
     B200ATTN_ERR_RANGE = 6,    /* a size, byte extent or stride overflows int64 or TMA limits */
     B200ATTN_ERR_SCALE = 7,    /* scale is NaN or infinite */
     B200ATTN_ERR_ARCH = 8,     /* the current device is not compute capability 10.0 (sm_100) */
