@@ -382,6 +382,8 @@ def run_gpu(args):
         clk["sm_max_mhz"] = clk["sm_mhz"]
     step_ms = [starts[s].elapsed_time(ends[s]) for s in range(args.steps)]
     attn_ms = [a_starts[s].elapsed_time(a_ends[s]) for s in range(args.steps)]
+    # the pre-pass (K mean + K subtract, or gate + quantisation): step start -> attention start
+    pre_ms = [starts[s].elapsed_time(a_starts[s]) for s in range(args.steps)]
     status = b2.attn_debug_status()
     if status != 0:
         raise RuntimeError(f"a kernel reported status {status} in the timed region")
@@ -548,6 +550,28 @@ def run_gpu(args):
     }
     if kgate is not None:
         line["k_smooth_gate"] = kgate
+    if c["kmean"] or fp8:
+        # bytes the pre-pass kernels move by design. K mean: read K; subtract: read K, write K'.
+        # FP8: the gate's sampled rows, then per tensor two reads (amax, convert) of bf16 and
+        # one write of E4M3 codes.
+        n_q = c["b"] * c["sq"] * c["hq"] * c["dqk"]
+        n_k = c["b"] * c["sk"] * c["hk"] * c["dqk"]
+        n_v = c["b"] * c["sk"] * c["hk"] * c["dv"]
+        if fp8:
+            stride = (c["sk"] + 2047) // 2048
+            sampled = c["b"] * ((c["sk"] + stride - 1) // stride) * c["hk"] * c["dqk"] * 2
+            pre_bytes = sampled + 5 * (n_q + n_k + n_v)
+            kernels = "k_gate_partial, k_gate_fold, 3 x (fp8_amax_partial, fp8_convert)"
+        else:
+            pre_bytes = 3 * n_k * 2
+            kernels = "k_mean_partial, k_mean_fold, k_sub_kernel"
+        pre_us = 1e3 * statistics.median(pre_ms)
+        gbs = pre_bytes / (pre_us * 1e-6) / 1e9
+        hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+        line["prepass"] = {"us_median": pre_us, "bytes": pre_bytes, "gbs": gbs,
+                           "frac_of_measured_hbm": gbs / hbm, "measured_hbm_gbs": hbm,
+                           "frac_of_datasheet_8tbs": gbs / 8000.0, "kernels": kernels,
+                           "note": "event-timed inside each step, L2 flushed before the step"}
     print(json.dumps(line), flush=True)
 
 
