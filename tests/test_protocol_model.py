@@ -1,0 +1,32 @@
+"""The attention kernel's mbarrier protocol, model-checked on random schedules (CPU only): no
+data hazard and no deadlock in any of the kernel's layouts, and each planted protocol mistake
+is caught."""
+import random
+
+import pytest
+
+from protocol_model import LAYOUTS, MUTANTS, Deadlock, Violation, random_units, run
+
+SEEDS = 300
+
+
+@pytest.mark.parametrize("layout", LAYOUTS, ids=[f"nt{a}_nsm{b}_qt{int(c)}_k{d}_v{e}"
+                                                 for a, b, c, d, e in LAYOUTS])
+def test_protocol_holds(layout):
+    NT, NSM, q_tmem, NK, NV = layout
+    for seed in range(SEEDS):
+        units = random_units(random.Random(seed * 7 + NT))
+        run(units, NT, NSM, q_tmem, NK, NV, seed)
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_model_catches_planted_mistake(mutant):
+    caught = 0
+    for NT, NSM, q_tmem, NK, NV in LAYOUTS:
+        for seed in range(60):
+            units = random_units(random.Random(seed * 7 + NT))
+            try:
+                run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=mutant)
+            except (Violation, Deadlock):
+                caught += 1
+    assert caught > 0, f"the model did not catch: {MUTANTS[mutant]}"
