@@ -548,6 +548,11 @@ def run_gpu(args):
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
+    if fp8:  # the E4M3 path against its own datasheet figure (4.5 PFLOP/s dense)
+        line["pct_of_dense_e4m3_peak"] = {
+            "value": 100.0 * value / world / (DATASHEET_BF16_TFLOPS * FP8_OVER_BF16),
+            "peak_tflops": DATASHEET_BF16_TFLOPS * FP8_OVER_BF16,
+            "peak_source": "B200 datasheet dense E4M3"}
     if kgate is not None:
         line["k_smooth_gate"] = kgate
     if c["kmean"] or fp8:
