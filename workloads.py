@@ -18,7 +18,7 @@ import math
 import torch
 
 # The workloads (sizes as the pages' benchmarks and the quantised-attention table give them).
-CONFIGS = {
+WORKLOADS = {
     1: dict(workload="mha_b1_h2_s128_d64", b=1, hq=2, hk=2, sq=128, sk=128, dqk=64, dv=64,
             causal=False, kmean=False),
     2: dict(workload="gqa_b8_hq48_hk8_s2048_d64_causal", b=8, hq=48, hk=8, sq=2048, sk=2048,
@@ -51,7 +51,7 @@ HEAD_DIMS = ((64, 64), (128, 128), (192, 128), (256, 256))
 
 def config(n: int) -> dict:
     """Copy of workload ``n`` with its seed and softmax scale filled in."""
-    c = dict(CONFIGS[n])
+    c = dict(WORKLOADS[n])
     c["id"] = n
     c["seed"] = 1000 + n
     c["scale"] = 1.0 / math.sqrt(c["dqk"])
