@@ -6,7 +6,6 @@ sample stride off by one, a strict gate threshold, an unsquared gate mean) must 
 caught by at least one pin. The planted copies are built in a temporary directory on the CPU;
 the real oracle is untouched."""
 import os
-import subprocess
 
 import pytest
 
