@@ -269,7 +269,8 @@ B200ATTN_API int fp8_quantize(const void* x, const float* mean, void* x8, float*
  *   q8       device uint8 [b, sq, hq, dqk];  k8: [b, sk, hk, dqk];  v8: [b, sk, hk, dv];
  *            16-byte aligned, E4M3 codes (no NaN codes). Read only.
  *   q_descale  device fp32 [b, hq];  k_descale, v_descale: [b, hk]; 4-byte aligned, positive
- *            and finite (the product scale * q_descale * k_descale is kept at 2^-100 or more).
+ *            and finite. The exp2 factor |scale| * log2(e) * q_descale * k_descale is kept at
+ *            2^-100 or more, as attn_fwd keeps its own (the sign of scale is applied by the MMA).
  *   out, lse as in attn_fwd (O in bf16).
  *   dqk, dv  (128, 128) only (else B200ATTN_ERR_HEADDIM).
  *   other arguments, errors, allocation and concurrency as in attn_fwd.
