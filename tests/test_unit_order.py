@@ -1,0 +1,65 @@
+"""The persistent kernel's unit schedule (unit_of in csrc/attn_fwd_kernel.cuh and the grid size
+of csrc/attn_api.cu), transcribed and checked on the CPU: in every order (0 round robin,
+1 snake, 2 weight-major snake) each unit is taken by exactly one (CTA, round); a CTA's positions
+grow with the round, so once a round is past the last unit every later one is too (the kernel's
+loops stop at the first such round); and order 2 takes, per round, the most expensive units that
+are left (the k-th heaviest unit of every (batch, head) before any (k+1)-th)."""
+import random
+
+import pytest
+
+
+def unit_of(r, c, grid, n_units, order, bh_count, n_qu):
+    pos = r * grid + (grid - 1 - c if (order != 0 and (r & 1)) else c)
+    if pos >= n_units:
+        return -1
+    if order == 2:
+        k = pos // bh_count  # rank within its head (0 = the unit that sees the most keys)
+        bh = pos - k * bh_count
+        return bh * n_qu + k
+    return pos
+
+
+def schedule(bh_count, n_qu, n_sm, order):
+    n_units = bh_count * n_qu
+    grid = min(n_units, n_sm)
+    taken = {}
+    for c in range(grid):
+        r, last_pos = 0, -1
+        while True:
+            u = unit_of(r, c, grid, n_units, order, bh_count, n_qu)
+            if u < 0:
+                # every later round of this CTA is past the end as well
+                for r2 in range(r + 1, r + 4):
+                    assert unit_of(r2, c, grid, n_units, order, bh_count, n_qu) < 0
+                break
+            pos = r * grid + (grid - 1 - c if (order != 0 and (r & 1)) else c)
+            assert pos > last_pos
+            last_pos = pos
+            assert u not in taken, f"unit {u} taken twice"
+            taken[u] = (c, r)
+            r += 1
+    assert sorted(taken) == list(range(n_units)), "some unit never taken"
+    return taken, grid
+
+
+@pytest.mark.parametrize("order", [0, 1, 2])
+def test_every_unit_once(order):
+    rnd = random.Random(order)
+    cases = [(384, 8, 148), (128, 32, 148), (5, 256, 148), (16, 16, 148), (1, 1, 148), (3, 1, 148),
+             (1, 300, 148), (148, 1, 148), (149, 2, 148)]
+    cases += [(rnd.randint(1, 400), rnd.randint(1, 64), rnd.choice([1, 7, 132, 148])) for _ in range(60)]
+    for bh_count, n_qu, n_sm in cases:
+        schedule(bh_count, n_qu, n_sm, order)
+
+
+def test_weight_major_takes_heaviest_first():
+    # within a head, unit index k covers the query rows that see the most keys first (causal);
+    # order 2 hands out all heads' rank-k units before any rank-(k+1) unit
+    bh_count, n_qu, n_sm = 5, 256, 148
+    taken, grid = schedule(bh_count, n_qu, n_sm, 2)
+    ranks_by_round = {}
+    for u, (c, r) in taken.items():
+        ranks_by_round.setdefault(r, []).append(u % n_qu)
+    for r in sorted(ranks_by_round)[:-1]:
+        assert max(ranks_by_round[r]) <= min(ranks_by_round[r + 1])
