@@ -236,13 +236,14 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 }
 
 // Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, softmax
-// warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe>. Tensor
+// warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe, E4M3
+// inputs>. Tensor
 // memory holds two score buffers, one O per query tile and (when it fits) each tile's Q; shared
 // memory holds the Q staging buffer and the K / V rings. The (tiles, warpgroups) choice per head
 // dim is the measured fastest on B200 (d64: two tiles and two warpgroups, except for packed
 // sequences). The share of score pairs whose exp2 runs on the FMA pipe is the measured best per
-// head dim (3 of 8 at d64, 2 of 8 at d128 / d192, none at d256, which is bound by the tensor
-// core).
+// head dim (3 of 8 at d64, 2 of 8 at d128 / d192 and for E4M3 inputs, none at d256, which is
+// bound by the tensor core).
 using T64 = AttnTraits<64, 64, 128, 2, 2, true, 5, 5, 0x92u>;   // smem 32 + 80 + 80 (+32) KB
 using T64V = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 (+16) KB
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 + 96 + 64 KB
