@@ -74,7 +74,10 @@ def pin_sdpa(lib):
         err_o = np.max(np.abs(o - o_ref))
         err_l = np.max(np.abs(lse - lse_ref))
         assert err_o <= TOL, f"O vs torch SDPA: {err_o} on case {n}"
-        assert err_l <= TOL, f"LSE vs torch logsumexp: {err_l} on case {n}"
+        if err_l > TOL:  # report where, and both values, before failing
+            at = np.unravel_index(np.argmax(np.abs(lse - lse_ref)), lse.shape)
+            raise AssertionError(f"LSE vs torch logsumexp: {err_l} on case {n} at {at}: oracle "
+                                 f"{lse[at]!r}, torch {lse_ref[at]!r}")
 
 
 def pin_uniform_scores(lib):
