@@ -1,6 +1,7 @@
-"""Fused attention forward pass (with per-row log-sum-exp) and the K channel-mean pre-pass on
-B200 (sm_100a), as a thin Python binding over the C ABI of ``libb200attn.so``
-(declared in ``include/b200attn.h``).
+"""Fused attention forward pass (with per-row log-sum-exp) on B200 (sm_100a) -- dense, packed
+sequences, sliding window with sinks, and E4M3 inputs -- with the K channel-mean pre-pass, the
+K-smoothing gate and the E4M3 quantiser, as a thin Python binding over the C ABI of
+``libb200attn.so`` (declared in ``include/b200attn.h``).
 
 The binding only marshals arguments: it checks dtypes/devices/contiguity, allocates outputs
 with ``torch.empty`` and passes raw device pointers plus the current CUDA stream. Every step of
@@ -8,9 +9,10 @@ the computation runs in the library's CUDA kernels; there is no CPU or PyTorch f
 importing this package fails loudly when the library is missing.
 
 Raw C entry points, with the header's names and argument order, are exposed through ``lib``
-(a ``ctypes.CDLL``): ``lib.attn_fwd``, ``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``,
-``lib.k_smooth_sub``, ``lib.fp8_quantize``, ``lib.attn_fwd_fp8``, ``lib.attn_status_string``,
-``lib.attn_debug_status``.
+(a ``ctypes.CDLL``): every name in ``EXPORTS`` (``lib.attn_fwd``, ``lib.attn_fwd_varlen``,
+``lib.attn_fwd_window_sink``, ``lib.attn_fwd_fp8``, ``lib.fp8_quantize``, ``lib.k_smooth_gate``,
+``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``, ``lib.k_smooth_sub``,
+``lib.attn_status_string``, ``lib.attn_debug_status``, ``lib.attn_debug_starve``).
 """
 from __future__ import annotations
 
