@@ -67,3 +67,23 @@ def test_reference_arm_prints_on_rank_zero_only():
     assert outs[1] == ""
     line = json.loads(outs[0].splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_reference_line_carries_the_contract_keys():
+    """The reference arm's JSON line has every key of the benchmark contract, with its own
+    cpu_baseline and an e2e that moves no bytes."""
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--config", "1", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, env=dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0"),
+                       capture_output=True, text=True, timeout=600)
+    assert p.returncode == 0, p.stderr[-2000:]
+    line = json.loads(p.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e", "impl", "gpu_launches"):
+        assert key in line, key
+    assert line["steps"] == 1 and line["warmup"] == 0 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "mha_b1_h2_s128_d64"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
