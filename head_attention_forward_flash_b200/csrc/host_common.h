@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <mutex>
 
 #include "../../include/b200attn.h"
 
@@ -58,11 +59,13 @@ inline int check_arch()
 inline cudaMemPool_t scratch_pool()
 {
     static cudaMemPool_t pools[64] = {nullptr};
+    static std::mutex mu;  // first calls from several host threads create one pool per device
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return nullptr;
     }
+    std::lock_guard<std::mutex> lock(mu);
     if (pools[dev] == nullptr) {
         cudaMemPoolProps props = {};
         props.allocType = cudaMemAllocationTypePinned;
