@@ -63,3 +63,29 @@ def test_weight_major_takes_heaviest_first():
         ranks_by_round.setdefault(r, []).append(u % n_qu)
     for r in sorted(ranks_by_round)[:-1]:
         assert max(ranks_by_round[r]) <= min(ranks_by_round[r + 1])
+
+
+def per_cta_balance(b, hq, sq, NT, order, n_sm=148):
+    """max / mean of the per-CTA key-block totals of a causal square problem (cost of a unit =
+    its visited key blocks x its tiles)."""
+    from test_unit_ranges import unit_ranges
+    n_qu = (sq + NT * 128 - 1) // (NT * 128)
+    bh_count = b * hq
+    taken, grid = schedule(bh_count, n_qu, n_sm, order)
+    cost = {}
+    for u in taken:
+        qu = n_qu - 1 - (u % n_qu)  # within a head: most keys first
+        jb, nb, _, _ = unit_ranges(qu * NT * 128, sq, sq, NT, 128, True, -1)
+        cost[u] = (nb - jb) * NT
+    load = [0] * grid
+    for u, (c, _) in taken.items():
+        load[c] += cost[u]
+    return max(load) / (sum(load) / grid)
+
+
+def test_causal_balance_by_order():
+    # the causal workloads' geometry: 8 x 48 heads 2048^2, 128 heads 8192^2, 5 heads 65536^2
+    for b, hq, sq in [(8, 48, 2048), (1, 128, 8192), (1, 5, 65536)]:
+        rr = per_cta_balance(b, hq, sq, 2, 0)
+        wm = per_cta_balance(b, hq, sq, 2, 2)
+        assert wm <= 1.02 < 1.1 < rr, (b, hq, sq, rr, wm)
