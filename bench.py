@@ -54,7 +54,11 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.WORKLOADS))
+    # default: the largest single-GPU workload (b1 h5 65536^2 d128 causal)
+    ap.add_argument("--config", type=int, default=5, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with this many query heads (kv heads scaled by the "
+                         "same factor): a smaller case of the same kernel, for profiler captures")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -288,7 +292,7 @@ def run_gpu(args):
 
     import head_attention_forward_flash_b200 as b2
 
-    c = workloads.config(args.config)
+    c = workloads.with_heads(workloads.config(args.config), args.heads)
     c_rank = dict(c)
     c_rank["seed"] = rank_seed(c["seed"], rank)
     varlen = bool(c.get("varlen"))
@@ -586,7 +590,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return  # the oracle arm runs on rank 0 only
-    c = workloads.config(args.config)
+    c = workloads.with_heads(workloads.config(args.config), args.heads)
     if c.get("varlen"):  # the oracle on rows of the first sequence (a dense b = 1 problem)
         c, inputs0 = varlen_first_sequence(c, workloads.config_varlen_inputs(c))
         s = OracleSampler(c, inputs0)

@@ -102,6 +102,43 @@ def _want(t, name, dims):
         raise ValueError(f"{name} must be contiguous (BSHD)")
 
 
+def _want_out(t, name, shape, dtype, device):
+    """A caller-supplied output (or auxiliary) buffer: exactly ``shape`` and ``dtype``,
+    contiguous and on ``device`` -- a smaller buffer would be written past its end."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, "
+                         f"got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(ref, *named):
+    for name, t in named:
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, expected {ref.device}")
+
+
+def _attn_outputs(out, lse, return_lse, out_shape, lse_shape, device):
+    """Allocates O and LSE, or checks the caller's buffers."""
+    import torch
+    if out is None:
+        out = torch.empty(out_shape, dtype=torch.bfloat16, device=device)
+    else:
+        _want_out(out, "out", out_shape, torch.bfloat16, device)
+    if lse is not None:
+        _want_out(lse, "lse", lse_shape, torch.float32, device)
+    elif return_lse:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=device)
+    return out, lse
+
+
 def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
              return_lse: bool = True):
     """O = softmax(scale * Q K^T [+ causal mask]) V and the per-row LSE (natural log).
@@ -120,12 +157,10 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None
     bv, skv, hkv, dv = v.shape
     if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
         raise ValueError("inconsistent q/k/v shapes")
+    _same_device(q, ("k", k), ("v", v))
     if scale is None:
         scale = 1.0 / math.sqrt(dqk)
-    if out is None:
-        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q.device)
-    if return_lse and lse is None:
-        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q.device)
+    out, lse = _attn_outputs(out, lse, return_lse, (b, sq, hq, dv), (b, hq, sq), q.device)
     st = lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                       lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
                       1 if causal else 0, float(scale), _stream_ptr(q))
@@ -148,16 +183,12 @@ def attn_fwd_window_sink(q, k, v, causal: bool = False, window_left: int = -1, s
     bv, skv, hkv, dv = v.shape
     if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
         raise ValueError("inconsistent q/k/v shapes")
+    _same_device(q, ("k", k), ("v", v))
     if sinks is not None:
-        _want(sinks, "sinks", 1)
-        if sinks.dtype != torch.float32 or sinks.shape[0] != hq:
-            raise ValueError("sinks must be float32 with one logit per query head")
+        _want_out(sinks, "sinks", (hq,), torch.float32, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(dqk)
-    if out is None:
-        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q.device)
-    if return_lse and lse is None:
-        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q.device)
+    out, lse = _attn_outputs(out, lse, return_lse, (b, sq, hq, dv), (b, hq, sq), q.device)
     st = lib.attn_fwd_window_sink(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                   lse.data_ptr() if lse is not None else None,
                                   sinks.data_ptr() if sinks is not None else None, b, hq, hk, sq,
@@ -194,12 +225,11 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, caus
     b = cu_seqlens_q.shape[0] - 1
     if b < 0 or cu_seqlens_k.shape[0] != b + 1:
         raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold b + 1 offsets")
+    _same_device(q, ("k", k), ("v", v), ("cu_seqlens_q", cu_seqlens_q),
+                 ("cu_seqlens_k", cu_seqlens_k))
     if scale is None:
         scale = 1.0 / math.sqrt(dqk)
-    if out is None:
-        out = torch.empty((total_q, hq, dv), dtype=torch.bfloat16, device=q.device)
-    if return_lse and lse is None:
-        lse = torch.empty((hq, total_q), dtype=torch.float32, device=q.device)
+    out, lse = _attn_outputs(out, lse, return_lse, (total_q, hq, dv), (hq, total_q), q.device)
     st = lib.attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              lse.data_ptr() if lse is not None else None,
                              cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), b, hq, hk, total_q,
@@ -226,13 +256,17 @@ def fp8_quantize(x, mean=None, out=None, descale=None):
         raise TypeError("x must be bfloat16")
     b, s, h, d = x.shape
     if mean is not None:
-        _want(mean, "mean", 3)
-        if mean.dtype != torch.float32 or tuple(mean.shape) != (b, h, d):
-            raise ValueError("mean must be float32 [b, h, d]")
+        _want_out(mean, "mean", (b, h, d), torch.float32, x.device)
     if out is None:
         out = torch.empty((b, s, h, d), dtype=torch.uint8, device=x.device)
+    else:
+        if out.dtype == torch.float8_e4m3fn:
+            out = out.view(torch.uint8)
+        _want_out(out, "out", (b, s, h, d), torch.uint8, x.device)
     if descale is None:
         descale = torch.empty((b, h), dtype=torch.float32, device=x.device)
+    else:
+        _want_out(descale, "descale", (b, h), torch.float32, x.device)
     _check("fp8_quantize", lib.fp8_quantize(x.data_ptr(),
                                             mean.data_ptr() if mean is not None else None,
                                             out.data_ptr(), descale.data_ptr(), b, s, h, d,
@@ -253,17 +287,13 @@ def attn_fwd_fp8(q8, k8, v8, q_descale, k_descale, v_descale, causal: bool = Fal
     bv, skv, hkv, dv = v8.shape
     if bk != b or bv != b or dqk2 != dqk or skv != sk or hkv != hk:
         raise ValueError("inconsistent q/k/v shapes")
+    _same_device(q8, ("k8", k8), ("v8", v8))
     for name, t, n in (("q_descale", q_descale, hq), ("k_descale", k_descale, hk),
                        ("v_descale", v_descale, hk)):
-        _want(t, name, 2)
-        if t.dtype != torch.float32 or tuple(t.shape) != (b, n):
-            raise ValueError(f"{name} must be float32 [b, {n}]")
+        _want_out(t, name, (b, n), torch.float32, q8.device)
     if scale is None:
         scale = 1.0 / math.sqrt(dqk)
-    if out is None:
-        out = torch.empty((b, sq, hq, dv), dtype=torch.bfloat16, device=q8.device)
-    if return_lse and lse is None:
-        lse = torch.empty((b, hq, sq), dtype=torch.float32, device=q8.device)
+    out, lse = _attn_outputs(out, lse, return_lse, (b, sq, hq, dv), (b, hq, sq), q8.device)
     st = lib.attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_descale.data_ptr(),
                           k_descale.data_ptr(), v_descale.data_ptr(), out.data_ptr(),
                           lse.data_ptr() if lse is not None else None, b, hq, hk, sq, sk, dqk, dv,
@@ -281,6 +311,8 @@ def k_smooth_mean(k, mean=None):
     b, sk, hk, d = k.shape
     if mean is None:
         mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    else:
+        _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
     _check("k_smooth_mean",
            lib.k_smooth_mean(k.data_ptr(), mean.data_ptr(), b, hk, sk, d, _stream_ptr(k)))
     return mean
@@ -291,10 +323,10 @@ def k_smooth_mean_noalloc(k, mean):
     ``mean`` [b, hk, d] fp32 must be supplied by the caller."""
     import torch
     _want(k, "k", 4)
-    _want(mean, "mean", 3)
-    if k.dtype != torch.bfloat16 or mean.dtype != torch.float32:
-        raise TypeError("k must be bfloat16 and mean float32")
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
     b, sk, hk, d = k.shape
+    _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
     _check("k_smooth_mean_noalloc", lib.k_smooth_mean_noalloc(k.data_ptr(), mean.data_ptr(), b, hk,
                                                               sk, d, _stream_ptr(k)))
     return mean
@@ -312,9 +344,15 @@ def k_smooth_gate(k, threshold: float, mean=None, gate=None, ratio=None, return_
     b, sk, hk, d = k.shape
     if mean is None:
         mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    else:
+        _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
     if gate is None:
         gate = torch.empty((b, hk), dtype=torch.int32, device=k.device)
-    if return_ratio and ratio is None:
+    else:
+        _want_out(gate, "gate", (b, hk), torch.int32, k.device)
+    if ratio is not None:
+        _want_out(ratio, "ratio", (b, hk), torch.float32, k.device)
+    elif return_ratio:
         ratio = torch.empty((b, hk), dtype=torch.float32, device=k.device)
     st = lib.k_smooth_gate(k.data_ptr(), mean.data_ptr(), gate.data_ptr(),
                            ratio.data_ptr() if ratio is not None else None, b, hk, sk, d,
@@ -327,14 +365,14 @@ def k_smooth_sub(k, mean, out=None):
     """bf16(K - mean) with the [b, hk, d] fp32 mean broadcast over the sequence axis."""
     import torch
     _want(k, "k", 4)
-    _want(mean, "mean", 3)
-    if k.dtype != torch.bfloat16 or mean.dtype != torch.float32:
-        raise TypeError("k must be bfloat16 and mean float32")
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
     b, sk, hk, d = k.shape
-    if tuple(mean.shape) != (b, hk, d):
-        raise ValueError("mean must be [b, hk, d]")
+    _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
     if out is None:
         out = torch.empty_like(k)
+    else:
+        _want_out(out, "out", (b, sk, hk, d), torch.bfloat16, k.device)
     _check("k_smooth_sub", lib.k_smooth_sub(k.data_ptr(), mean.data_ptr(), out.data_ptr(), b, hk,
                                             sk, d, _stream_ptr(k)))
     return out

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <mutex>
 
 #include "attn_fwd_kernel.cuh"
@@ -39,20 +40,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+// Per-device caches below are atomics: concurrent first calls from several host threads store
+// the same value, and no thread reads a half-written one.
 int* status_word()
 {
-    static int* addr[64] = {nullptr};
+    static std::atomic<int*> addr[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (addr[dev] == nullptr) {
+    int* a = addr[dev].load(std::memory_order_relaxed);
+    if (a == nullptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
-        addr[dev] = static_cast<int*>(p);
+        a = static_cast<int*>(p);
+        addr[dev].store(a, std::memory_order_relaxed);
     }
-    return addr[dev];
+    return a;
 }
 
 // 4-D tensor map over a BSHD tensor [b, s, h, d] (innermost first: d, h, s, b) of bf16
@@ -88,18 +93,18 @@ bool tma_extent_ok(int64_t b, int64_t s, int64_t h, int64_t d)
 
 int sm_count()
 {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
             return 0;
         }
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 // Problem geometry. Dense: b batches of sq queries and sk keys. Packed sequences: b sequences,
@@ -123,14 +128,14 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
                 const Shape& sh, float scale, cudaStream_t stream)
 {
     const int64_t b = sh.b, hq = sh.hq, hk = sh.hk, sq = sh.sq, sk = sh.sk;
-    static bool attr_done[64] = {false};
+    static std::atomic<bool> attr_done[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
     auto kern = attn_fwd_kernel<T, CAUSAL, VARLEN, EXT>;
-    if (!attr_done[dev]) {
+    if (!attr_done[dev].load(std::memory_order_relaxed)) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)T::SMEM_BYTES) != cudaSuccess) {
             cudaGetLastError();
@@ -149,7 +154,7 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
                 (int64_t)2 * 128 * T::SOFTMAX_REGS + 128 * T::AUX_REGS)
                 return B200ATTN_ERR_CUDA;
         }
-        attr_done[dev] = true;
+        attr_done[dev].store(true, std::memory_order_relaxed);
     }
     // packed sequences: one batch of all rows; each unit adds its sequence's first row
     const int64_t mb = VARLEN ? 1 : b;

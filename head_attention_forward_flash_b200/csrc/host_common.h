@@ -4,6 +4,7 @@
 
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/b200attn.h"
@@ -34,13 +35,17 @@ inline bool numel(std::initializer_list<int64_t> dims, int64_t* out)
 // sm_100 check for the current device (cached per device). Returns a status code.
 inline int check_arch()
 {
-    static int cached[64] = {0};  // 0 unknown, 1 ok, 2 wrong arch
+    // 0 unknown, 1 ok, 2 wrong arch; atomic, so concurrent first calls do not race
+    static std::atomic<int> cached[64] = {};
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
-    if (dev < 64 && cached[dev] != 0) return cached[dev] == 1 ? B200ATTN_OK : B200ATTN_ERR_ARCH;
+    if (dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c != 0) return c == 1 ? B200ATTN_OK : B200ATTN_ERR_ARCH;
+    }
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
@@ -48,7 +53,7 @@ inline int check_arch()
         return B200ATTN_ERR_CUDA;
     }
     const bool ok = (major == 10 && minor == 0);
-    if (dev < 64) cached[dev] = ok ? 1 : 2;
+    if (dev < 64) cached[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
     return ok ? B200ATTN_OK : B200ATTN_ERR_ARCH;
 }
 

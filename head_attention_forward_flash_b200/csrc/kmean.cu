@@ -7,6 +7,7 @@
 // each channel in a fixed order, so the result is bit-identical from run to run (the two
 // deterministic kernels behind one host call of "[HIP] Mha v4: run the K-smoothing gate as one
 // HIP call", Summary and commit message).
+#include <atomic>
 #include <cmath>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -298,21 +299,24 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
 // host-side name of a __device__ array is not a device address).
 static float* noalloc_scratch()
 {
-    static float* addr[64] = {nullptr};
+    // atomic: concurrent first calls from several host threads store the same address
+    static std::atomic<float*> addr[64] = {};
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return nullptr;
     }
-    if (addr[dev] == nullptr) {
+    float* a = addr[dev].load(std::memory_order_relaxed);
+    if (a == nullptr) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_kmean_scratch) != cudaSuccess) {
             cudaGetLastError();
             return nullptr;
         }
-        addr[dev] = static_cast<float*>(p);
+        a = static_cast<float*>(p);
+        addr[dev].store(a, std::memory_order_relaxed);
     }
-    return addr[dev];
+    return a;
 }
 
 extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk,

@@ -434,7 +434,7 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1)
 // SM) to the other pairs. Round-to-nearest splits x = j + f with |f| <= 1/2 (adding and then
 // subtracting 1.5 * 2^23 rounds to an integer, and leaves j in the low bits of the sum),
 // 2^f comes from the cubic 1 + f (c1 + f (c2 + f c3)) (a minimax fit, relative error 1.0e-4
-// in fp32; fit_exp2_poly.py derives it), and j is added to the exponent field as an integer.
+// in fp32; tests/fit_exp2_poly.py derives it), and j is added to the exponent field as an integer.
 // x is clamped at -127 first: there j = -127, f = 0, 2^f = 1 exactly and the result is +0, as
 // for every smaller x (so -inf, a masked score, gives exactly 0 like ex2.approx.ftz).
 constexpr float kExp2C1 = 0.6932829022407532f;

@@ -22,6 +22,13 @@
  *   - Kernels never read past a tensor's logical end: tile loads past an edge are clipped and
  *     zero-filled by TMA, and stores are predicated (the same page's notes on speculative
  *     reads past the logical sequence).
+ *   - Concurrency: calls from several host threads, or on several streams, may overlap; no two
+ *     of them share scratch memory (k_smooth_mean_noalloc excepted: see there), and the
+ *     library's per-device caches are atomics. Two things are shared by every attention launch
+ *     on a device: the device error word -- attn_debug_status() reports and clears a
+ *     bounded-wait timeout from whichever launch set it -- and the failure test that
+ *     attn_debug_starve() arms, which applies to the next attention launch of the process,
+ *     whatever thread makes it.
  */
 #ifndef B200ATTN_H
 #define B200ATTN_H
@@ -81,7 +88,7 @@ enum b200attn_status {
  *   dqk, dv  one of (64,64), (128,128), (192,128), (256,256).
  *   causal   0 or nonzero.
  *   scale    finite; usually 1/sqrt(dqk).
- * Allocates nothing. Safe to call concurrently on different streams.
+ * Allocates nothing. Concurrency as in the conventions above.
  */
 B200ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
              int64_t b, int64_t hq, int64_t hk, int64_t sq, int64_t sk, int64_t dqk, int64_t dv,
@@ -135,7 +142,7 @@ B200ATTN_API int attn_fwd_window_sink(const void* q, const void* k, const void* 
  *   b, total_q, max_sq  may be 0 (nothing is launched); total_k may be 0 (every row empty).
  *   hk, hq, dqk, dv, causal, scale  as in attn_fwd.
  * Errors as attn_fwd; also ERR_RANGE when total_q, total_k or b * hq * ceil(max_sq / 128)
- * reaches 2^31. Allocates nothing. Safe to call concurrently on different streams.
+ * reaches 2^31. Allocates nothing. Concurrency as in the conventions above.
  */
 B200ATTN_API int attn_fwd_varlen(const void* q, const void* k, const void* v, void* out, float* lse,
                                  const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
@@ -211,7 +218,7 @@ B200ATTN_API int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, in
  *   threshold  finite (NaN / inf -> ERR_SCALE).
  *   b, hk, sk, d  as in k_smooth_mean (sk > 0, d in {64, 128, 256}).
  * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`
- * (as k_smooth_mean). Safe to call concurrently on different streams.
+ * (as k_smooth_mean). Concurrency as in the conventions above.
  */
 B200ATTN_API int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* ratio, int64_t b,
                                int64_t hk, int64_t sk, int64_t d, float threshold, void* stream);
@@ -249,7 +256,7 @@ B200ATTN_API int k_smooth_sub(const void* k, const float* mean, void* k_out, int
  *   descale   device fp32 [b, h], 4-byte aligned. Fully written.
  *   b, h      >= 0 (0: nothing to do);  s >= 0 (0: every descale is 1);  d in {64, 128, 256}.
  * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`.
- * Two kernels (per-chunk amax, then fold and convert). Safe on concurrent streams.
+ * Two kernels (per-chunk amax, then fold and convert). Concurrency as in the conventions above.
  */
 B200ATTN_API int fp8_quantize(const void* x, const float* mean, void* x8, float* descale,
                               int64_t b, int64_t s, int64_t h, int64_t d, void* stream);

@@ -4,7 +4,7 @@ p(f) = 1 + f * (c1 + f * (c2 + f * c3)) on f in [-1/2, 1/2], minimising the larg
 |p(f) / 2^f - 1| with Lawson's iteratively re-weighted least squares (a minimax fit). The constant
 term is pinned to exactly 1, so that p(0) = 1 and the exponent trick maps x = -127 to +0 exactly.
 
-Run: python fit_exp2_poly.py   (prints the three fp32 coefficients and the fp32 error bound).
+Run: python tests/fit_exp2_poly.py   (prints the three fp32 coefficients and the fp32 error bound).
 """
 import numpy as np
 

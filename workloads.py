@@ -58,6 +58,20 @@ def config(n: int) -> dict:
     return c
 
 
+def with_heads(c: dict, hq: int) -> dict:
+    """Workload ``c`` with ``hq`` query heads and the kv heads scaled by the same factor (the
+    group size stays), named after the new head count; ``hq`` = 0 leaves it unchanged."""
+    if not hq or hq == c["hq"]:
+        return c
+    group = c["hq"] // c["hk"]
+    if hq % group != 0:
+        raise ValueError(f"{hq} query heads do not form groups of {group}")
+    c = dict(c)
+    c["hq"], c["hk"] = hq, hq // group
+    c["workload"] = f"{c['workload']}_heads{hq}"
+    return c
+
+
 def flops(c: dict) -> float:
     """Algorithmic FLOPs of one forward pass: 2*b*hq*sq*sk*(dqk+dv), halved when causal (for
     packed sequences, the sum of that over the sequences; with a sliding window, 2*b*hq*(dqk+dv)
