@@ -90,6 +90,7 @@ struct AttnParams {
     int* status;      // device error word
     unsigned long long timeout_ns;
     int starve;       // failure test: the TMA producer loads nothing (see attn_debug_starve)
+    int alt;          // two tiles: their softmax take turns block by block (else run freely)
     // E4M3 inputs: fp32 descales per (batch, head) of Q [b, hq], K and V [b, hk] (else null)
     const float* q_descale;
     const float* k_descale;
@@ -148,15 +149,16 @@ struct AttnTraits {
     static constexpr uint32_t BARS_OFF = O_OFF + (O_TMA ? O_STAGE_BYTES : 0);
     static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(NSM == 1 || NSM == NT, "");
+    static_assert(NSM == NT, "one softmax warpgroup per query tile (and one MMA issuer each)");
     // Threads: NSM softmax warpgroups, then the MMA warp and the TMA warp. With two softmax
     // warpgroups the block is three full warpgroups (two warps idle) so that registers can
     // move between them: at launch every thread has LAUNCH_REGS (the cap for 384 threads);
     // the third warpgroup drops to AUX_REGS and the softmax warpgroups rise to SOFTMAX_REGS,
     // which keeps the block's total unchanged (a larger total would never be granted).
     static constexpr int NUM_THREADS = NSM == 1 ? 192 : 384;
-    static constexpr int MMA_WARP = 4 * NSM;
+    static constexpr int MMA_WARP = 4 * NSM;       // MMA issuer (tile 0, or every tile when NT = 1)
     static constexpr int TMA_WARP = 4 * NSM + 1;
+    static constexpr int MMA_WARP2 = 4 * NSM + 2;  // NT = 2: issuer of tile 1's MMAs
     static constexpr int LAUNCH_REGS = 168;
     static constexpr int SOFTMAX_REGS = 224;
     static constexpr int AUX_REGS = 56;
@@ -377,11 +379,11 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NK; ++s) {
             mbar_init(bar_kfull(s), 1);
-            mbar_init(bar_kempty(s), 1);
+            mbar_init(bar_kempty(s), NT);  // one commit per MMA issuer
         }
         for (int s = 0; s < NV; ++s) {
             mbar_init(bar_vfull(s), 1);
-            mbar_init(bar_vempty(s), 1);
+            mbar_init(bar_vempty(s), NT);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_s_full(s), 1);
@@ -389,8 +391,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         }
         mbar_init(bar_pv_done, 1);
         mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : 1);  // per-tile copy-out / last Q K^T
-        mbar_init(bar_mma_done, 1);
+        // per-tile copy-out (Q in TMEM) / each issuer's last Q K^T of the unit
+        mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : NT);
+        mbar_init(bar_mma_done, NT);
         for (int t = 0; t < NT; ++t) {
             mbar_init(bar_q_tmem(t), 128);
             mbar_init(bar_o_full(t), 1);
@@ -534,76 +537,83 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             if (q_cnt > 0)
                 mbar_wait_drain(bar_q_full, (uint32_t)(q_cnt - 1) & 1u, p.timeout_ns, p.status);
         }
-    } else if (warp == T::MMA_WARP) {
-        // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
+    } else if (warp == T::MMA_WARP || (NT == 2 && warp == T::MMA_WARP2)) {
+        // ------------------------------ MMA issuers ------------------------------
+        // NT = 2: one warp per query tile (warp MMA_WARP issues tile 0's MMAs, warp MMA_WARP2
+        // tile 1's), so the two tiles' instruction streams are issued side by side. Each tile has
+        // one score buffer, so its chain is Q K^T(j), then P V(j) once P(j) is out, then
+        // Q K^T(j+1). NT = 1: one warp; its tile alternates between the two score buffers, so
+        // Q K^T(g+1) is issued before P V(g).
+        // The whole warp runs the loop (waits included) with warp-uniform values; one elected
+        // lane issues each batch of MMAs and its commits.
+        {
+            const int my_tt = (warp == T::MMA_WARP) ? 0 : 1;
             bool ok = true;
-            int kq = 0, vq = 0;  // K / V items taken
-            int64_t gi = 0;      // global item counter (score buffer and barrier phases)
+            int kq = 0, vq = 0;  // K / V blocks taken
+            int64_t jg = 0;      // key blocks stepped through (all units)
             int units = 0;       // busy units started
-            uint32_t kaddr = 0, vaddr = 0;
-            int kslot = 0, vslot = 0;
-            // Q K^T of item gi = (block j, tile tt) of the current unit.
-            // (first: the unit's first visited key block)
-            auto qk = [&](bool first, int tt, bool last_item) {
+            auto wait_all = [&](uint32_t bar, uint32_t parity) {
+                return __all_sync(FULL, mbar_wait(bar, parity, wc, kErrTimeout));
+            };
+            // Q K^T of item g = (block, tile tt) of the current unit. Every issuer takes K(j)
+            // itself: the slot is freed when all NT issuers have committed kempty.
+            auto qk = [&](int64_t g, bool first, int tt, bool last_item) {
                 if (T::Q_TMEM && first) {  // this tile's Q of the new unit must be in TMEM
-                    if (!mbar_wait(bar_q_tmem(tt), (uint32_t)(units & 1), wc, kErrTimeout)) {
+                    if (!wait_all(bar_q_tmem(tt), (uint32_t)(units & 1))) {
                         ok = false;
                         return;
                     }
                     tc_fence_after_sync();
                 }
-                if (tt == 0) {
-                    kslot = kq % NK;
-                    const uint32_t phase = (uint32_t)(kq / NK) & 1u;
-                    ++kq;
-                    if (!mbar_wait(bar_kfull(kslot), phase, wc, kErrTimeout)) {
-                        ok = false;
-                        return;
-                    }
-                    kaddr = k_slots + kslot * T::K_TILE_BYTES;
-                }
-                issue_qk_mmas<T>(tmem + (uint32_t)(gi & 1) * BN,
-                                 T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
-                                           : q_stage + tt * T::Q_TILE_BYTES,
-                                 kaddr, p.idesc_qk);
-                tc_commit(bar_s_full(gi & 1));
-                if (tt == NT - 1) tc_commit(bar_kempty(kslot));
-                if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
-            };
-            // P V of item g = (block j, tile tt) of busy unit number uidx.
-            auto pv = [&](int64_t g, bool first, int tt, bool last_block, int uidx) {
-                if (!mbar_wait(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u, wc, kErrTimeout)) {
+                const int kslot = kq % NK;
+                const uint32_t phase = (uint32_t)(kq / NK) & 1u;
+                ++kq;
+                if (!wait_all(bar_kfull(kslot), phase)) {
                     ok = false;
                     return;
                 }
-                if (first && uidx > 0 &&
-                    !mbar_wait(bar_o_free(tt), (uint32_t)(uidx - 1) & 1u, wc, kErrTimeout)) {
+                if (elect_one()) {
+                    issue_qk_mmas<T>(tmem + (uint32_t)(g & 1) * BN,
+                                     T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
+                                               : q_stage + tt * T::Q_TILE_BYTES,
+                                     k_slots + kslot * T::K_TILE_BYTES, p.idesc_qk);
+                    tc_commit(bar_s_full(g & 1));
+                    tc_commit(bar_kempty(kslot));
+                    if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
+                }
+                __syncwarp();
+            };
+            // P V of item g = (block, tile tt) of busy unit number uidx.
+            auto pv = [&](int64_t g, bool first, int tt, bool last_block, int uidx) {
+                if (!wait_all(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u)) {
+                    ok = false;
+                    return;
+                }
+                if (first && uidx > 0 && !wait_all(bar_o_free(tt), (uint32_t)(uidx - 1) & 1u)) {
                     ok = false;
                     return;
                 }
                 tc_fence_after_sync();
-                if (tt == 0) {
-                    vslot = vq % NV;
-                    const uint32_t phase = (uint32_t)(vq / NV) & 1u;
-                    ++vq;
-                    if (!mbar_wait(bar_vfull(vslot), phase, wc, kErrTimeout)) {
-                        ok = false;
-                        return;
-                    }
-                    vaddr = v_slots + vslot * T::V_TILE_BYTES;
+                const int vslot = vq % NV;
+                const uint32_t phase = (uint32_t)(vq / NV) & 1u;
+                ++vq;
+                if (!wait_all(bar_vfull(vslot), phase)) {
+                    ok = false;
+                    return;
                 }
-                issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)(g & 1) * BN, vaddr,
-                                 !first);
-                if (NT == 1) tc_commit(bar_pv_done);
-                if (tt == NT - 1) tc_commit(bar_vempty(vslot));
-                if (last_block) tc_commit(bar_o_full(tt));
+                if (elect_one()) {
+                    issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)(g & 1) * BN,
+                                     v_slots + vslot * T::V_TILE_BYTES, !first);
+                    if (NT == 1) tc_commit(bar_pv_done);
+                    tc_commit(bar_vempty(vslot));
+                    if (last_block) tc_commit(bar_o_full(tt));
+                }
+                __syncwarp();
             };
-            // The P V of each item is issued after the next item's Q K^T (also across units), so
-            // the tensor core computes the next S while the softmax works on this one.
-            bool pend = false, pend_last = false;
-            bool pend_first = false;
-            int pend_tt = 0, pend_u = 0;
+            // NT = 1: the P V of each item is issued after the next item's Q K^T (also across
+            // units), so the tensor core computes the next S while the softmax works on this one.
+            bool pend = false, pend_last = false, pend_first = false;
+            int pend_u = 0;
             int64_t pend_g = 0;
             for (int64_t r = 0; ok; ++r) {
                 const int64_t u = unit_of(r);
@@ -611,31 +621,35 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 if (t.n_blocks <= t.j_begin) continue;
                 if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
-                    if (!mbar_wait(bar_q_full, (uint32_t)(units & 1), wc, kErrTimeout)) {
+                    if (!wait_all(bar_q_full, (uint32_t)(units & 1))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after_sync();
                 }
-                for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
-                    for (int tt = 0; tt < NT && ok; ++tt) {
-                        const bool last_item = (j == t.n_blocks - 1) && (tt == NT - 1);
-                        qk(j == t.j_begin, tt, last_item);
+                for (int j = t.j_begin; j < t.n_blocks && ok; ++j, ++jg) {
+                    const bool first = j == t.j_begin, last = j == t.n_blocks - 1;
+                    if constexpr (NT == 2) {
+                        const int64_t g = jg * 2 + my_tt;
+                        qk(g, first, my_tt, last);
+                        if (ok) pv(g, first, my_tt, last, units);
+                    } else {
+                        qk(jg, first, 0, last);
                         if (!ok) break;
-                        if (pend) pv(pend_g, pend_first, pend_tt, pend_last, pend_u);
+                        if (pend) pv(pend_g, pend_first, 0, pend_last, pend_u);
                         pend = true;
-                        pend_g = gi;
-                        pend_first = (j == t.j_begin);
-                        pend_tt = tt;
-                        pend_last = (j == t.n_blocks - 1);
+                        pend_g = jg;
+                        pend_first = first;
+                        pend_last = last;
                         pend_u = units;
-                        ++gi;
                     }
                 }
                 ++units;
             }
-            if (ok && pend) pv(pend_g, pend_first, pend_tt, pend_last, pend_u);
-            tc_commit(bar_mma_done);  // drain every MMA this thread issued before teardown
+            if (NT == 1 && ok && pend) pv(pend_g, pend_first, 0, pend_last, pend_u);
+            // drain every MMA this warp issued before teardown
+            if (elect_one()) tc_commit(bar_mma_done);
+            __syncwarp();
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
     } else if (warp < T::MMA_WARP) {
@@ -683,7 +697,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 
         // Epilogue of tile tt of busy unit number uidx: wait for that tile's last P V, read this
         // row of its O from TMEM (then free the accumulator), write O / l in bf16 and the LSE.
-        auto epilogue = [&](const UnitInfo& t, int tt, float m_ref, float l, int uidx) -> bool {
+        auto epilogue = [&](int64_t u, int tt, float m_ref, float l, int uidx) -> bool {
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
             if (!__all_sync(FULL,
                             mbar_wait(bar_o_full(tt), (uint32_t)(uidx & 1), wc, kErrTimeout)))
                 return false;
@@ -766,8 +781,138 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             return true;
         };
 
+        // One key block of one query tile: mask (MASKED only), row max, lazy rescale, exp2 and
+        // row sums, P into tensor memory. MASKED is a compile-time flag, so the common block
+        // with every key allowed runs one straight-line body with no per-chunk branches.
+        int64_t lim[NTW] = {};  // last allowed key of this thread's row in each tile
+        int64_t lol[NTW] = {};  // first allowed key (the window's lower bound), may be negative
+        float m_ref[NTW] = {};  // exponent reference (log2 units); moves lazily
+        float l[NTW] = {};      // sum of exp2(x - m_ref) over the keys seen so far
+        int j_begin = 0;
+        auto softmax_block = [&](const bool MASKED, uint32_t(&sr)[BN], int k, int tt, int j,
+                                 int64_t g, uint32_t s_col) -> bool {
+            // Keys j*BN + c with lor <= c <= rel are allowed. Per 32-key chunk the warp takes
+            // one of three uniform paths: every row of the warp allows the whole chunk
+            // (nothing to do), none allows any of it (skipped below: no max, P = 0 without
+            // exp2), or the chunk holds some row's bound: then the disallowed scores become
+            // -inf, so the max ignores them and their p = exp2(-inf) is exactly 0 (the scale
+            // factor is never 0: the launch clamps it to at least 2^-100).
+            uint32_t skip = 0;  // bit ch: no row of this warp allows a key of chunk ch
+            if (MASKED) {
+                int64_t rel64 = lim[k] - (int64_t)j * BN;
+                rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
+                int lor = 0;  // no lower bound without a window
+                if (EXT) {
+                    int64_t lor64 = lol[k] - (int64_t)j * BN;
+                    lor = (int)(lor64 < 0 ? 0 : (lor64 > BN ? BN : lor64));
+                }
+                const int rel = (int)rel64;
+                const int rel_lo = __reduce_min_sync(FULL, rel);
+                const int rel_hi = __reduce_max_sync(FULL, rel);
+                const int lor_lo = EXT ? __reduce_min_sync(FULL, lor) : 0;
+                const int lor_hi = EXT ? __reduce_max_sync(FULL, lor) : 0;
+#pragma unroll
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    if (ch * 32 > rel_hi || ch * 32 + 31 < lor_lo) {
+                        skip |= 1u << ch;
+                        continue;
+                    }
+                    if (ch * 32 + 31 <= rel_lo && ch * 32 >= lor_hi) continue;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = ch * 32 + e;
+                        sr[c] = (c <= rel && c >= lor) ? sr[c] : 0xff800000u;
+                    }
+                }
+            }
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                if (MASKED && ((skip >> ch) & 1u)) continue;
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    mx[c & 3] = fmax3(mx[c & 3], __uint_as_float(sr[ch * 32 + 2 * c]),
+                                      __uint_as_float(sr[ch * 32 + 2 * c + 1]));
+            }
+            const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
+            const float m_new = fmaxf(m_ref[k], m_blk);
+            // Lazy rescale: keep the old reference while the running max stays within 2^8 of
+            // it; the final O / l uses the same reference, so the result is exact.
+            const bool need = m_new > m_ref[k] + 8.0f;
+            float alpha = 1.f;
+            if (need) {
+                alpha = ex2(m_ref[k] - m_new);
+                m_ref[k] = m_new;
+                l[k] *= alpha;
+            }
+            if (j > j_begin && __any_sync(FULL, need)) {
+                // O holds blocks < j of this tile: scale it in place once its last P V is
+                // complete. With two tiles that P V was issued by this tile's issuer before this
+                // item's Q K^T, so it is complete now that S has landed (a commit covers all
+                // earlier MMAs of its thread). With one tile it is item g-1, issued after this
+                // item's Q K^T: wait for it (bar_pv_done is then in phase g-1 or g, so the
+                // parity test on phase g-1 is unambiguous).
+                if (NT == 1) {
+                    if (!__all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(g - 1) & 1u, wc,
+                                                    kErrTimeout)))
+                        return false;
+                    tc_fence_after_sync();
+                }
+#pragma unroll 1
+                for (int c = 0; c < T::DV / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+                    tmem_st32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
+                }
+            }
+            const float neg_m = (m_ref[k] == -INFINITY) ? 0.f : -m_ref[k];
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t pk[16];
+                if (MASKED && ((skip >> ch) & 1u)) {  // no row of this warp allows a key here
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) pk[c] = 0u;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int e = ch * 32 + 2 * c;
+                        float x0, x1;
+                        fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2, neg_m, x0,
+                             x1);
+                        float p0, p1;
+                        if ((T::EXP_FMA_PAIRS >> (c & 7)) & 1u) {
+                            exp2_fma_pair(x0, x1, p0, p1);
+                        } else {
+                            p0 = ex2(x0);
+                            p1 = ex2(x1);
+                        }
+                        add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
+                        if constexpr (T::FP8) {  // four E4M3 weights per column
+                            const uint32_t h2 = pack_e4m3x2(p0, p1);
+                            if (c & 1) pk[c >> 1] |= h2 << 16;
+                            else pk[c >> 1] = h2;
+                        } else {
+                            pk[c] = pack_bf16x2(p0, p1);
+                        }
+                    }
+                }
+                // P chunk ch (16 columns of bf16 pairs, or 8 of E4M3 quads) overwrites S columns
+                // already read
+                if constexpr (T::FP8) tmem_st8(s_col + ch * 8, pk);
+                else tmem_st16(s_col + ch * 16, pk);
+            }
+            l[k] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            return true;
+        };
+
         bool pend = false;  // a finished unit whose epilogues have not run yet
-        UnitInfo pend_t{};
+        int64_t pend_u = 0;
         float pend_m[NTW], pend_l[NTW];
 #pragma unroll
         for (int k = 0; k < NTW; ++k) pend_m[k] = pend_l[k] = 0.f;
@@ -795,8 +940,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 continue;
             }
-            const int64_t rn = busy_from(r + 1);
-            const int64_t un = rn >= 0 ? unit_of(rn) : -1;
+            const bool has_next = busy_from(r + 1) >= 0;
             if constexpr (T::FP8) {
                 // S holds sums of code products; the descales fold into the exp2 factor, kept at
                 // 2^-100 or more as on the host (a NaN product also becomes 2^-100)
@@ -804,10 +948,6 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                                 __ldg(p.k_descale + t.bi * p.hk + t.g);
                 sl2 = f > 0x1p-100f ? f : 0x1p-100f;
             }
-            int64_t lim[NTW];  // last allowed key of this thread's row in each tile
-            int64_t lol[NTW];  // first allowed key (the window's lower bound), may be negative
-            float m_ref[NTW];  // exponent reference (log2 units); moves lazily
-            float l[NTW];      // sum of exp2(x - m_ref) over the keys seen so far
             // A sink logit starts every row with that logit as reference and exp2(0) = 1 in
             // the sum: it then joins the denominator exactly, through every lazy rescale.
             const bool has_sink = EXT && p.sinks != nullptr;
@@ -822,19 +962,34 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 m_ref[k] = sink_l2;
                 l[k] = has_sink ? 1.f : 0.f;
             }
+            j_begin = t.j_begin;
+            const int n_blocks = t.n_blocks, mask_lo = t.mask_lo, mask_from = t.mask_from;
 
-            for (int j = t.j_begin; j < t.n_blocks && ok; ++j, ++jg) {
+            for (int j = j_begin; j < n_blocks && ok; ++j, ++jg) {
 #pragma unroll
                 for (int k = 0; k < NTW; ++k) {
                     const int tt = tile_of(k);
                     const int64_t g = jg * NT + tt;  // global item number
                     const int sb = (int)(g & 1);     // score buffer
                     const uint32_t s_col = tl + sb * BN;
+                    if (NT == 2 && p.alt) {
+                        // The two tiles' softmax take turns: tile 1's block jg after tile 0's,
+                        // tile 0's block jg after tile 1's block jg-1 (p_full of the other tile
+                        // completes once per block, and cannot run a phase ahead of this wait).
+                        bool w = true;
+                        if (tt == 1)
+                            w = mbar_wait(bar_p_full(0), (uint32_t)(jg & 1), wc, kErrTimeout);
+                        else if (jg > 0)
+                            w = mbar_wait(bar_p_full(1), (uint32_t)((jg - 1) & 1), wc,
+                                          kErrTimeout);
+                        ok = __all_sync(FULL, w);
+                        if (!ok) break;
+                    }
                     ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(g >> 1) & 1u, wc,
                                                     kErrTimeout));
                     if (!ok) break;
                     tc_fence_after_sync();
-                    if (T::Q_TMEM && j == t.n_blocks - 1 && un >= 0) {
+                    if (T::Q_TMEM && j == n_blocks - 1 && has_next) {
                         // This tile's last Q K^T of the unit is complete (its S has landed), so
                         // its Q columns can take the next unit's Q now, ahead of this softmax.
                         ok = copy_q(units + 1, tt);
@@ -845,130 +1000,17 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     for (int c = 0; c < BN / 32; ++c)
                         tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                     tmem_wait_ld();
-
-                    // Keys j*BN + c with lor <= c <= rel are allowed. Per 32-key chunk the warp
-                    // takes one of three uniform paths: every row of the warp allows the whole
-                    // chunk (nothing to do), none allows any of it (skipped below: no max, P = 0
-                    // without exp2), or the chunk holds some row's bound: then the disallowed
-                    // scores become -inf, so the max ignores them and their p = exp2(-inf) is
-                    // exactly 0 (the scale factor is never 0: the launch clamps it to at least
-                    // 2^-100).
-                    uint32_t skip = 0;  // bit ch: no row of this warp allows a key of chunk ch
-                    if ((EXT && j < t.mask_lo) || j >= t.mask_from) {
-                        int64_t rel64 = lim[k] - (int64_t)j * BN;
-                        rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
-                        int lor = 0;  // no lower bound without a window
-                        if (EXT) {
-                            int64_t lor64 = lol[k] - (int64_t)j * BN;
-                            lor = (int)(lor64 < 0 ? 0 : (lor64 > BN ? BN : lor64));
-                        }
-                        const int rel = (int)rel64;
-                        const int rel_lo = __reduce_min_sync(FULL, rel);
-                        const int rel_hi = __reduce_max_sync(FULL, rel);
-                        const int lor_lo = EXT ? __reduce_min_sync(FULL, lor) : 0;
-                        const int lor_hi = EXT ? __reduce_max_sync(FULL, lor) : 0;
-#pragma unroll
-                        for (int ch = 0; ch < BN / 32; ++ch) {
-                            if (ch * 32 > rel_hi || ch * 32 + 31 < lor_lo) {
-                                skip |= 1u << ch;
-                                continue;
-                            }
-                            if (ch * 32 + 31 <= rel_lo && ch * 32 >= lor_hi) continue;
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int c = ch * 32 + e;
-                                sr[c] = (c <= rel && c >= lor) ? sr[c] : 0xff800000u;
-                            }
-                        }
-                    }
-                    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-                    for (int ch = 0; ch < BN / 32; ++ch) {
-                        if ((skip >> ch) & 1u) continue;
-#pragma unroll
-                        for (int c = 0; c < 16; ++c)
-                            mx[c & 3] = fmax3(mx[c & 3], __uint_as_float(sr[ch * 32 + 2 * c]),
-                                              __uint_as_float(sr[ch * 32 + 2 * c + 1]));
-                    }
-                    const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-                    const float m_blk = (bmax == -INFINITY) ? -INFINITY : bmax * sl2;
-                    const float m_new = fmaxf(m_ref[k], m_blk);
-                    // Lazy rescale: keep the old reference while the running max stays within
-                    // 2^8 of it; the final O / l uses the same reference, so the result is exact.
-                    const bool need = m_new > m_ref[k] + 8.0f;
-                    float alpha = 1.f;
-                    if (need) {
-                        alpha = ex2(m_ref[k] - m_new);
-                        m_ref[k] = m_new;
-                        l[k] *= alpha;
-                    }
-                    if (j > t.j_begin && __any_sync(FULL, need)) {
-                        // O holds blocks < j of this tile: scale it in place once its last P V
-                        // is complete. With two tiles that P V is item g-2, issued before this
-                        // item's Q K^T, so it is complete now that S has landed. With one tile it
-                        // is item g-1: wait for it (bar_pv_done is then in phase g-1 or g, so
-                        // the parity test on phase g-1 is unambiguous).
-                        if (NT == 1) {
-                            ok = __all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(g - 1) & 1u,
-                                                            wc, kErrTimeout));
-                            if (!ok) break;
-                            tc_fence_after_sync();
-                        }
-#pragma unroll 1
-                        for (int c = 0; c < T::DV / 32; ++c) {
-                            uint32_t r[32];
-                            tmem_ld32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-                            tmem_st32(tl + T::O_COL0 + tt * T::DV + c * 32, r);
-                        }
-                    }
-                    const float neg_m = (m_ref[k] == -INFINITY) ? 0.f : -m_ref[k];
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ch = 0; ch < BN / 32; ++ch) {
-                        uint32_t pk[16];
-                        if ((skip >> ch) & 1u) {  // no row of this warp allows any key here
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) pk[c] = 0u;
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 16; ++c) {
-                                const int e = ch * 32 + 2 * c;
-                                float x0, x1;
-                                fma2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sl2,
-                                     neg_m, x0, x1);
-                                float p0, p1;
-                                if ((T::EXP_FMA_PAIRS >> (c & 7)) & 1u) {
-                                    exp2_fma_pair(x0, x1, p0, p1);
-                                } else {
-                                    p0 = ex2(x0);
-                                    p1 = ex2(x1);
-                                }
-                                add2(acc[(2 * c) & 3], acc[(2 * c + 1) & 3], p0, p1);
-                                if constexpr (T::FP8) {  // four E4M3 weights per column
-                                    const uint32_t h2 = pack_e4m3x2(p0, p1);
-                                    if (c & 1) pk[c >> 1] |= h2 << 16;
-                                    else pk[c >> 1] = h2;
-                                } else {
-                                    pk[c] = pack_bf16x2(p0, p1);
-                                }
-                            }
-                        }
-                        // P chunk ch (16 columns of bf16 pairs, or 8 of E4M3 quads) overwrites S
-                        // columns already read
-                        if constexpr (T::FP8) tmem_st8(s_col + ch * 8, pk);
-                        else tmem_st16(s_col + ch * 16, pk);
-                    }
-                    l[k] += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                    if ((EXT && j < mask_lo) || j >= mask_from)
+                        ok = softmax_block(true, sr, k, tt, j, g, s_col);
+                    else
+                        ok = softmax_block(false, sr, k, tt, j, g, s_col);
+                    if (!ok) break;
                     tmem_wait_st();
                     tc_fence_before_sync();
                     mbar_arrive(bar_p_full(sb));
-                    if (j == t.j_begin && pend) {
+                    if (j == j_begin && pend) {
                         // Tile tt of the previous unit, now that its successor's first P is out.
-                        ok = epilogue(pend_t, tt, pend_m[k], pend_l[k], pend_idx);
+                        ok = epilogue(pend_u, tt, pend_m[k], pend_l[k], pend_idx);
                         if (k == NTW - 1) pend = false;
                         if (!ok) break;
                     }
@@ -976,7 +1018,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             }
             if (!ok) break;
             pend = true;
-            pend_t = t;
+            pend_u = u;
 #pragma unroll
             for (int k = 0; k < NTW; ++k) {
                 pend_m[k] = m_ref[k];
@@ -987,7 +1029,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         }
         if (ok && pend)
             for (int k = 0; k < NTW && ok; ++k)
-                ok = epilogue(pend_t, tile_of(k), pend_m[k], pend_l[k], pend_idx);
+                ok = epilogue(pend_u, tile_of(k), pend_m[k], pend_l[k], pend_idx);
         // every O store this warp issued is complete before the CTA exits
         if (OTMA && lane == 0) bulk_wait_all();
     }

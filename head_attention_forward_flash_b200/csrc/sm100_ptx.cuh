@@ -93,6 +93,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     return mbar_wait_slow(bar, parity, w, code);
 }
 
+// One lane of the (fully active) warp returns true. Issuing a tcgen05 operation from an elected
+// lane of a warp that runs the surrounding loop uniformly keeps the operands warp-uniform, which
+// issues faster than a loop run by lane 0 alone (measured on B200: 43-49 vs 72 cycles per MMA
+// with softmax warps busy on the same SM sub-partition).
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), tile mode, no multicast
 // ------------------------------------------------------------------------------------------

@@ -3,9 +3,10 @@
 TEST INFRASTRUCTURE: a model of the kernel's design, not of the method; it shares no code with
 the CUDA library and the library never uses it.
 
-Roles (as in the kernel): one TMA producer, one MMA issuer, and the softmax warpgroups. These
-are either one warpgroup for every query tile (NSM = 1) or one warpgroup per tile (NSM = NT).
-The tensor core runs issued MMAs and commits in order. TMA loads land at random later times.
+Roles (as in the kernel): one TMA producer, one MMA issuer and one softmax warpgroup per
+query tile (one or two tiles per work unit).
+The tensor core runs each issuer's MMAs and commits in its issue order, interleaving issuers at
+random. TMA loads land at random later times.
 A random scheduler interleaves everything. mbarriers count arrivals and transaction bytes and
 complete phases; a wait on parity p passes once the phase with that parity has completed, as
 on the hardware.
@@ -29,7 +30,7 @@ import random
 
 MUTANTS = {
     "k_slot_reused_without_wait": "the producer refills a K slot without waiting for kempty",
-    "kempty_after_first_tile": "the MMA warp frees a K slot after tile 0 instead of the last tile",
+    "kempty_after_first_tile": "a K slot is freed by the first MMA issuer's commit alone",
     "no_o_free_wait": "the MMA warp starts a unit's first P V without waiting for o_free",
     "no_pv_done_wait": "with one tile, the softmax rescales O without waiting for bar_pv_done",
     "q_refill_without_wait": "the producer refills the Q staging buffer without waiting q_empty",
@@ -92,27 +93,33 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
     rnd = random.Random(seed)
     clock = [0]
     kfull = [Bar(1, f"kfull{i}", clock) for i in range(NK)]
-    kempty = [Bar(1, f"kempty{i}", clock) for i in range(NK)]
+    # one commit per MMA issuer (the planted mistake counts one)
+    kempty = [Bar(1 if mutant == "kempty_after_first_tile" else NT, f"kempty{i}", clock)
+              for i in range(NK)]
     vfull = [Bar(1, f"vfull{i}", clock) for i in range(NV)]
-    vempty = [Bar(1, f"vempty{i}", clock) for i in range(NV)]
+    vempty = [Bar(NT, f"vempty{i}", clock) for i in range(NV)]
     s_full = [Bar(1, "s_full0", clock), Bar(1, "s_full1", clock)]
     p_full = [Bar(128, "p_full0", clock), Bar(128, "p_full1", clock)]
     pv_done = Bar(1, "pv_done", clock)
     q_full = Bar(1, "q_full", clock)
-    q_empty = Bar(128 * NT if q_tmem else 1, "q_empty", clock)
+    q_empty = Bar(128 * NT if q_tmem else NT, "q_empty", clock)
     q_tmem_bar = [Bar(128, f"q_tmem{t}", clock) for t in range(NT)]
     o_full = [Bar(1, f"o_full{t}", clock) for t in range(NT)]
     o_free = [Bar(128, f"o_free{t}", clock) for t in range(NT)]
-    mma_done = Bar(1, "mma_done", clock)
+
+    mma_done = Bar(NT, "mma_done", clock)
 
     kslot = [None] * NK
     vslot = [None] * NV
     qstage = [None]
     qtm = {}            # tile -> unit whose Q is in tensor memory
-    sbuf = [None, None]  # score buffer -> ((unit, block, tile), 'S' | 'P' | 'consumed')
+    # score buffer -> per half ("lo": the columns P overwrites, "hi": the rest) the item and
+    # its state: 'S' (scores landed), 'read' (in the softmax's registers), 'P' (P written),
+    # 'consumed' (read by P V)
+    sbuf = [{"lo": None, "hi": None}, {"lo": None, "hi": None}]
     obuf = {}           # tile -> [unit, blocks accumulated, 'acc' | 'read']
     landings = []       # TMA loads in flight
-    tensor = []         # issued MMAs and commits, executed in order
+    tensor = []         # issued MMAs and commits: (issuer, kind, x); in order per issuer
     busy = [u for u in units if u["n"] > 0]
     current = [None]  # the role being stepped
     waits = {}        # role -> (barrier, parity, completed phases) it last blocked on
@@ -174,52 +181,65 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
         if pend and pend[2] == 0:
             yield from load_kv("v", pend[0], pend[1])
 
-    # ------------------------------ MMA issuer ------------------------------
-    def mma():
-        st = {"k": 0, "v": 0, "kslot": None, "vslot": None, "units": 0}
+    # ------------------------------ MMA issuers ------------------------------
+    # NT = 2: one issuer per query tile; its tile's chain is Q K^T(j), P V(j) once P(j) is out,
+    # then Q K^T(j+1) (one score buffer per tile). NT = 1: one issuer; the tile alternates
+    # between the two score buffers, so Q K^T(g+1) goes before P V(g).
+    def mma(tiles):
+        st = {"k": 0, "v": 0, "units": 0, "kslot": None}
+        me = tiles[0]
 
-        def qk(u, j, tt, g, last):
-            if q_tmem and j == 0:
-                yield from wait(q_tmem_bar[tt], st["units"] & 1)
-            if tt == 0:
-                s = st["k"] % NK
-                ph = (st["k"] // NK) & 1
-                st["k"] += 1
-                yield from wait(kfull[s], ph)
-                st["kslot"] = s
-            s = st["kslot"]
+        class Q:  # this issuer's view of the tensor queue
+            @staticmethod
+            def append(x):
+                tensor.append((me,) + x)
 
-            def op(s=s, item=(u["id"], j, tt), g=g):
+        def take_k():
+            s = st["k"] % NK
+            ph = (st["k"] // NK) & 1
+            st["k"] += 1
+            yield from wait(kfull[s], ph)
+            st["kslot"] = s
+
+        def qk_op(s, item, g, halves):
+            def op():
                 check(kslot[s] == item[:2], f"Q K^T {item} reads K {kslot[s]}")
                 q = qtm.get(item[2]) if q_tmem else qstage[0]
                 check(q == item[0], f"Q K^T {item} reads the Q of unit {q}")
-                check(sbuf[g & 1] is None or sbuf[g & 1][1] == "consumed",
-                      f"Q K^T {item} overwrites {sbuf[g & 1]}")
-                sbuf[g & 1] = (item, "S")
-            tensor.append(("op", op))
-            tensor.append(("commit", s_full[g & 1]))
-            if tt == (0 if mutant == "kempty_after_first_tile" else NT - 1):
-                tensor.append(("commit", kempty[s]))
+                b = sbuf[g & 1]
+                for h in halves:
+                    free = ("consumed",) if h == "lo" else ("read", "consumed")
+                    check(b[h] is None or b[h][1] in free, f"Q K^T {item} overwrites {h} {b[h]}")
+                    b[h] = (item, "S")
+            return op
+
+        def qk(u, j, tt, g, last):  # a whole Q K^T (both key halves)
+            if q_tmem and j == 0:
+                yield from wait(q_tmem_bar[tt], st["units"] & 1)
+            yield from take_k()
+            s = st["kslot"]
+            Q.append(("op", qk_op(s, (u["id"], j, tt), g, ("lo", "hi"))))
+            Q.append(("commit", s_full[g & 1]))
+            Q.append(("commit", kempty[s]))
             if not q_tmem and last:
-                tensor.append(("commit", q_empty))
+                Q.append(("commit", q_empty))
             yield True
 
         def pv(g, u, j, tt, last_block, uidx):
+            item = (u["id"], j, tt)
             yield from wait(p_full[g & 1], (g >> 1) & 1)
             if j == 0 and uidx > 0 and mutant != "no_o_free_wait":
                 yield from wait(o_free[tt], (uidx - 1) & 1)
-            if tt == 0:
-                s = st["v"] % NV
-                ph = (st["v"] // NV) & 1
-                st["v"] += 1
-                yield from wait(vfull[s], ph)
-                st["vslot"] = s
-            s = st["vslot"]
+            s = st["v"] % NV
+            ph = (st["v"] // NV) & 1
+            st["v"] += 1
+            yield from wait(vfull[s], ph)
 
-            def op(s=s, item=(u["id"], j, tt), g=g):
+            def op(s=s, item=item, g=g):
                 check(vslot[s] == item[:2], f"P V {item} reads V {vslot[s]}")
-                check(sbuf[g & 1] == (item, "P"), f"P V {item} reads {sbuf[g & 1]}")
-                sbuf[g & 1] = (item, "consumed")
+                lo = sbuf[g & 1]["lo"]
+                check(lo == (item, "P"), f"P V {item} reads {lo}")
+                sbuf[g & 1]["lo"] = (item, "consumed")
                 o = obuf.get(item[2])
                 if item[1] == 0:
                     check(o is None or o[2] == "read", f"P V {item} overwrites unread O {o}")
@@ -227,31 +247,36 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
                 else:
                     check(o[0] == item[0] and o[1] == item[1], f"P V {item} finds O {o}")
                     o[1] += 1
-            tensor.append(("op", op))
+            Q.append(("op", op))
             if NT == 1:
-                tensor.append(("commit", pv_done))
-            if tt == NT - 1:
-                tensor.append(("commit", vempty[s]))
+                Q.append(("commit", pv_done))
+            Q.append(("commit", vempty[s]))
             if last_block:
-                tensor.append(("commit", o_full[tt]))
+                Q.append(("commit", o_full[tt]))
             yield True
 
         pend = None
-        g = 0
+        jg = 0
         for u in busy:
             if not q_tmem:
                 yield from wait(q_full, st["units"] & 1)
             for j in range(u["n"]):
-                for tt in range(NT):
-                    yield from qk(u, j, tt, g, j == u["n"] - 1 and tt == NT - 1)
-                    if pend:
-                        yield from pv(*pend)
-                    pend = (g, u, j, tt, j == u["n"] - 1, st["units"])
-                    g += 1
+                last = j == u["n"] - 1
+                for tt in tiles:
+                    g = jg * NT + tt
+                    if NT == 2:
+                        yield from qk(u, j, tt, g, last)
+                        yield from pv(g, u, j, tt, last, st["units"])
+                    else:
+                        yield from qk(u, j, tt, g, last)
+                        if pend:
+                            yield from pv(*pend)
+                        pend = (g, u, j, tt, last, st["units"])
+                jg += 1
             st["units"] += 1
         if pend:
             yield from pv(*pend)
-        tensor.append(("commit", mma_done))
+        Q.append(("commit", mma_done))
         yield True
 
     # ------------------------ softmax + epilogue warpgroups ------------------------
@@ -286,25 +311,33 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
                 for tt in tiles:
                     g = jg * NT + tt
                     sb = g & 1
+                    item = (u["id"], j, tt)
+                    if NT == 2:  # the two tiles' softmax take turns, block by block
+                        if tt == 1:
+                            yield from wait(p_full[0], jg & 1)
+                        elif jg > 0:
+                            yield from wait(p_full[1], (jg - 1) & 1)
                     parity = ((g >> 1) & 1) ^ (1 if mutant == "s_full_wrong_parity" else 0)
                     yield from wait(s_full[sb], parity)
                     if q_tmem and j == u["n"] - 1 and nxt:
                         yield from copy_q(ui + 1, tt, nxt["id"])
-                    check(sbuf[sb] == ((u["id"], j, tt), "S"),
-                          f"softmax of {(u['id'], j, tt)} reads {sbuf[sb]}")
+                    b = sbuf[sb]
+                    check(b["lo"] == (item, "S") and b["hi"] == (item, "S"),
+                          f"softmax of {item} reads {b}")
+                    b["lo"], b["hi"] = (item, "read"), (item, "read")
                     if j > 0 and rnd.random() < 0.3:  # the running max grew: rescale O
                         if NT == 1 and mutant != "no_pv_done_wait":
                             yield from wait(pv_done, (g - 1) & 1)
                         o = obuf.get(tt)
                         check(o is not None and o[0] == u["id"] and o[1] == j,
-                              f"rescale of {(u['id'], j, tt)} finds O {o}")
+                              f"rescale of {item} finds O {o}")
                     if mutant == "p_full_early":
                         p_full[sb].arrive(128)
                         yield True
-                        sbuf[sb] = ((u["id"], j, tt), "P")
+                        b["lo"] = (item, "P")
                     else:
                         yield True
-                        sbuf[sb] = ((u["id"], j, tt), "P")
+                        b["lo"] = (item, "P")
                         p_full[sb].arrive(128)
                     if j == 0 and pend:
                         yield from epilogue(pend[0], tt, pend[1])
@@ -314,7 +347,9 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             for tt in tiles:
                 yield from epilogue(pend[0], tt, pend[1])
 
-    roles = {"tma": producer(), "mma": mma()}
+    roles = {"tma": producer()}
+    for t in range(NT):  # one MMA issuer per query tile
+        roles[f"mma{t}"] = mma([t])
     if NSM == 1:
         roles["softmax"] = softmax(list(range(NT)))
     else:
@@ -334,7 +369,10 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             landings.pop(rnd.randrange(len(landings)) if rnd.random() < 0.3 else 0)()
             blocked.clear()
         elif c == "tensor":
-            kind, x = tensor.pop(0)
+            # the next operation of a random issuer (in issue order within each issuer)
+            issuer = rnd.choice(sorted({e[0] for e in tensor}))
+            idx = next(i for i, e in enumerate(tensor) if e[0] == issuer)
+            _, kind, x = tensor.pop(idx)
             x() if kind == "op" else x.arrive(1)
             blocked.clear()
         else:
@@ -352,7 +390,7 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
                 blocked.clear()
             else:
                 blocked.add(c)
-    check(mma_done.completed == 1, "MMAs not drained")
+    check(mma_done.completed == 1, "MMAs not drained")  # every issuer committed once
     return steps
 
 
@@ -360,8 +398,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
 # csrc/attn_api.cu (d64 dense, d64 packed, d128, d192/128, d256, E4M3 d128) plus ring-depth edge
 # cases (a single slot).
 LAYOUTS = [(2, 2, True, 5, 5), (1, 1, True, 6, 6), (2, 2, False, 3, 2), (2, 2, False, 2, 1),
-           (1, 1, True, 2, 2), (2, 2, False, 4, 4), (2, 1, True, 2, 2), (2, 2, True, 1, 1),
-           (1, 1, False, 1, 1)]
+           (1, 1, True, 2, 2), (2, 2, False, 4, 4), (2, 2, True, 1, 1), (1, 1, False, 1, 1),
+           (2, 2, False, 1, 1)]
 
 
 def random_units(rnd):

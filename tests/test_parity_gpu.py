@@ -14,7 +14,8 @@ import torch
 
 import oracle
 from libutil import ensure_built
-from workloads import HEAD_DIMS, bf16_bits, config, config_inputs, make_inputs, sample_rows
+from workloads import (HEAD_DIMS, bf16_bits, config, config_inputs, make_inputs, sample_rows,
+                       tile_edge_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -111,7 +112,10 @@ def test_config1_matches_stored_oracle_values(b2):
         assert abs(lse[bi, h, i] - g["lse"][n]) <= TOL_LSE
 
 
-def _sampled(b2, n, n_pos):
+def _sampled(b2, n, n_pos, edges=False):
+    """Workload n at full size on the GPU; the oracle on n_pos sampled query positions of every
+    (batch, head), plus (edges) the first and last row of every 128-row query tile, so that a
+    work unit the scheduler dropped or misplaced cannot escape."""
     c = config(n)
     q, k, v = config_inputs(c)
     kk = k
@@ -130,6 +134,8 @@ def _sampled(b2, n, n_pos):
         o, lse = b2.attn_fwd(q.to(dev), k.to(dev), v.to(dev), causal=c["causal"], scale=c["scale"])
     torch.cuda.synchronize()
     rows = sample_rows(c, n_pos).numpy()
+    if edges:
+        rows = np.unique(np.concatenate([rows, tile_edge_rows(c).numpy()]), axis=0)
     o_ref, lse_ref = oracle.attn_rows(bf16_bits(q), kk_ref, bf16_bits(v), c["b"], c["hq"], c["hk"],
                                       c["sq"], c["sk"], c["dqk"], c["dv"], c["causal"], c["scale"],
                                       rows)
@@ -147,6 +153,21 @@ def _sampled(b2, n, n_pos):
 @pytest.mark.parametrize("n,n_pos", [(2, 16), (3, 12), (4, 48), (5, 256)])
 def test_full_size_configs_sampled_rows(b2, n, n_pos):
     _sampled(b2, n, n_pos)
+
+
+@pytest.mark.parametrize("n", [3, 4, 5])
+def test_full_size_every_query_tile(b2, n):
+    """Full-size workloads with the first and last row of every query tile of every head checked
+    against the oracle (the scheduler's unit orders at the real geometry: head-major for the
+    many-head workload, weight-major for the five-head one)."""
+    _sampled(b2, n, 8, edges=True)
+
+
+def test_config2_every_row(b2):
+    """The b8 hq48:hk8 2048^2 d64 causal workload compared with the oracle on every output row."""
+    c = config(2)
+    check_full(b2, c["b"], c["hq"], c["hk"], c["sq"], c["sk"], c["dqk"], c["dv"], c["causal"],
+               c["scale"], c["seed"])
 
 
 def test_k_mean_and_sub_match_oracle(b2):

@@ -172,6 +172,16 @@ def sample_rows(c: dict, n_pos: int = 256) -> torch.Tensor:
     return torch.tensor(rows, dtype=torch.int64)
 
 
+def tile_edge_rows(c: dict, tile: int = 128) -> torch.Tensor:
+    """Every (batch, head) pair at the first and the last query row of every ``tile``-row query
+    tile, as int64 (batch, head, query) triples: each work unit of the attention kernel (one or
+    two 128-row tiles of one (batch, head)) then contributes its first and last row."""
+    sq = c["sq"]
+    pos = sorted({p for t in range(0, sq, tile) for p in (t, min(t + tile - 1, sq - 1))})
+    rows = [(bi, h, i) for bi in range(c["b"]) for h in range(c["hq"]) for i in pos]
+    return torch.tensor(rows, dtype=torch.int64)
+
+
 def bf16_bits(t: torch.Tensor):
     """The raw bf16 bit patterns of ``t`` as a contiguous numpy uint16 array."""
     import numpy as np
