@@ -245,18 +245,22 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 
 // Head-dim table: (dqk, dv) -> <DQK, DV, keys per block, query tiles per unit, softmax
 // warpgroups, Q in TMEM, K slots, V slots, score pairs whose exp2 runs on the FMA pipe, E4M3
-// inputs>. Tensor
-// memory holds two score buffers, one O per query tile and (when it fits) each tile's Q; shared
-// memory holds the Q staging buffer and the K / V rings. The (tiles, warpgroups) choice per head
-// dim is the measured fastest on B200 (d64: two tiles and two warpgroups, except for packed
-// sequences). The share of score pairs whose exp2 runs on the FMA pipe is the measured best per
-// head dim (3 of 8 at d64, 2 of 8 at d128 / d192 and for E4M3 inputs, none at d256, which is
-// bound by the tensor core).
-using T64 = AttnTraits<64, 64, 128, 2, 2, true, 5, 5, 0x92u>;   // smem 32 + 80 + 80 (+32) KB
-using T64V = AttnTraits<64, 64, 128, 1, 1, true, 6, 6, 0x92u>;  // smem 16 + 96 + 96 (+16) KB
-using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;   // smem 64 + 96 + 64 KB
-using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;   // smem 96 + 96 + 32 KB
-using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;     // smem 64 + 64 + 64 KB
+// inputs, pipelined two-tile layout>. Shared memory holds the Q staging buffer and the K / V
+// rings (and, when it fits, the O staging tile). Measured on B200 (TFLOP/s, causal-halved):
+//  - d64: the pipelined layout (two 64-key score buffers per tile, the two tiles' softmax side
+//    by side): b8 hq48:hk8 2048^2 causal 501 vs 455 with one 128-key buffer per tile; 8192^2
+//    with a 128-key window and sinks 119 vs 80.
+//  - d128, d192/128: one 128-key score buffer per tile, the tiles' softmax taking turns (the
+//    pipelined layout's 64-key Q K^T from shared memory runs at 2/3 of the tensor rate: 1027 vs
+//    1041 at 65536^2 d128, 996 vs 1021 at 8192^2 d192/128).
+//  - d256: one tile, two 64-key score buffers.
+// The share of score pairs whose exp2 runs on the FMA pipe is the measured best per head dim
+// (3 of 8 at d64, 2 of 8 at d128 / d192 and for E4M3 inputs, none at d256, bound by the tensor
+// core).
+using T64P = AttnTraits<64, 64, 64, 2, 2, true, 8, 8, 0x92u, false, true>;  // 32 + 64 + 64 (+32) KB
+using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;         // 64 + 96 + 64 KB
+using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;         // 96 + 96 + 32 KB
+using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;                  // 64 + 64 + 64 KB
 // E4M3 inputs, (128, 128): the d128 layout with half-size tiles, so four K and four V slots fit
 // next to the Q staging buffer and the O staging tile.
 using T128F8 = AttnTraits<128, 128, 128, 2, 2, false, 4, 4, 0x11u, true>;  // 32 + 64 + 64 (+64) KB
@@ -282,22 +286,22 @@ int dispatch_varlen(int causal, const void* q, const void* k, const void* v, voi
                   : launch_attn<T, false, true, false>(q, k, v, out, lse, sh, scale, st);
 }
 
-// d64 packed sequences use the one-warpgroup layout (measured faster there: 310 vs 278 TFLOP/s
-// on 8 sequences of 1024-2048; the two-tile layout is faster for dense and windowed d64).
+// Packed sequences take the dense layouts (equal-length packed input is then bitwise the dense
+// result).
 int dispatch_dims(int64_t dqk, int causal, bool varlen, const void* q, const void* k,
                   const void* v, void* out, float* lse, const Shape& sh, float scale,
                   cudaStream_t st)
 {
     if (varlen) {
         switch (dqk) {
-        case 64: return dispatch_varlen<T64V>(causal, q, k, v, out, lse, sh, scale, st);
+        case 64: return dispatch_varlen<T64P>(causal, q, k, v, out, lse, sh, scale, st);
         case 128: return dispatch_varlen<T128>(causal, q, k, v, out, lse, sh, scale, st);
         case 192: return dispatch_varlen<T192>(causal, q, k, v, out, lse, sh, scale, st);
         default: return dispatch_varlen<T256>(causal, q, k, v, out, lse, sh, scale, st);
         }
     }
     switch (dqk) {
-    case 64: return dispatch_dense<T64>(causal, q, k, v, out, lse, sh, scale, st);
+    case 64: return dispatch_dense<T64P>(causal, q, k, v, out, lse, sh, scale, st);
     case 128: return dispatch_dense<T128>(causal, q, k, v, out, lse, sh, scale, st);
     case 192: return dispatch_dense<T192>(causal, q, k, v, out, lse, sh, scale, st);
     default: return dispatch_dense<T256>(causal, q, k, v, out, lse, sh, scale, st);

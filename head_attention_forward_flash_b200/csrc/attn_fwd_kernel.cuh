@@ -98,7 +98,7 @@ struct AttnParams {
 };
 
 template <int DQK_, int DV_, int BN_, int NT_, int NSM_, bool Q_TMEM_, int NK_, int NV_,
-          uint32_t EXP_FMA_PAIRS_ = 0, bool FP8_ = false>
+          uint32_t EXP_FMA_PAIRS_ = 0, bool FP8_ = false, bool PIPE_ = false>
 struct AttnTraits {
     static constexpr int DQK = DQK_;
     static constexpr int DV = DV_;
@@ -124,11 +124,19 @@ struct AttnTraits {
     static constexpr uint32_t V_TILE_BYTES = BN * DV * EB;
     static_assert(!FP8 || (!Q_TMEM && (DQK * EB) % 128 == 0 && (DV * EB) % 128 == 0),
                   "E4M3 inputs: Q from shared memory, whole 128-byte row chunks");
+    // PIPE (two tiles): every tile owns two score buffers and runs its own pipelined MMA order,
+    // Q K^T of block j+1 before P V of block j, so the tensor core computes a tile's next S while
+    // its softmax works on the current one and the two tiles' softmax run side by side. Without
+    // PIPE two tiles share the two score buffers (one each), and NT = 1 alternates between them.
+    static constexpr bool PIPE = PIPE_;
+    static_assert(!PIPE || NT == 2, "");
+    static constexpr int NSBUF = PIPE ? 2 * NT : 2;  // score buffers
     // tensor memory columns
-    static constexpr uint32_t O_COL0 = 2 * BN;
-    static constexpr uint32_t Q_COL0 = 2 * BN + NT * DV;
+    static constexpr uint32_t O_COL0 = NSBUF * BN;
+    static constexpr uint32_t Q_COL0 = NSBUF * BN + NT * DV;
     static constexpr uint32_t TMEM_COLS = 512;
-    static_assert(2 * BN + NT * DV + (Q_TMEM ? NT * DQK / 2 : 0) <= 512, "tensor memory budget");
+    static_assert(NSBUF * BN + NT * DV + (Q_TMEM ? NT * DQK / 2 : 0) <= 512,
+                  "tensor memory budget");
     static_assert(DQK % 64 == 0 && DV % 64 == 0 && BN % 64 == 0 && BN <= 256 && DV <= 256, "");
     static_assert(NT == 1 || NT == 2, "");
     // shared memory: [Q staging][K slots][V slots][O staging, if used][barriers][TMEM base,
@@ -136,7 +144,7 @@ struct AttnTraits {
     static constexpr uint32_t K_OFF = Q_BYTES;
     static constexpr uint32_t V_OFF = K_OFF + NK * K_TILE_BYTES;
     static constexpr uint32_t O_OFF = V_OFF + NV * V_TILE_BYTES;
-    static constexpr int NBAR = 2 * NK + 2 * NV + 8 + 3 * NT;
+    static constexpr int NBAR = 2 * NK + 2 * NV + 2 * NSBUF + 3 + 4 * NT;
     // The epilogue writes O through a shared-memory tile and TMA stores (one per warp and
     // 64-column box: slab o_slab(tile, box, warp % 4), 32 rows x 128 bytes) when the tiles fit
     // next to the rings; otherwise each thread stores its own row.
@@ -150,15 +158,21 @@ struct AttnTraits {
     static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(NSM == NT, "one softmax warpgroup per query tile (and one MMA issuer each)");
-    // Threads: NSM softmax warpgroups, then the MMA warp and the TMA warp. With two softmax
-    // warpgroups the block is three full warpgroups (two warps idle) so that registers can
-    // move between them: at launch every thread has LAUNCH_REGS (the cap for 384 threads);
-    // the third warpgroup drops to AUX_REGS and the softmax warpgroups rise to SOFTMAX_REGS,
-    // which keeps the block's total unchanged (a larger total would never be granted).
+    // Threads. One softmax warpgroup: warps 0-3 softmax, warp 4 MMA issuer, warp 5 TMA producer.
+    // Two: warpgroup 0 holds the MMA issuers (warps 0 and 2) and the TMA producer (warp 1; warp
+    // 3 idles), warpgroups 1 and 2 the softmax of tiles 0 and 1. The block is three full
+    // warpgroups so that registers can move between them: at launch every thread has
+    // LAUNCH_REGS (the cap for 384 threads); the issuers' warpgroup drops to AUX_REGS and the
+    // softmax warpgroups rise to SOFTMAX_REGS, which keeps the block's total unchanged (a larger
+    // total would never be granted). The issuers come first: the warp schedulers favour older
+    // warps, and an issuer that waits for issue slots behind two busy softmax warps on its SM
+    // sub-partition delays its tile's next S (measured on B200).
     static constexpr int NUM_THREADS = NSM == 1 ? 192 : 384;
-    static constexpr int MMA_WARP = 4 * NSM;       // MMA issuer (tile 0, or every tile when NT = 1)
-    static constexpr int TMA_WARP = 4 * NSM + 1;
-    static constexpr int MMA_WARP2 = 4 * NSM + 2;  // NT = 2: issuer of tile 1's MMAs
+    static constexpr int AUX_WG = NSM == 1 ? 1 : 0;  // the warpgroup of the MMA and TMA warps
+    static constexpr int SM_WG0 = NSM == 1 ? 0 : 1;  // the first softmax warpgroup
+    static constexpr int MMA_WARP = 4 * AUX_WG;      // MMA issuer (tile 0, or every tile when NT = 1)
+    static constexpr int TMA_WARP = 4 * AUX_WG + 1;
+    static constexpr int MMA_WARP2 = 4 * AUX_WG + 2; // NT = 2: issuer of tile 1's MMAs
     static constexpr int LAUNCH_REGS = 168;
     static constexpr int SOFTMAX_REGS = 224;
     static constexpr int AUX_REGS = 56;
@@ -362,16 +376,27 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     auto bar_vfull = [&](int s) { return bar(2 * NK + s); };
     auto bar_vempty = [&](int s) { return bar(2 * NK + NV + s); };
     constexpr int B0 = 2 * NK + 2 * NV;
+    constexpr int NSB = T::NSBUF;
     auto bar_s_full = [&](int s) { return bar(B0 + s); };
-    auto bar_p_full = [&](int s) { return bar(B0 + 2 + s); };
-    const uint32_t bar_pv_done = bar(B0 + 4);
-    const uint32_t bar_q_full = bar(B0 + 5);
-    const uint32_t bar_q_empty = bar(B0 + 6);
-    const uint32_t bar_mma_done = bar(B0 + 7);
+    auto bar_p_full = [&](int s) { return bar(B0 + NSB + s); };
+    // per tile: its last P V is complete (NT = 1 and PIPE, where S(j+1) lands before P V(j))
+    auto bar_pv_done = [&](int t) { return bar(B0 + 2 * NSB + t); };
+    const uint32_t bar_q_full = bar(B0 + 2 * NSB + NT);
+    const uint32_t bar_q_empty = bar(B0 + 2 * NSB + NT + 1);
+    const uint32_t bar_mma_done = bar(B0 + 2 * NSB + NT + 2);
+    constexpr int B1 = B0 + 2 * NSB + NT + 3;
     // per query tile: its Q is in TMEM / its O is final / its O has been read out
-    auto bar_q_tmem = [&](int t) { return bar(B0 + 8 + t); };
-    auto bar_o_full = [&](int t) { return bar(B0 + 8 + NT + t); };
-    auto bar_o_free = [&](int t) { return bar(B0 + 8 + 2 * NT + t); };
+    auto bar_q_tmem = [&](int t) { return bar(B1 + t); };
+    auto bar_o_full = [&](int t) { return bar(B1 + NT + t); };
+    auto bar_o_free = [&](int t) { return bar(B1 + 2 * NT + t); };
+    // Score buffer of tile tt's key block number jg (counted over all units), and the parity of
+    // the phase of that buffer's barriers the block completes.
+    auto sbuf_of = [&](int64_t jg, int tt) -> int {
+        return T::PIPE ? tt * 2 + (int)(jg & 1) : (NT == 2 ? tt : (int)(jg & 1));
+    };
+    auto sphase_of = [&](int64_t jg) -> uint32_t {
+        return (T::PIPE || NT == 1) ? (uint32_t)(jg >> 1) & 1u : (uint32_t)jg & 1u;
+    };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -385,11 +410,11 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             mbar_init(bar_vfull(s), 1);
             mbar_init(bar_vempty(s), NT);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSB; ++s) {
             mbar_init(bar_s_full(s), 1);
             mbar_init(bar_p_full(s), 128);  // one warpgroup writes each P
         }
-        mbar_init(bar_pv_done, 1);
+        for (int t = 0; t < NT; ++t) mbar_init(bar_pv_done(t), 1);
         mbar_init(bar_q_full, 1);
         // per-tile copy-out (Q in TMEM) / each issuer's last Q K^T of the unit
         mbar_init(bar_q_empty, T::Q_TMEM ? 128 * NT : NT);
@@ -441,7 +466,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     };
 
     if constexpr (T::NSM == 2) {
-        if (warp >= T::MMA_WARP) setmaxnreg_dec<T::AUX_REGS>();  // registers to the softmax
+        if ((warp >> 2) == T::AUX_WG) setmaxnreg_dec<T::AUX_REGS>();  // registers to the softmax
     }
     if (warp == T::TMA_WARP) {
         // ------------------------------ TMA producer ------------------------------
@@ -504,8 +529,10 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, unit_of(r));
                 const int64_t rn = busy_from(r + 1);
                 const int64_t un = rn >= 0 ? unit_of(rn) : -1;
+                // PIPE: each tile's issuer takes K(j+1) before V(j), as with one tile
+                constexpr int NTP = T::PIPE ? 1 : NT;
                 for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
-                    for (int tt = 0; tt < NT && ok; ++tt) {
+                    for (int tt = 0; tt < NTP && ok; ++tt) {
                         if (tt == 0) load_k(t, j);  // the Q K^T step of item (j, tt)
                         if (ok && T::Q_TMEM && j == t.j_begin && tt == 0 && un >= 0)
                             load_q(un);  // the staging buffer was emptied into TMEM
@@ -555,9 +582,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             auto wait_all = [&](uint32_t bar, uint32_t parity) {
                 return __all_sync(FULL, mbar_wait(bar, parity, wc, kErrTimeout));
             };
-            // Q K^T of item g = (block, tile tt) of the current unit. Every issuer takes K(j)
+            // Q K^T of tile tt's current block into score buffer sb. Every issuer takes K(j)
             // itself: the slot is freed when all NT issuers have committed kempty.
-            auto qk = [&](int64_t g, bool first, int tt, bool last_item) {
+            auto qk = [&](int sb, bool first, int tt, bool last_item) {
                 if (T::Q_TMEM && first) {  // this tile's Q of the new unit must be in TMEM
                     if (!wait_all(bar_q_tmem(tt), (uint32_t)(units & 1))) {
                         ok = false;
@@ -573,19 +600,20 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     return;
                 }
                 if (elect_one()) {
-                    issue_qk_mmas<T>(tmem + (uint32_t)(g & 1) * BN,
+                    issue_qk_mmas<T>(tmem + (uint32_t)sb * BN,
                                      T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
                                                : q_stage + tt * T::Q_TILE_BYTES,
                                      k_slots + kslot * T::K_TILE_BYTES, p.idesc_qk);
-                    tc_commit(bar_s_full(g & 1));
+                    tc_commit(bar_s_full(sb));
                     tc_commit(bar_kempty(kslot));
                     if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
                 }
                 __syncwarp();
             };
-            // P V of item g = (block, tile tt) of busy unit number uidx.
-            auto pv = [&](int64_t g, bool first, int tt, bool last_block, int uidx) {
-                if (!wait_all(bar_p_full(g & 1), (uint32_t)(g >> 1) & 1u)) {
+            // P V of tile tt's block whose P is in score buffer sb (phase ph), of busy unit
+            // number uidx.
+            auto pv = [&](int sb, uint32_t ph, bool first, int tt, bool last_block, int uidx) {
+                if (!wait_all(bar_p_full(sb), ph)) {
                     ok = false;
                     return;
                 }
@@ -602,19 +630,20 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     return;
                 }
                 if (elect_one()) {
-                    issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)(g & 1) * BN,
+                    issue_pv_mmas<T>(tmem + T::O_COL0 + tt * T::DV, tmem + (uint32_t)sb * BN,
                                      v_slots + vslot * T::V_TILE_BYTES, !first);
-                    if (NT == 1) tc_commit(bar_pv_done);
+                    if (NT == 1 || T::PIPE) tc_commit(bar_pv_done(tt));
                     tc_commit(bar_vempty(vslot));
                     if (last_block) tc_commit(bar_o_full(tt));
                 }
                 __syncwarp();
             };
-            // NT = 1: the P V of each item is issued after the next item's Q K^T (also across
-            // units), so the tensor core computes the next S while the softmax works on this one.
+            // NT = 1 and PIPE: the P V of each block is issued after the next block's Q K^T (also
+            // across units), so the tensor core computes the next S while the softmax works on
+            // this one.
             bool pend = false, pend_last = false, pend_first = false;
-            int pend_u = 0;
-            int64_t pend_g = 0;
+            int pend_u = 0, pend_sb = 0;
+            uint32_t pend_ph = 0;
             for (int64_t r = 0; ok; ++r) {
                 const int64_t u = unit_of(r);
                 if (u < 0) break;
@@ -629,16 +658,17 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 for (int j = t.j_begin; j < t.n_blocks && ok; ++j, ++jg) {
                     const bool first = j == t.j_begin, last = j == t.n_blocks - 1;
-                    if constexpr (NT == 2) {
-                        const int64_t g = jg * 2 + my_tt;
-                        qk(g, first, my_tt, last);
-                        if (ok) pv(g, first, my_tt, last, units);
+                    if constexpr (NT == 2 && !T::PIPE) {
+                        qk(my_tt, first, my_tt, last);
+                        if (ok) pv(my_tt, (uint32_t)jg & 1u, first, my_tt, last, units);
                     } else {
-                        qk(jg, first, 0, last);
+                        const int tt = T::PIPE ? my_tt : 0;
+                        qk(sbuf_of(jg, tt), first, tt, last);
                         if (!ok) break;
-                        if (pend) pv(pend_g, pend_first, 0, pend_last, pend_u);
+                        if (pend) pv(pend_sb, pend_ph, pend_first, tt, pend_last, pend_u);
                         pend = true;
-                        pend_g = jg;
+                        pend_sb = sbuf_of(jg, tt);
+                        pend_ph = sphase_of(jg);
                         pend_first = first;
                         pend_last = last;
                         pend_u = units;
@@ -646,20 +676,21 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 ++units;
             }
-            if (NT == 1 && ok && pend) pv(pend_g, pend_first, 0, pend_last, pend_u);
+            if ((NT == 1 || T::PIPE) && ok && pend)
+                pv(pend_sb, pend_ph, pend_first, T::PIPE ? my_tt : 0, pend_last, pend_u);
             // drain every MMA this warp issued before teardown
             if (elect_one()) tc_commit(bar_mma_done);
             __syncwarp();
             mbar_wait_drain(bar_mma_done, 0, p.timeout_ns, p.status);
         }
-    } else if (warp < T::MMA_WARP) {
-        // ---------------- softmax + epilogue warpgroups (warps 0 .. 4*NSM-1) ----------------
+    } else if ((warp >> 2) != T::AUX_WG) {
+        // ------ softmax + epilogue warpgroups (warps 0-3 with one, 4-11 with two warpgroups) ------
         // NSM = 1: the warpgroup takes every query tile's items in order. NSM = 2: warpgroup w
         // takes the items of query tile w. Either way each thread keeps its whole score row of
         // the current item in registers (one TMEM read, a single pass).
         if constexpr (T::NSM == 2) setmaxnreg_inc<T::SOFTMAX_REGS>();
         constexpr int NTW = T::NSM == 1 ? NT : 1;  // query tiles this warpgroup handles
-        const int wg = warp >> 2;
+        const int wg = (warp >> 2) - T::SM_WG0;
         const int w4 = warp & 3;                  // TMEM lanes 32*w4 .. 32*w4+31
         const int row = threadIdx.x & 127;        // TMEM lane = row of the query tile
         const uint32_t tl = tmem + ((uint32_t)(w4 * 32) << 16);
@@ -790,7 +821,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         float l[NTW] = {};      // sum of exp2(x - m_ref) over the keys seen so far
         int j_begin = 0;
         auto softmax_block = [&](const bool MASKED, uint32_t(&sr)[BN], int k, int tt, int j,
-                                 int64_t g, uint32_t s_col) -> bool {
+                                 int64_t jgb, uint32_t s_col) -> bool {
             // Keys j*BN + c with lor <= c <= rel are allowed. Per 32-key chunk the warp takes
             // one of three uniform paths: every row of the warp allows the whole chunk
             // (nothing to do), none allows any of it (skipped below: no max, P = 0 without
@@ -848,13 +879,14 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             }
             if (j > j_begin && __any_sync(FULL, need)) {
                 // O holds blocks < j of this tile: scale it in place once its last P V is
-                // complete. With two tiles that P V was issued by this tile's issuer before this
-                // item's Q K^T, so it is complete now that S has landed (a commit covers all
-                // earlier MMAs of its thread). With one tile it is item g-1, issued after this
-                // item's Q K^T: wait for it (bar_pv_done is then in phase g-1 or g, so the
-                // parity test on phase g-1 is unambiguous).
-                if (NT == 1) {
-                    if (!__all_sync(FULL, mbar_wait(bar_pv_done, (uint32_t)(g - 1) & 1u, wc,
+                // complete. With two tiles sharing the score buffers that P V was issued by this
+                // tile's issuer before this block's Q K^T, so it is complete now that S has
+                // landed (a commit covers all earlier MMAs of its thread). With one tile, or with
+                // PIPE, it was issued after this block's Q K^T: wait for it on the tile's
+                // bar_pv_done (one phase per block; that barrier is then in the phase of block
+                // jg-1 or jg, so the parity test on jg-1 is unambiguous).
+                if (NT == 1 || T::PIPE) {
+                    if (!__all_sync(FULL, mbar_wait(bar_pv_done(tt), (uint32_t)(jgb - 1) & 1u, wc,
                                                     kErrTimeout)))
                         return false;
                     tc_fence_after_sync();
@@ -969,10 +1001,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < NTW; ++k) {
                     const int tt = tile_of(k);
-                    const int64_t g = jg * NT + tt;  // global item number
-                    const int sb = (int)(g & 1);     // score buffer
+                    const int sb = sbuf_of(jg, tt);  // score buffer
                     const uint32_t s_col = tl + sb * BN;
-                    if (NT == 2 && p.alt) {
+                    if (NT == 2 && !T::PIPE && p.alt) {
                         // The two tiles' softmax take turns: tile 1's block jg after tile 0's,
                         // tile 0's block jg after tile 1's block jg-1 (p_full of the other tile
                         // completes once per block, and cannot run a phase ahead of this wait).
@@ -985,7 +1016,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         ok = __all_sync(FULL, w);
                         if (!ok) break;
                     }
-                    ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), (uint32_t)(g >> 1) & 1u, wc,
+                    ok = __all_sync(FULL, mbar_wait(bar_s_full(sb), sphase_of(jg), wc,
                                                     kErrTimeout));
                     if (!ok) break;
                     tc_fence_after_sync();
@@ -1001,9 +1032,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                         tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                     tmem_wait_ld();
                     if ((EXT && j < mask_lo) || j >= mask_from)
-                        ok = softmax_block(true, sr, k, tt, j, g, s_col);
+                        ok = softmax_block(true, sr, k, tt, j, jg, s_col);
                     else
-                        ok = softmax_block(false, sr, k, tt, j, g, s_col);
+                        ok = softmax_block(false, sr, k, tt, j, jg, s_col);
                     if (!ok) break;
                     tmem_wait_st();
                     tc_fence_before_sync();

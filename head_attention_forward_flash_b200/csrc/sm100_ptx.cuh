@@ -93,6 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
     return mbar_wait_slow(bar, parity, w, code);
 }
 
+
 // One lane of the (fully active) warp returns true. Issuing a tcgen05 operation from an elected
 // lane of a warp that runs the surrounding loop uniformly keeps the operands warp-uniform, which
 // issues faster than a loop run by lane 0 alone (measured on B200: 43-49 vs 72 cycles per MMA

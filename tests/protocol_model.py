@@ -32,7 +32,8 @@ MUTANTS = {
     "k_slot_reused_without_wait": "the producer refills a K slot without waiting for kempty",
     "kempty_after_first_tile": "a K slot is freed by the first MMA issuer's commit alone",
     "no_o_free_wait": "the MMA warp starts a unit's first P V without waiting for o_free",
-    "no_pv_done_wait": "with one tile, the softmax rescales O without waiting for bar_pv_done",
+    "no_pv_done_wait": "where S(j+1) can land before P V(j) (one tile, or the pipelined two-tile "
+                       "layout), the softmax rescales O without waiting for its bar_pv_done",
     "q_refill_without_wait": "the producer refills the Q staging buffer without waiting q_empty",
     "s_full_wrong_parity": "the softmax waits for the wrong phase of its score buffer",
     "p_full_early": "the softmax hands over P before writing it",
@@ -88,7 +89,7 @@ class Bar:
         return (self.completed & 1) != parity
 
 
-def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
+def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
     """One random schedule over `units` (dicts with 'id' and 'n' = key blocks, 0 = skipped)."""
     rnd = random.Random(seed)
     clock = [0]
@@ -98,9 +99,19 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
               for i in range(NK)]
     vfull = [Bar(1, f"vfull{i}", clock) for i in range(NV)]
     vempty = [Bar(NT, f"vempty{i}", clock) for i in range(NV)]
-    s_full = [Bar(1, "s_full0", clock), Bar(1, "s_full1", clock)]
-    p_full = [Bar(128, "p_full0", clock), Bar(128, "p_full1", clock)]
-    pv_done = Bar(1, "pv_done", clock)
+    # pipe (two tiles): each tile owns two score buffers and pipelines its own MMAs (Q K^T of
+    # block j+1 before P V of block j); otherwise two tiles own one buffer each and take turns,
+    # and one tile alternates between the two buffers
+    nsbuf = 2 * NT if pipe else 2
+    s_full = [Bar(1, f"s_full{i}", clock) for i in range(nsbuf)]
+    p_full = [Bar(128, f"p_full{i}", clock) for i in range(nsbuf)]
+    pv_done = [Bar(1, f"pv_done{t}", clock) for t in range(NT)]
+
+    def sbuf_of(jg, tt):
+        return tt * 2 + (jg & 1) if pipe else (tt if NT == 2 else jg & 1)
+
+    def sphase_of(jg):
+        return (jg >> 1) & 1 if (pipe or NT == 1) else jg & 1
     q_full = Bar(1, "q_full", clock)
     q_empty = Bar(128 * NT if q_tmem else NT, "q_empty", clock)
     q_tmem_bar = [Bar(128, f"q_tmem{t}", clock) for t in range(NT)]
@@ -116,7 +127,7 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
     # score buffer -> per half ("lo": the columns P overwrites, "hi": the rest) the item and
     # its state: 'S' (scores landed), 'read' (in the softmax's registers), 'P' (P written),
     # 'consumed' (read by P V)
-    sbuf = [{"lo": None, "hi": None}, {"lo": None, "hi": None}]
+    sbuf = [{"lo": None, "hi": None} for _ in range(nsbuf)]
     obuf = {}           # tile -> [unit, blocks accumulated, 'acc' | 'read']
     landings = []       # TMA loads in flight
     tensor = []         # issued MMAs and commits: (issuer, kind, x); in order per issuer
@@ -168,7 +179,7 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
         for ui, u in enumerate(busy):
             nxt = busy[ui + 1] if ui + 1 < len(busy) else None
             for j in range(u["n"]):
-                for tt in range(NT):
+                for tt in range(1 if pipe else NT):
                     if tt == 0:
                         yield from load_kv("k", u, j)
                     if q_tmem and j == 0 and tt == 0 and nxt:
@@ -201,33 +212,33 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             yield from wait(kfull[s], ph)
             st["kslot"] = s
 
-        def qk_op(s, item, g, halves):
+        def qk_op(s, item, sb, halves):
             def op():
                 check(kslot[s] == item[:2], f"Q K^T {item} reads K {kslot[s]}")
                 q = qtm.get(item[2]) if q_tmem else qstage[0]
                 check(q == item[0], f"Q K^T {item} reads the Q of unit {q}")
-                b = sbuf[g & 1]
+                b = sbuf[sb]
                 for h in halves:
                     free = ("consumed",) if h == "lo" else ("read", "consumed")
                     check(b[h] is None or b[h][1] in free, f"Q K^T {item} overwrites {h} {b[h]}")
                     b[h] = (item, "S")
             return op
 
-        def qk(u, j, tt, g, last):  # a whole Q K^T (both key halves)
+        def qk(u, j, tt, sb, last):  # a whole Q K^T (both key halves) into score buffer sb
             if q_tmem and j == 0:
                 yield from wait(q_tmem_bar[tt], st["units"] & 1)
             yield from take_k()
             s = st["kslot"]
-            Q.append(("op", qk_op(s, (u["id"], j, tt), g, ("lo", "hi"))))
-            Q.append(("commit", s_full[g & 1]))
+            Q.append(("op", qk_op(s, (u["id"], j, tt), sb, ("lo", "hi"))))
+            Q.append(("commit", s_full[sb]))
             Q.append(("commit", kempty[s]))
             if not q_tmem and last:
                 Q.append(("commit", q_empty))
             yield True
 
-        def pv(g, u, j, tt, last_block, uidx):
+        def pv(sb, ph, u, j, tt, last_block, uidx):
             item = (u["id"], j, tt)
-            yield from wait(p_full[g & 1], (g >> 1) & 1)
+            yield from wait(p_full[sb], ph)
             if j == 0 and uidx > 0 and mutant != "no_o_free_wait":
                 yield from wait(o_free[tt], (uidx - 1) & 1)
             s = st["v"] % NV
@@ -235,11 +246,11 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             st["v"] += 1
             yield from wait(vfull[s], ph)
 
-            def op(s=s, item=item, g=g):
+            def op(s=s, item=item, sb=sb):
                 check(vslot[s] == item[:2], f"P V {item} reads V {vslot[s]}")
-                lo = sbuf[g & 1]["lo"]
+                lo = sbuf[sb]["lo"]
                 check(lo == (item, "P"), f"P V {item} reads {lo}")
-                sbuf[g & 1]["lo"] = (item, "consumed")
+                sbuf[sb]["lo"] = (item, "consumed")
                 o = obuf.get(item[2])
                 if item[1] == 0:
                     check(o is None or o[2] == "read", f"P V {item} overwrites unread O {o}")
@@ -248,8 +259,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
                     check(o[0] == item[0] and o[1] == item[1], f"P V {item} finds O {o}")
                     o[1] += 1
             Q.append(("op", op))
-            if NT == 1:
-                Q.append(("commit", pv_done))
+            if NT == 1 or pipe:
+                Q.append(("commit", pv_done[tt]))
             Q.append(("commit", vempty[s]))
             if last_block:
                 Q.append(("commit", o_full[tt]))
@@ -263,15 +274,15 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             for j in range(u["n"]):
                 last = j == u["n"] - 1
                 for tt in tiles:
-                    g = jg * NT + tt
-                    if NT == 2:
-                        yield from qk(u, j, tt, g, last)
-                        yield from pv(g, u, j, tt, last, st["units"])
+                    sb = sbuf_of(jg, tt)
+                    if NT == 2 and not pipe:
+                        yield from qk(u, j, tt, sb, last)
+                        yield from pv(sb, sphase_of(jg), u, j, tt, last, st["units"])
                     else:
-                        yield from qk(u, j, tt, g, last)
+                        yield from qk(u, j, tt, sb, last)
                         if pend:
                             yield from pv(*pend)
-                        pend = (g, u, j, tt, last, st["units"])
+                        pend = (sb, sphase_of(jg), u, j, tt, last, st["units"])
                 jg += 1
             st["units"] += 1
         if pend:
@@ -309,15 +320,14 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
             nxt = busy[ui + 1] if ui + 1 < len(busy) else None
             for j in range(u["n"]):
                 for tt in tiles:
-                    g = jg * NT + tt
-                    sb = g & 1
+                    sb = sbuf_of(jg, tt)
                     item = (u["id"], j, tt)
-                    if NT == 2:  # the two tiles' softmax take turns, block by block
+                    if NT == 2 and not pipe:  # the two tiles' softmax take turns, block by block
                         if tt == 1:
                             yield from wait(p_full[0], jg & 1)
                         elif jg > 0:
                             yield from wait(p_full[1], (jg - 1) & 1)
-                    parity = ((g >> 1) & 1) ^ (1 if mutant == "s_full_wrong_parity" else 0)
+                    parity = sphase_of(jg) ^ (1 if mutant == "s_full_wrong_parity" else 0)
                     yield from wait(s_full[sb], parity)
                     if q_tmem and j == u["n"] - 1 and nxt:
                         yield from copy_q(ui + 1, tt, nxt["id"])
@@ -326,8 +336,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
                           f"softmax of {item} reads {b}")
                     b["lo"], b["hi"] = (item, "read"), (item, "read")
                     if j > 0 and rnd.random() < 0.3:  # the running max grew: rescale O
-                        if NT == 1 and mutant != "no_pv_done_wait":
-                            yield from wait(pv_done, (g - 1) & 1)
+                        if (NT == 1 or pipe) and mutant != "no_pv_done_wait":
+                            yield from wait(pv_done[tt], (jg - 1) & 1)
                         o = obuf.get(tt)
                         check(o is not None and o[0] == u["id"] and o[1] == j,
                               f"rescale of {item} finds O {o}")
@@ -394,12 +404,13 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None):
     return steps
 
 
-# The kernel's layouts: (NT, NSM, Q in tensor memory, K slots, V slots), from the traits table of
-# csrc/attn_api.cu (d64 dense, d64 packed, d128, d192/128, d256, E4M3 d128) plus ring-depth edge
-# cases (a single slot).
-LAYOUTS = [(2, 2, True, 5, 5), (1, 1, True, 6, 6), (2, 2, False, 3, 2), (2, 2, False, 2, 1),
-           (1, 1, True, 2, 2), (2, 2, False, 4, 4), (2, 2, True, 1, 1), (1, 1, False, 1, 1),
-           (2, 2, False, 1, 1)]
+# The kernel's layouts: (NT, NSM, Q in tensor memory, K slots, V slots, pipelined two-tile), from
+# the traits table of csrc/attn_api.cu (d64, d128, d192/128, d256, E4M3 d128) plus ring-depth
+# edge cases (a single slot) and layouts the kernel supports but does not dispatch.
+LAYOUTS = [(2, 2, True, 8, 8, True), (2, 2, False, 3, 2, False), (2, 2, False, 2, 1, False),
+           (1, 1, True, 2, 2, False), (2, 2, False, 4, 4, False), (1, 1, True, 6, 6, False),
+           (2, 2, True, 1, 1, True), (1, 1, False, 1, 1, False), (2, 2, False, 1, 1, False),
+           (2, 2, False, 2, 2, True), (2, 2, True, 5, 5, False)]
 
 
 def random_units(rnd):

@@ -10,23 +10,23 @@ from protocol_model import LAYOUTS, MUTANTS, Deadlock, Violation, random_units, 
 SEEDS = 300
 
 
-@pytest.mark.parametrize("layout", LAYOUTS, ids=[f"nt{a}_nsm{b}_qt{int(c)}_k{d}_v{e}"
-                                                 for a, b, c, d, e in LAYOUTS])
+@pytest.mark.parametrize("layout", LAYOUTS, ids=[f"nt{a}_nsm{b}_qt{int(c)}_k{d}_v{e}_pipe{int(f)}"
+                                                 for a, b, c, d, e, f in LAYOUTS])
 def test_protocol_holds(layout):
-    NT, NSM, q_tmem, NK, NV = layout
+    NT, NSM, q_tmem, NK, NV, pipe = layout
     for seed in range(SEEDS):
         units = random_units(random.Random(seed * 7 + NT))
-        run(units, NT, NSM, q_tmem, NK, NV, seed)
+        run(units, NT, NSM, q_tmem, NK, NV, seed, pipe=pipe)
 
 
 @pytest.mark.parametrize("mutant", sorted(MUTANTS))
 def test_model_catches_planted_mistake(mutant):
     caught = 0
-    for NT, NSM, q_tmem, NK, NV in LAYOUTS:
+    for NT, NSM, q_tmem, NK, NV, pipe in LAYOUTS:
         for seed in range(60):
             units = random_units(random.Random(seed * 7 + NT))
             try:
-                run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=mutant)
+                run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=mutant, pipe=pipe)
             except (Violation, Deadlock):
                 caught += 1
     assert caught > 0, f"the model did not catch: {MUTANTS[mutant]}"

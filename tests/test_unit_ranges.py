@@ -89,7 +89,7 @@ def test_unit_ranges_random(seed):
 
 def test_unit_ranges_workload_shapes():
     # the benchmark shapes' geometry (per head): 2048^2, 8192^2 (and its window), 4096^2, 65536^2
-    for sq, NT, BN, causal, window in [(2048, 2, 128, True, -1), (8192, 2, 128, True, -1),
-                                       (8192, 2, 128, True, 128), (4096, 1, 64, False, -1),
+    for sq, NT, BN, causal, window in [(2048, 2, 64, True, -1), (8192, 2, 128, True, -1),
+                                       (8192, 2, 64, True, 128), (4096, 1, 64, False, -1),
                                        (65536, 2, 128, True, -1)]:
         check_shape(sq, sq, NT, BN, causal, window)
