@@ -21,6 +21,28 @@ __device__ int g_attn_status;
 std::mutex g_starve_mu;
 unsigned long long g_starve_timeout_ns = 0;
 
+// Device address of the error word on the current device (the host-side name of a __device__
+// variable is not a device address), cached per device. The per-device caches of this library
+// are atomics: concurrent first calls from several host threads store the same value, and no
+// thread reads a half-written one.
+int* status_word()
+{
+    static std::atomic<int*> addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    int* a = addr[dev].load(std::memory_order_relaxed);
+    if (a == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        a = static_cast<int*>(p);
+        addr[dev].store(a, std::memory_order_relaxed);
+    }
+    return a;
+}
+
 namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -38,26 +60,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
             cudaGetLastError();
     });
     return fn;
-}
-
-// Per-device caches below are atomics: concurrent first calls from several host threads store
-// the same value, and no thread reads a half-written one.
-int* status_word()
-{
-    static std::atomic<int*> addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    int* a = addr[dev].load(std::memory_order_relaxed);
-    if (a == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_attn_status) != cudaSuccess) {
-            cudaGetLastError();
-            return nullptr;
-        }
-        a = static_cast<int*>(p);
-        addr[dev].store(a, std::memory_order_relaxed);
-    }
-    return a;
 }
 
 // 4-D tensor map over a BSHD tensor [b, s, h, d] (innermost first: d, h, s, b) of bf16

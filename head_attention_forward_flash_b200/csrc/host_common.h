@@ -57,6 +57,11 @@ inline int check_arch()
     return ok ? B200ATTN_OK : B200ATTN_ERR_ARCH;
 }
 
+// Device address of the library's error word on the current device, where kernels whose
+// bounded waits give up record B200ATTN_ERR_TIMEOUT (read and cleared by attn_debug_status);
+// null if CUDA fails. Defined in attn_api.cu.
+int* status_word();
+
 // Stream-ordered pool for the pre-passes' partial results (k_smooth_mean, k_smooth_gate,
 // fp8_quantize), one per device. Its release threshold is
 // "never", so memory freed at the end of a call stays in the pool for the next call instead of

@@ -1,75 +1,131 @@
-"""The work split of the K-mean and K-smoothing-gate pre-passes (csrc/kmean.cu), transcribed and
-checked on the CPU: k_mean_partial sums every (key row, 8-channel group) exactly once, and
-k_gate_partial reads exactly the strided sample 0, stride, 2*stride, ... < sk (every key up to
-2048 keys, at most 2048 samples beyond), each sampled row in exactly one chunk."""
+"""The work split of the one-pass K-mean and K-smoothing-gate kernels (csrc/kmean.cu: make_split,
+sum_chunks and the two folds), transcribed and checked on the CPU:
+  - phase 1 sums every (key row, 8-channel group) of every batch exactly once (the gate: exactly
+    the strided sample 0, stride, 2*stride, ... < sk, every key up to 2048 keys, at most 2048
+    samples beyond), and every partial it writes lies inside the scratch sized for the split;
+  - the fold covers every (batch, column) of the mean once (the gate: every (batch, kv head)),
+    and its chunk ranges (per warp, per channel group) cover every chunk exactly once;
+  - the allocation-free entry point's split never needs more partials than its fixed array holds.
+"""
 import random
 
 import pytest
 
-THREADS = 256
+THREADS = 512
 COLS_PER_CTA = THREADS * 8
-TARGET_CTAS = 4 * 148
-MIN_ROWS_PER_CHUNK = 16
+FOLD_WARPS = THREADS // 32
+SMS = 148
+NOALLOC_FLOATS = 1 << 20
 
 
-def mean_split(b, hk, sk, d):
-    cols = hk * d
-    col_ctas = (cols + COLS_PER_CTA - 1) // COLS_PER_CTA
-    nchunks = (TARGET_CTAS + col_ctas * b - 1) // (col_ctas * b)
-    nchunks = min(nchunks, (sk + MIN_ROWS_PER_CHUNK - 1) // MIN_ROWS_PER_CHUNK, 1024)
-    nchunks = max(nchunks, 1)
-    rpc = (sk + nchunks - 1) // nchunks
-    nchunks = (sk + rpc - 1) // rpc
-    return cols, col_ctas, nchunks, rpc
+def make_split(b, cols, n_rows, max_chunks, grid_max):
+    colgroups = (cols + COLS_PER_CTA - 1) // COLS_PER_CTA
+    nch = (grid_max + b * colgroups - 1) // (b * colgroups)
+    nch = min(nch, (n_rows + 15) // 16, max_chunks, 1024)
+    nch = max(nch, 1)
+    rpc = (n_rows + nch - 1) // nch
+    nchunks = (n_rows + rpc - 1) // rpc
+    n_items = b * colgroups * nchunks
+    return colgroups, rpc, nchunks, n_items, min(n_items, grid_max)
 
 
-def gate_split(b, hk, sk, d):
-    cols = hk * d
-    stride = (sk + 2047) // 2048
-    n_samp = (sk + stride - 1) // stride
-    col_ctas = (cols + COLS_PER_CTA - 1) // COLS_PER_CTA
-    nchunks = (TARGET_CTAS + col_ctas * b - 1) // (col_ctas * b)
-    nchunks = min(nchunks, (n_samp + 31) // 32, 1024)
-    nchunks = max(nchunks, 1)
-    per_chunk = (n_samp + nchunks - 1) // nchunks
-    nchunks = (n_samp + per_chunk - 1) // per_chunk
-    return cols, col_ctas, stride, n_samp, nchunks, per_chunk
+def phase1(b, cols, n_rows, stride, split, planes):
+    """(bi, row, 8-channel group) -> times summed, and the largest partial index written."""
+    colgroups, rpc, nchunks, n_items, grid = split
+    c8 = cols // 8
+    seen = {}
+    top = -1
+    for cta in range(grid):
+        for it in range(cta, n_items, grid):
+            chunk = it % nchunks
+            bcg = it // nchunks
+            cg, bi = bcg % colgroups, bcg // colgroups
+            for tid in range(THREADS):
+                g8 = cg * THREADS + tid
+                if g8 >= c8:
+                    continue
+                for t in range(chunk * rpc, min(chunk * rpc + rpc, n_rows)):
+                    key = (bi, t * stride, g8)
+                    seen[key] = seen.get(key, 0) + 1
+                base = ((bi * nchunks + chunk) * planes) * cols + g8 * 8
+                top = max(top, base + (planes - 1) * cols + 7)
+    return seen, top
 
 
 CASES = [(1, 16, 4096, 256), (1, 5, 65536, 128), (8, 8, 2048, 64), (2, 3, 100, 64),
-         (1, 1, 1, 128), (3, 5, 17, 256), (1, 4, 2049, 64), (1, 2, 5000, 128)]
+         (1, 1, 1, 128), (3, 5, 17, 256), (1, 4, 2049, 64), (1, 2, 5000, 128), (2, 40, 300, 256)]
 
 
-@pytest.mark.parametrize("seed", range(3))
-def test_mean_covers_every_row_once(seed):
+def random_cases(rnd, max_sk):
+    return [(rnd.randint(1, 6), rnd.randint(1, 24), rnd.randint(1, max_sk),
+             rnd.choice([64, 128, 256])) for _ in range(12)]
+
+
+@pytest.mark.parametrize("seed", range(2))
+def test_mean_sums_every_row_once_inside_its_scratch(seed):
     rnd = random.Random(seed)
-    cases = CASES + [(rnd.randint(1, 8), rnd.randint(1, 40), rnd.randint(1, 9000),
-                      rnd.choice([64, 128, 256])) for _ in range(25)]
-    for b, hk, sk, d in cases:
-        cols, col_ctas, nchunks, rpc = mean_split(b, hk, sk, d)
-        assert 1 <= nchunks <= 1024
-        c8 = cols // 8
-        groups = {g8 for x in range(col_ctas) for g8 in range(x * THREADS, (x + 1) * THREADS)
-                  if g8 < c8}
-        assert groups == set(range(c8))  # every 8-channel group has one thread per chunk
-        rows = [s for chunk in range(nchunks) for s in range(chunk * rpc, min(chunk * rpc + rpc, sk))]
-        assert sorted(rows) == list(range(sk)), (b, hk, sk, d)
+    for b, hk, sk, d in CASES + random_cases(rnd, 3000):
+        cols = hk * d
+        split = make_split(b, cols, sk, 1024, SMS)
+        colgroups, rpc, nchunks, n_items, grid = split
+        assert 1 <= nchunks <= 1024 and 1 <= grid <= SMS
+        if sk * b * cols > 4_000_000:  # the full transcription is slow: check the row split only
+            rows = [t for ch in range(nchunks) for t in range(ch * rpc, min(ch * rpc + rpc, sk))]
+            assert sorted(rows) == list(range(sk))
+            continue
+        seen, top = phase1(b, cols, sk, 1, split, 1)
+        assert set(seen.values()) == {1}
+        assert len(seen) == b * sk * (cols // 8), (b, hk, sk, d)
+        assert top < b * nchunks * cols  # the partials the host allocates
 
 
-@pytest.mark.parametrize("seed", range(3))
+@pytest.mark.parametrize("seed", range(2))
 def test_gate_reads_the_strided_sample_once(seed):
     rnd = random.Random(10 + seed)
-    cases = CASES + [(rnd.randint(1, 8), rnd.randint(1, 40), rnd.randint(1, 70000),
-                      rnd.choice([64, 128, 256])) for _ in range(25)]
-    for b, hk, sk, d in cases:
-        cols, col_ctas, stride, n_samp, nchunks, per_chunk = gate_split(b, hk, sk, d)
-        assert 1 <= nchunks <= 1024
+    for b, hk, sk, d in CASES + random_cases(rnd, 70000):
+        cols = hk * d
+        stride = (sk + 2047) // 2048
+        n_samp = (sk + stride - 1) // stride
         if sk <= 2048:
             assert stride == 1 and n_samp == sk
         else:
             assert n_samp <= 2048
-        ts = [t for chunk in range(nchunks)
-              for t in range(chunk * per_chunk, min(chunk * per_chunk + per_chunk, n_samp))]
+        split = make_split(b, cols, n_samp, 1024, SMS)
+        colgroups, rpc, nchunks, n_items, grid = split
+        ts = [t for ch in range(nchunks) for t in range(ch * rpc, min(ch * rpc + rpc, n_samp))]
         assert sorted(ts) == list(range(n_samp))
-        keys = [t * stride for t in ts]
-        assert sorted(keys) == list(range(0, sk, stride)), (b, hk, sk, d)
+        assert sorted(t * stride for t in ts) == list(range(0, sk, stride)), (b, hk, sk, d)
+        if n_samp * b * cols <= 4_000_000:
+            seen, top = phase1(b, cols, n_samp, stride, split, 2)
+            assert set(seen.values()) == {1} and len(seen) == b * n_samp * (cols // 8)
+            assert top < b * nchunks * 2 * cols
+
+
+def test_fold_covers_every_column_and_chunk_once():
+    for b, hk, sk, d in CASES:
+        cols = hk * d
+        _, _, nchunks, _, grid = make_split(b, cols, sk, 1024, SMS)
+        nblk = (cols + 31) // 32
+        outs = [(f // nblk, (f % nblk) * 32 + lane) for cta in range(grid)
+                for f in range(cta, b * nblk, grid) for lane in range(32)
+                if (f % nblk) * 32 + lane < cols]
+        assert sorted(outs) == [(bi, c) for bi in range(b) for c in range(cols)]
+        ranges = [c for w in range(FOLD_WARPS)
+                  for c in range(w * nchunks // FOLD_WARPS, (w + 1) * nchunks // FOLD_WARPS)]
+        assert ranges == list(range(nchunks))
+        # gate fold: (batch, kv head) items, 512/d channel groups over the chunks
+        groups = THREADS // d
+        heads = [f for cta in range(grid) for f in range(cta, b * hk, grid)]
+        assert sorted(heads) == list(range(b * hk))
+        ranges = [c for g in range(groups)
+                  for c in range(g * nchunks // groups, (g + 1) * nchunks // groups)]
+        assert ranges == list(range(nchunks))
+
+
+def test_noalloc_split_fits_the_fixed_scratch():
+    for b, hk, sk, d in CASES + [(4, 1024, 40, 256), (1, 4096, 300, 256), (64, 64, 5000, 256)]:
+        cols = hk * d
+        if b * cols > NOALLOC_FLOATS:
+            continue  # refused with ERR_SCRATCH
+        _, _, nchunks, _, grid = make_split(b, cols, sk, NOALLOC_FLOATS // (b * cols), SMS)
+        assert b * nchunks * cols <= NOALLOC_FLOATS and grid <= 1024
