@@ -256,11 +256,13 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 //    pipelined layout's 64-key Q K^T from shared memory runs at 2/3 of the tensor rate: 1027 vs
 //    1041 at 65536^2 d128, 996 vs 1021 at 8192^2 d192/128).
 //  - d256: one tile, two 64-key score buffers.
-// The share of score pairs whose exp2 runs on the FMA pipe is the measured best per head dim
-// (3 of 8 at d64, 2 of 8 at d128 / d192 and for E4M3 inputs, none at d256, bound by the tensor
-// core).
+// The share of score pairs whose exp2 runs on the FMA pipe is the measured best per head dim:
+// 3 of 8 at d128 (pairs 0, 2, 5 of every 8: 1141 vs 1060 with 2 of 8 at 65536^2, interleaved
+// A/B), 2 of 8 at d192 (3 of 8 is no faster there) and for E4M3 inputs (3 of 8 loses 1-3 %),
+// none at d256, bound by the tensor core. At d64 the share makes no measurable difference
+// (3 of 8 kept).
 using T64P = AttnTraits<64, 64, 64, 2, 2, true, 8, 8, 0x92u, false, true>;  // 32 + 64 + 64 (+32) KB
-using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x11u>;         // 64 + 96 + 64 KB
+using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x25u>;         // 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;         // 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;                  // 64 + 64 + 64 KB
 // E4M3 inputs, (128, 128): the d128 layout with half-size tiles, so four K and four V slots fit
