@@ -12,7 +12,7 @@ Raw C entry points, with the header's names and argument order, are exposed thro
 (a ``ctypes.CDLL``): every name in ``EXPORTS`` (``lib.attn_fwd``, ``lib.attn_fwd_varlen``,
 ``lib.attn_fwd_window_sink``, ``lib.attn_fwd_fp8``, ``lib.fp8_quantize``, ``lib.k_smooth_gate``,
 ``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``, ``lib.k_smooth_sub``,
-``lib.attn_status_string``, ``lib.attn_debug_status``, ``lib.attn_debug_starve``).
+``lib.k_smooth_mean_sub``, ``lib.attn_status_string``, ``lib.attn_debug_status``, ``lib.attn_debug_starve``).
 """
 from __future__ import annotations
 
@@ -30,7 +30,7 @@ STATUS = {
 }
 EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "attn_fwd_fp8", "fp8_quantize",
            "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
-           "attn_status_string", "attn_debug_status", "attn_debug_starve")
+           "k_smooth_mean_sub", "attn_status_string", "attn_debug_status", "attn_debug_starve")
 
 
 class B200AttnError(RuntimeError):
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
     lib.k_smooth_gate.restype = ctypes.c_int
     lib.k_smooth_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_sub.restype = ctypes.c_int
+    lib.k_smooth_mean_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.k_smooth_mean_sub.restype = ctypes.c_int
     lib.attn_status_string.argtypes = [ctypes.c_int]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_debug_status.argtypes = [vp]
@@ -376,6 +378,27 @@ def k_smooth_sub(k, mean, out=None):
     _check("k_smooth_sub", lib.k_smooth_sub(k.data_ptr(), mean.data_ptr(), out.data_ptr(), b, hk,
                                             sk, d, _stream_ptr(k)))
     return out
+
+
+def k_smooth_mean_sub(k, mean=None, out=None):
+    """k_smooth_mean and k_smooth_sub in one launch: returns ``(mean [b, hk, d] fp32,
+    bf16(K - mean) [b, sk, hk, d])``, bit-identical to the two calls in sequence."""
+    import torch
+    _want(k, "k", 4)
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
+    b, sk, hk, d = k.shape
+    if mean is None:
+        mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    else:
+        _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
+    if out is None:
+        out = torch.empty_like(k)
+    else:
+        _want_out(out, "out", (b, sk, hk, d), torch.bfloat16, k.device)
+    _check("k_smooth_mean_sub", lib.k_smooth_mean_sub(k.data_ptr(), mean.data_ptr(), out.data_ptr(),
+                                                      b, hk, sk, d, _stream_ptr(k)))
+    return mean, out
 
 
 def attn_debug_status(stream=None) -> int:

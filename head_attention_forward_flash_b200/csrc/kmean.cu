@@ -1,5 +1,6 @@
 // kmean.cu -- the K channel-mean pre-pass (k_smooth_mean, k_smooth_mean_noalloc), the K-smoothing
-// gate (k_smooth_gate) and the mean subtraction (k_smooth_sub).
+// gate (k_smooth_gate), the mean subtraction (k_smooth_sub) and both steps in one launch
+// (k_smooth_mean_sub).
 //
 // K is [b, sk, hk, d] bf16; for a fixed (batch, key position) the hk*d channels of all kv heads
 // are one contiguous row, so the mean over the key axis is a column sum of a [sk, hk*d] matrix
@@ -12,7 +13,10 @@
 //            carries this call's tag, then fold the partials in a fixed order.
 // The fold order never depends on timing, so results are bit-identical from run to run: the
 // "two deterministic kernels behind one host call" of "[HIP] Mha v4: run the K-smoothing gate as
-// one HIP call" (Summary, commit message) become two phases of one kernel.
+// one HIP call" (Summary, commit message) become two phases of one kernel. The fused mean and
+// subtraction adds
+//   phase 3  the fold CTAs publish their columns of the mean in a second set of flags; once every
+//            one has, all CTAs write K - mean, re-reading K (from L2 when it fits there).
 #include <atomic>
 #include <cmath>
 #include <cuda_bf16.h>
@@ -29,6 +33,9 @@ constexpr int kFoldWarps = kThreads / 32;
 constexpr int kSubThreads = 256;
 constexpr int kErrTimeout = 10;                       // B200ATTN_ERR_TIMEOUT
 constexpr uint64_t kTagMagic = 0x6B6D65616EULL << 24;  // high bits of every flag tag
+constexpr int kMaxGrid = 1024;  // CTAs of a one-pass launch at most (flag words per set)
+constexpr int kGo1 = kMaxGrid, kGo2 = kMaxGrid + 16;  // go words after the phase-1 flags
+constexpr int kFlagWords = kMaxGrid + 32;  // one flag set with its go words (16 words apart)
 
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& x)
 {
@@ -65,10 +72,11 @@ __device__ __forceinline__ void publish(unsigned long long* flag, unsigned long 
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(flag), "l"(tag) : "memory");
 }
 
-__device__ __forceinline__ unsigned long long observe(const unsigned long long* flag)
+// A relaxed (strong, unordered) load of a flag word: polls of several flags issue together.
+__device__ __forceinline__ unsigned long long peek(const unsigned long long* flag)
 {
     unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flag) : "memory");
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(flag));
     return v;
 }
 
@@ -82,32 +90,77 @@ __device__ __forceinline__ void publish_cta(unsigned long long* flags, unsigned 
     }
 }
 
-// Waits until each CTA of the grid has published `tag` (the first warp polls, each lane a share
-// of the flags, backing off between polls so that waiting CTAs load L2 as little as possible);
-// false, with the error word set, if that takes longer than timeout_ns.
+// Polls until every flag flags[c], c < n (<= 1024), carries `tag`, with the first warp: lane l
+// watches flags l, l + 32, ... and loads its unseen ones eight at a time each round (relaxed
+// loads, so they do not wait for one another), backing off between rounds. False, with the
+// error word set, if that takes longer than timeout_ns (counted from t0). Warp 0 only.
+__device__ __forceinline__ bool poll_flags(const unsigned long long* flags, unsigned long long tag,
+                                           int n, int* status, uint64_t t0,
+                                           unsigned long long timeout_ns)
+{
+    const int lane = threadIdx.x & 31;
+    const int mine = lane < n ? (n - lane + 31) / 32 : 0;  // flags lane, lane + 32, ...
+    uint32_t pending = mine >= 32 ? 0xFFFFFFFFu : ((1u << mine) - 1u);
+    while (pending) {
+        for (int j0 = 0; j0 < mine; j0 += 8) {  // eight loads in flight per lane
+            unsigned long long v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if ((pending >> (j0 + j)) & 1u) v[j] = peek(flags + lane + 32 * (j0 + j));
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (((pending >> (j0 + j)) & 1u) && v[j] == tag) pending &= ~(1u << (j0 + j));
+        }
+        if (!pending) break;
+        if (global_ns() - t0 > timeout_ns) {
+            atomicCAS(status, 0, kErrTimeout);
+            return false;
+        }
+        __nanosleep(32);
+    }
+    return true;
+}
+
+// Waits until each of the first n CTAs of the grid has published `tag` in flags[c]; `waiters` is
+// the number of CTAs (the first ones, CTA 0 among them) that call this. A few waiters poll the n
+// flags themselves. Many waiters would queue behind each other on the flags' few L2 lines, so
+// then only CTA 0 reads the n flags; it publishes `tag` in *go, and every other CTA polls that one
+// word (two hops instead of one, but one L2 line polled once per round per CTA).
+// A relaxed read followed by a fence is an acquire, and CTA 0's release of *go passes on every
+// publisher's writes that it observed (release is cumulative); the CTA barrier then orders the
+// waiting thread's view before every thread of its CTA. False, with the error word set, if a wait
+// takes longer than timeout_ns.
 __device__ __forceinline__ bool wait_all_published(const unsigned long long* flags,
-                                                   unsigned long long tag, int* status,
+                                                   unsigned long long tag, int n, int waiters,
+                                                   unsigned long long* go, int* status,
                                                    unsigned long long timeout_ns)
 {
     bool ok = true;
-    if (threadIdx.x < 32) {
-        const uint64_t t0 = global_ns();
-        for (int c = threadIdx.x; c < (int)gridDim.x && ok; c += 32) {
-            while (observe(flags + c) != tag) {
-                if (global_ns() - t0 > timeout_ns) {
-                    atomicCAS(status, 0, kErrTimeout);
-                    ok = false;
-                    break;
-                }
-                __nanosleep(32);
-            }
+    const uint64_t t0 = global_ns();
+    if (waiters <= 16 || blockIdx.x == 0) {
+        if (threadIdx.x < 32) {
+            ok = __all_sync(0xFFFFFFFFu, poll_flags(flags, tag, n, status, t0, timeout_ns));
+            __threadfence();
+            __syncwarp();  // every lane's acquire is ordered before lane 0's release
+            if (waiters > 16 && threadIdx.x == 0 && ok) publish(go, tag);
         }
+    } else if (threadIdx.x == 0) {
+        while (peek(go) != tag) {
+            if (global_ns() - t0 > timeout_ns) {
+                atomicCAS(status, 0, kErrTimeout);
+                ok = false;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence();
     }
     return __syncthreads_and(ok) != 0;
 }
 
 // sum over c in [c_lo, c_hi) of src[c * pitch], added in order of c; the loads are issued eight
-// at a time (L2 hits, after the flags), so the chain is not one load latency per term.
+// at a time (L2 hits, after the flags), so the chain is not one load latency per term. (Sixteen
+// at a time made ptxas give the mean kernel fewer registers than its phase 1 needs.)
 __device__ __forceinline__ float ordered_sum(const float* src, int64_t pitch, int c_lo, int c_hi)
 {
     float sum = 0.f;
@@ -126,7 +179,9 @@ __device__ __forceinline__ float ordered_sum(const float* src, int64_t pitch, in
 struct OnePass {
     const uint4* k;
     float* partial;             // [b][nchunks][planes][cols]
-    unsigned long long* flags;  // [gridDim.x]
+    unsigned long long* flags;  // [gridDim.x] phase 1 done, then go words at kGo1 and kGo2
+    unsigned long long* flags2; // fused mean and subtraction only: [gridDim.x], fold done
+    uint4* k_out;               // fused mean and subtraction only: [b, sk, hk, d] bf16
     float* mean;                // [b][cols]
     int* gate;                  // gate only: [b][hk]
     float* ratio;               // gate only, may be null
@@ -193,19 +248,16 @@ __device__ __forceinline__ void sum_chunks(const OnePass& a)
 // mean[bi][col] = (sum of partial[bi][chunk][col] over the chunks) / sk. Fold items are blocks of
 // 32 columns of one batch; warp w of the CTA sums the chunks of its fixed contiguous range
 // [w*nchunks/16, (w+1)*nchunks/16) in order, then the 16 warp sums are added in warp order.
-__global__ void __launch_bounds__(kThreads) k_mean_onepass(const OnePass a)
+// Run by CTAs below n_fold(a), after the wait for every CTA's phase 1.
+__device__ __forceinline__ int64_t n_fold(const OnePass& a) { return a.b * ((a.cols + 31) / 32); }
+
+__device__ __forceinline__ void fold_mean(const OnePass& a, float (&red)[kFoldWarps][32])
 {
-    __shared__ float red[kFoldWarps][32];
-    sum_chunks<false>(a);
-    publish_cta(a.flags, a.tag);
     const int64_t nblk = (a.cols + 31) / 32;
-    const int64_t n_fold = a.b * nblk;
-    if ((int64_t)blockIdx.x >= n_fold) return;
-    if (!wait_all_published(a.flags, a.tag, a.status, a.timeout_ns)) return;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int c_lo = (int)((int64_t)w * a.nchunks / kFoldWarps);
     const int c_hi = (int)((int64_t)(w + 1) * a.nchunks / kFoldWarps);
-    for (int64_t f = blockIdx.x; f < n_fold; f += gridDim.x) {
+    for (int64_t f = blockIdx.x; f < n_fold(a); f += gridDim.x) {
         const int64_t bi = f / nblk;
         const int64_t col = (f - bi * nblk) * 32 + lane;
         float sum = 0.f;
@@ -223,57 +275,103 @@ __global__ void __launch_bounds__(kThreads) k_mean_onepass(const OnePass a)
     }
 }
 
+__global__ void __launch_bounds__(kThreads) k_mean_onepass(const OnePass a)
+{
+    __shared__ float red[kFoldWarps][32];
+    sum_chunks<false>(a);
+    publish_cta(a.flags, a.tag);
+    const int64_t nf = n_fold(a);
+    if ((int64_t)blockIdx.x >= nf) return;
+    const int waiters = (int)(nf < (int64_t)gridDim.x ? nf : (int64_t)gridDim.x);
+    if (!wait_all_published(a.flags, a.tag, (int)gridDim.x, waiters, a.flags + kGo1, a.status,
+                            a.timeout_ns))
+        return;
+    fold_mean(a, red);
+}
+
 // The gate (see k_smooth_gate). Phase 1 sums K and K^2 over the strided sample; phase 2 item =
-// (bi, kv head): the 512 threads form 512/d groups of d (one thread per channel); group grp sums
-// the chunks of its fixed contiguous range, the group sums are added in group order, giving mu_c
-// and e_c; then sum mu_c^2 and sum e_c over the d channels by a fixed tree; ratio = first /
-// second (0 for an all-zero K); gate = ratio >= threshold; mean = mu where the gate is on, else 0.
+// (bi, kv head). Its 2d partial columns (d channel sums, then d sums of squares) are read as d/2
+// float4 columns: thread t takes float4 column t % (d/2) over the chunks of group t / (d/2)
+// (1024/d groups, each a fixed contiguous range of chunks, added in chunk order, up to twelve
+// 16-byte loads in flight: sixteen made ptxas spill); the group sums are added in group order,
+// giving mu_c and e_c; then sum mu_c^2 and sum e_c over the d channels by a fixed tree (a
+// butterfly in each warp of 32 channels, then the warp sums in order); ratio = first / second
+// (0 for an all-zero K); gate = ratio >= threshold; mean = mu where the gate is on, else 0.
 __global__ void __launch_bounds__(kThreads) k_gate_onepass(const OnePass a)
 {
-    __shared__ float gs[kThreads], gq[kThreads];
-    __shared__ float num[256], den[256];
+    __shared__ float4 gsum[kThreads];  // [group][float4 column]
+    __shared__ float num[8], den[8];  // per warp of 32 channels
     sum_chunks<true>(a);
     publish_cta(a.flags, a.tag);
     const int64_t n_fold = a.b * a.hk;
     if ((int64_t)blockIdx.x >= n_fold) return;
-    if (!wait_all_published(a.flags, a.tag, a.status, a.timeout_ns)) return;
+    const int waiters = (int)(n_fold < (int64_t)gridDim.x ? n_fold : (int64_t)gridDim.x);
+    if (!wait_all_published(a.flags, a.tag, (int)gridDim.x, waiters, a.flags + kGo1, a.status,
+                            a.timeout_ns))
+        return;
     const int d = (int)a.d;
-    const int groups = kThreads / d;
-    const int c = threadIdx.x % d, grp = threadIdx.x / d;
+    const int c4s = d / 2;  // float4 columns: d/4 of sums, then d/4 of squares
+    const int groups = kThreads / c4s;
+    const int c4 = threadIdx.x % c4s, grp = threadIdx.x / c4s;
+    const int plane = c4 < d / 4 ? 0 : 1;
+    const int ch = 4 * (c4 - plane * (d / 4));  // first of the column's four channels
     const int c_lo = (int)((int64_t)grp * a.nchunks / groups);
     const int c_hi = (int)((int64_t)(grp + 1) * a.nchunks / groups);
+    const int64_t pitch = 2 * a.cols / 4;  // float4s from one chunk's row to the next's
     for (int64_t f = blockIdx.x; f < n_fold; f += gridDim.x) {
         const int64_t bi = f / a.hk, g = f - bi * a.hk;
-        const int64_t col = g * d + c;
-        const float* src = a.partial + (bi * a.nchunks * 2) * a.cols + col;
-        const float sum = ordered_sum(src, 2 * a.cols, c_lo, c_hi);
-        const float sq = ordered_sum(src + a.cols, 2 * a.cols, c_lo, c_hi);
-        gs[threadIdx.x] = sum;
-        gq[threadIdx.x] = sq;
+        const float4* src = reinterpret_cast<const float4*>(
+            a.partial + (bi * a.nchunks * 2 + plane) * a.cols + g * d + ch);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        int c = c_lo;
+        for (; c < c_hi; c += 12) {
+            float4 v[12];
+#pragma unroll
+            for (int e = 0; e < 12; ++e)
+                if (c + e < c_hi) v[e] = __ldcg(src + (int64_t)(c + e) * pitch);
+#pragma unroll
+            for (int e = 0; e < 12; ++e)
+                if (c + e < c_hi) {
+                    acc.x += v[e].x;
+                    acc.y += v[e].y;
+                    acc.z += v[e].z;
+                    acc.w += v[e].w;
+                }
+        }
+        gsum[threadIdx.x] = acc;
         __syncthreads();
-        if (grp == 0) {
-            float s = 0.f, e = 0.f;
+        if ((int)threadIdx.x < d) {
+            const int cc = threadIdx.x;  // channel
+            const float* gs = reinterpret_cast<const float*>(gsum);
+            float s = 0.f, e = 0.f;  // a group's row: d channel sums, then d sums of squares
             for (int q = 0; q < groups; ++q) {
-                s += gs[q * d + c];
-                e += gq[q * d + c];
+                s += gs[q * 2 * d + cc];
+                e += gs[q * 2 * d + d + cc];
             }
             const float mu = __fdiv_rn(s, a.n_rows_f);
-            num[c] = mu * mu;
-            den[c] = __fdiv_rn(e, a.n_rows_f);
-            // only the d threads of group 0 take part: a barrier over exactly those warps (d is
-            // a multiple of 32), id 1
-            asm volatile("bar.sync 1, %0;" ::"r"(d) : "memory");
-            for (int wdt = d / 2; wdt > 0; wdt >>= 1) {
-                if (c < wdt) {
-                    num[c] += num[c + wdt];
-                    den[c] += den[c + wdt];
-                }
-                asm volatile("bar.sync 1, %0;" ::"r"(d) : "memory");
+            float nu = mu * mu, de = __fdiv_rn(e, a.n_rows_f);
+            // fixed tree: butterfly within each warp of 32 channels, then the d/32 warp sums
+            // in warp order (only the first d threads take part: a barrier over exactly those
+            // warps, d a multiple of 32, id 1)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                nu += __shfl_xor_sync(0xFFFFFFFFu, nu, o);
+                de += __shfl_xor_sync(0xFFFFFFFFu, de, o);
             }
-            const float r = den[0] > 0.f ? __fdiv_rn(num[0], den[0]) : 0.f;
+            if ((cc & 31) == 0) {
+                num[cc >> 5] = nu;
+                den[cc >> 5] = de;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(d) : "memory");
+            float tn = 0.f, td = 0.f;
+            for (int w = 0; w < d / 32; ++w) {
+                tn += num[w];
+                td += den[w];
+            }
+            const float r = td > 0.f ? __fdiv_rn(tn, td) : 0.f;
             const bool on = r >= a.threshold;
-            a.mean[f * d + c] = on ? mu : 0.f;
-            if (c == 0) {
+            a.mean[f * d + cc] = on ? mu : 0.f;
+            if (cc == 0) {
                 a.gate[f] = on ? 1 : 0;
                 if (a.ratio) a.ratio[f] = r;
             }
@@ -282,18 +380,9 @@ __global__ void __launch_bounds__(kThreads) k_gate_onepass(const OnePass a)
     }
 }
 
-// k_out = bf16_rne(float(K) - mean[bi, col]), 8 channels (16 bytes) per group; each thread has
-// four groups in flight per step.
-__device__ __forceinline__ void sub_group(const float* __restrict__ mean, uint4* __restrict__ k_out,
-                                          int64_t t, const uint4& x, int64_t c8, int64_t sk,
-                                          int64_t cols)
+// 8 channels of K - mean (16 bytes of bf16, each an fp32 subtraction rounded to bf16).
+__device__ __forceinline__ uint4 sub8(const uint4& x, const float (&mv)[8])
 {
-    const int64_t r = t / c8;  // bi * sk + s
-    const int64_t g8 = t - r * c8;
-    const int64_t bi = r / sk;
-    const float4* m = reinterpret_cast<const float4*>(mean + bi * cols + g8 * 8);
-    const float4 m0 = __ldg(m), m1 = __ldg(m + 1);
-    const float mv[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
     const uint32_t w[4] = {x.x, x.y, x.z, x.w};
     uint32_t o[4];
 #pragma unroll
@@ -303,33 +392,101 @@ __device__ __forceinline__ void sub_group(const float* __restrict__ mean, uint4*
         __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
         o[q] = *reinterpret_cast<uint32_t*>(&v);
     }
-    k_out[t] = make_uint4(o[0], o[1], o[2], o[3]);
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The mean is read through the read-only path (NC) when no CTA of the launch writes it, else
+// through L2; so is K (the fused kernel reads K through L2, where phase 1 left it).
+template <bool NC, class T>
+__device__ __forceinline__ T load(const T* p) { return NC ? __ldg(p) : __ldcg(p); }
+
+template <bool NC>
+__device__ __forceinline__ void load_mean8(float (&mv)[8], const float* m)
+{
+    const float4 m0 = load<NC>(reinterpret_cast<const float4*>(m));
+    const float4 m1 = load<NC>(reinterpret_cast<const float4*>(m) + 1);
+    mv[0] = m0.x; mv[1] = m0.y; mv[2] = m0.z; mv[3] = m0.w;
+    mv[4] = m1.x; mv[5] = m1.y; mv[6] = m1.z; mv[7] = m1.w;
+}
+
+// k_out = bf16_rne(float(K) - mean[bi, col]) over the [b*sk rows, c8 groups of 8 channels] view
+// of K, by nthreads threads (this one is tid). With nthreads >= c8, thread tid < R*c8 (R =
+// nthreads / c8) owns channel group tid % c8 at rows tid / c8, + R, + 2R, ...; otherwise it owns
+// groups tid, tid + nthreads, ... at every row. Each thread keeps its group's 8 mean values and
+// moves to the next batch's when its row crosses into it, so no index is divided per group. G
+// groups in flight per thread.
+template <int G, bool NC>
+__device__ __forceinline__ void sub_all(const uint4* k, const float* mean, uint4* k_out,
+                                        int64_t tid, int64_t nthreads, int64_t b, int64_t sk,
+                                        int64_t c8)
+{
+    const int64_t rows = b * sk, cols = c8 * 8;
+    const bool by_rows = nthreads >= c8;
+    const int64_t R = by_rows ? nthreads / c8 : 1;
+    if (by_rows && tid >= R * c8) return;
+    for (int64_t g8 = by_rows ? tid % c8 : tid; g8 < c8; g8 += by_rows ? c8 : nthreads) {
+        const int64_t r0 = by_rows ? tid / c8 : 0;
+        if (r0 >= rows) return;
+        int64_t bi = r0 / sk, b_end = (bi + 1) * sk;
+        float mv[8];
+        load_mean8<NC>(mv, mean + bi * cols + g8 * 8);
+        for (int64_t r = r0; r < rows; r += G * R) {
+            uint4 x[G];
+#pragma unroll
+            for (int e = 0; e < G; ++e)
+                if (r + e * R < rows) x[e] = load<NC>(k + (r + e * R) * c8 + g8);
+#pragma unroll
+            for (int e = 0; e < G; ++e) {
+                const int64_t re = r + e * R;
+                if (re < rows) {
+                    if (re >= b_end) {  // first row of a later batch
+                        bi = re / sk;
+                        b_end = (bi + 1) * sk;
+                        load_mean8<NC>(mv, mean + bi * cols + g8 * 8);
+                    }
+                    k_out[re * c8 + g8] = sub8(x[e], mv);
+                }
+            }
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kSubThreads)
     k_sub_kernel(const uint4* __restrict__ k, const float* __restrict__ mean,
-                 uint4* __restrict__ k_out, int64_t rows, int64_t sk, int64_t cols)
+                 uint4* __restrict__ k_out, int64_t b, int64_t sk, int64_t c8)
 {
-    const int64_t c8 = cols / 8;
-    const int64_t n = rows * c8;
-    const int64_t stride = (int64_t)gridDim.x * kSubThreads;
-    int64_t t = (int64_t)blockIdx.x * kSubThreads + threadIdx.x;
-    for (; t + 3 * stride < n; t += 4 * stride) {
-        uint4 x[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = __ldg(k + t + e * stride);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) sub_group(mean, k_out, t + e * stride, x[e], c8, sk, cols);
+    sub_all<8, true>(k, mean, k_out, (int64_t)blockIdx.x * kSubThreads + threadIdx.x,
+                     (int64_t)gridDim.x * kSubThreads, b, sk, c8);
+}
+
+// The mean (phases 1 and 2 exactly as k_mean_onepass, so the same split gives the same bits),
+// then k_out = K - mean over the whole tensor once every fold CTA has published its columns.
+__global__ void __launch_bounds__(kThreads) k_mean_sub_onepass(const OnePass a)
+{
+    __shared__ float red[kFoldWarps][32];
+    sum_chunks<false>(a);
+    publish_cta(a.flags, a.tag);
+    const int64_t nf = n_fold(a);
+    const int fold_ctas = (int)(nf < (int64_t)gridDim.x ? nf : (int64_t)gridDim.x);
+    if ((int)blockIdx.x < fold_ctas) {
+        if (!wait_all_published(a.flags, a.tag, (int)gridDim.x, fold_ctas, a.flags + kGo1,
+                                a.status, a.timeout_ns))
+            return;
+        fold_mean(a, red);
+        publish_cta(a.flags2, a.tag);
     }
-    for (; t < n; t += stride) sub_group(mean, k_out, t, __ldg(k + t), c8, sk, cols);
+    if (!wait_all_published(a.flags2, a.tag, fold_ctas, (int)gridDim.x, a.flags + kGo2, a.status,
+                            a.timeout_ns))
+        return;
+    sub_all<8, false>(a.k, a.mean, a.k_out, (int64_t)blockIdx.x * kThreads + threadIdx.x,
+                      (int64_t)gridDim.x * kThreads, a.b, a.sk, a.c8);
 }
 
 // Fixed scratch for k_smooth_mean_noalloc: file-scope device memory that every GPU loading this
-// library holds until the process exits: 2^20 floats of partial sums (4 MiB), then 1024 64-bit
-// flag words (8 KiB), one per CTA of the one-pass kernel.
+// library holds until the process exits: 2^20 floats of partial sums (4 MiB), then one set of
+// flag words (1024 + 32 64-bit words: one per CTA of the one-pass kernel, then the go words).
 constexpr int64_t kNoAllocScratchFloats = (int64_t)1 << 20;
-constexpr int kMaxGrid = 1024;
-__device__ __align__(256) float g_kmean_scratch[kNoAllocScratchFloats + 2 * kMaxGrid];
+__device__ __align__(256) float g_kmean_scratch[kNoAllocScratchFloats + 2 * kFlagWords];
 
 int check_kmean_args(const void* k, const void* mean, int64_t b, int64_t hk, int64_t sk,
                      int64_t d, int64_t* cols_out)
@@ -387,7 +544,10 @@ unsigned long long next_tag()
 
 // Work split of the one-pass kernels: the rows of every (bi, column group of 4096 channels) cut
 // into chunks, so that the grid's CTAs get about one item each; at least 16 rows per chunk, at
-// most max_chunks chunks (the scratch), at most 1024.
+// most max_chunks chunks (the scratch), at most 1024. (Splitting a chunk's rows among several
+// row lanes of a CTA, for K with few channels, made the gate of the b1 hk5 d128 65536-key
+// workload slower: 17.7 vs 13.7 us. Fewer CTAs then issue the loads, and each SM's outstanding
+// loads queue.)
 struct Split {
     int64_t colgroups, rows_per_chunk, n_items;
     int nchunks, grid;
@@ -422,14 +582,18 @@ int launch_onepass(void (*kernel)(const OnePass), OnePass& a, int grid, cudaStre
 }
 
 // The mean through the one-pass kernel with split sp, partials (room for sp.nchunks chunks) and
-// flags (kMaxGrid words) at the given device addresses.
-int run_mean(const void* k, float* mean, int64_t b, int64_t sk, int64_t cols, const Split& sp,
-             float* partial, unsigned long long* flags, int* status, cudaStream_t st)
+// flags (kFlagWords words) at the given device addresses; with k_out, the fused kernel, which
+// also writes K - mean and takes a second set of kFlagWords words after the first.
+int run_mean(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, int64_t cols,
+             const Split& sp, float* partial, unsigned long long* flags, int* status,
+             cudaStream_t st)
 {
     OnePass a{};
     a.k = static_cast<const uint4*>(k);
     a.partial = partial;
     a.flags = flags;
+    a.flags2 = k_out ? flags + kFlagWords : nullptr;
+    a.k_out = static_cast<uint4*>(k_out);
     a.mean = mean;
     a.b = b;
     a.sk = sk;
@@ -445,8 +609,37 @@ int run_mean(const void* k, float* mean, int64_t b, int64_t sk, int64_t cols, co
     a.tag = next_tag();
     a.status = status;
     a.timeout_ns = 4000000000ull;
-    return launch_onepass(k_mean_onepass, a, sp.grid, st);
+    return launch_onepass(k_out ? k_mean_sub_onepass : k_mean_onepass, a, sp.grid, st);
 }
+
+// k_smooth_mean and k_smooth_mean_sub: scratch (the split's partials, then two flag arrays) from
+// the library pool on `st`, returned to it after the launch.
+int mean_pooled(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, int64_t cols,
+                int grid_max, cudaStream_t st)
+{
+    int* status = status_word();
+    if (!status || grid_max <= 0) return B200ATTN_ERR_CUDA;
+    const Split sp = make_split(b, cols, sk, 1024, grid_max);
+    const size_t part_bytes = (size_t)(b * sp.nchunks * cols) * sizeof(float);
+    const size_t nbytes = part_bytes + 2 * kFlagWords * sizeof(unsigned long long);
+    char* scratch = nullptr;
+    cudaMemPool_t pool = scratch_pool();
+    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), nbytes, pool, st) !=
+                     cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    const int rc =
+        run_mean(k, mean, k_out, b, sk, cols, sp, reinterpret_cast<float*>(scratch),
+                 reinterpret_cast<unsigned long long*>(scratch + part_bytes), status, st);
+    if (cudaFreeAsync(scratch, st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    return rc;
+}
+
+std::atomic<int> g_mean_sub_grid[64];
 
 }  // namespace
 }  // namespace b200
@@ -461,28 +654,26 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
     if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
-    int* status = status_word();
-    const int grid_max = onepass_grid(k_mean_onepass, g_mean_grid);
-    if (!status || grid_max <= 0) return B200ATTN_ERR_CUDA;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // scratch: the partials of the split's chunks, then the grid's flags
-    const Split sp = make_split(b, cols, sk, 1024, grid_max);
-    const size_t part_bytes = (size_t)(b * sp.nchunks * cols) * sizeof(float);
-    const size_t nbytes = part_bytes + kMaxGrid * sizeof(unsigned long long);
-    char* scratch = nullptr;
-    cudaMemPool_t pool = scratch_pool();
-    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), nbytes, pool, st) !=
-                     cudaSuccess) {
-        cudaGetLastError();
-        return B200ATTN_ERR_CUDA;
-    }
-    rc = run_mean(k, mean, b, sk, cols, sp, reinterpret_cast<float*>(scratch),
-                  reinterpret_cast<unsigned long long*>(scratch + part_bytes), status, st);
-    if (cudaFreeAsync(scratch, st) != cudaSuccess) {
-        cudaGetLastError();
-        return B200ATTN_ERR_CUDA;
-    }
-    return rc;
+    return mean_pooled(k, mean, nullptr, b, sk, cols, onepass_grid(k_mean_onepass, g_mean_grid),
+                       static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int64_t b, int64_t hk,
+                                 int64_t sk, int64_t d, void* stream)
+{
+    int64_t cols = 0;
+    int rc = check_kmean_args(k, mean, b, hk, sk, d, &cols);
+    if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
+    if (!k_out) return B200ATTN_ERR_NULL;
+    if (!aligned(k_out, 16)) return B200ATTN_ERR_ALIGN;
+    rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    // The mean's split must be the one k_smooth_mean takes (same bits): both grids are the SM
+    // count whenever one CTA of each kernel fits on an SM, which the occupancy query confirms.
+    const int grid = onepass_grid(k_mean_onepass, g_mean_grid);
+    const int grid2 = onepass_grid(k_mean_sub_onepass, g_mean_sub_grid);
+    if (grid2 != grid) return B200ATTN_ERR_CUDA;
+    return mean_pooled(k, mean, k_out, b, sk, cols, grid, static_cast<cudaStream_t>(stream));
 }
 
 // Device address of g_kmean_scratch on the current device, looked up once per device (the
@@ -526,7 +717,7 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     // partial the fold reads is written earlier in the same launch, and a flag counts only when
     // it carries this call's tag, so nothing needs clearing between calls.
     const Split sp = make_split(b, cols, sk, kNoAllocScratchFloats / (b * cols), grid_max);
-    return run_mean(k, mean, b, sk, cols, sp, scratch,
+    return run_mean(k, mean, nullptr, b, sk, cols, sp, scratch,
                     reinterpret_cast<unsigned long long*>(scratch + kNoAllocScratchFloats),
                     status, static_cast<cudaStream_t>(stream));
 }
@@ -553,7 +744,7 @@ extern "C" int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* r
     const int64_t n_samp = (sk + stride - 1) / stride;
     const Split sp = make_split(b, cols, n_samp, 1024, grid_max);
     const size_t part_bytes = (size_t)(b * sp.nchunks * 2 * cols) * sizeof(float);
-    const size_t nbytes = part_bytes + kMaxGrid * sizeof(unsigned long long);
+    const size_t nbytes = part_bytes + kFlagWords * sizeof(unsigned long long);
     char* scratch = nullptr;
     cudaMemPool_t pool = scratch_pool();
     if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), nbytes, pool, st) !=
@@ -604,9 +795,9 @@ extern "C" int k_smooth_sub(const void* k, const float* mean, void* k_out, int64
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
     const int64_t n = b * sk * (cols / 8);
-    int64_t blocks = (n + 4 * kSubThreads - 1) / (4 * kSubThreads);
+    int64_t blocks = (n + 8 * kSubThreads - 1) / (8 * kSubThreads);
     if (blocks > 148 * 8) blocks = 148 * 8;
     k_sub_kernel<<<(unsigned)blocks, kSubThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4*>(k), mean, static_cast<uint4*>(k_out), b * sk, sk, cols);
+        static_cast<const uint4*>(k), mean, static_cast<uint4*>(k_out), b, sk, cols / 8);
     return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
 }

@@ -236,6 +236,22 @@ B200ATTN_API int k_smooth_sub(const void* k, const float* mean, void* k_out, int
                  int64_t sk, int64_t d, void* stream);
 
 /*
+ * k_smooth_mean_sub -- k_smooth_mean and k_smooth_sub in one launch: the K channel mean and the
+ * smoothed K' = bf16_rne(float(K) - mean) that the attention pass then reads. Bit-identical to
+ * k_smooth_mean followed by k_smooth_sub with that mean. The cooperative launch sums the key
+ * chunks, folds the mean, and then writes K'. It re-reads K from L2 when K fits there.
+ *
+ *   k      device bf16 [b, sk, hk, d], 16-byte aligned. Read only.
+ *   mean   device fp32 [b, hk, d], 16-byte aligned. Fully written.
+ *   k_out  device bf16 [b, sk, hk, d], 16-byte aligned. Fully written. Must not overlap k or mean.
+ *   b, hk, sk, d  as in k_smooth_mean (sk > 0, d in {64, 128, 256}).
+ * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`
+ * (as k_smooth_mean). Concurrency as in the conventions above.
+ */
+B200ATTN_API int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int64_t b, int64_t hk,
+                                   int64_t sk, int64_t d, void* stream);
+
+/*
  * fp8_quantize -- E4M3 codes of a bf16 BSHD tensor with one fp32 scale per (batch, head), for the
  * FP8 attention recipe ("[HIP] Mha v4: run the K-smoothing gate as one HIP call", Summary: the
  * quantized recipes apply the K-smoothing gate before quantizing K; "Tune MHA config &

@@ -60,7 +60,7 @@ def test_noalloc_mean_size_limit():
     assert b2.lib.k_smooth_mean_noalloc(A, A, 1, 4, 16, 96, None) == 4
 
 
-@pytest.mark.parametrize("fn", ["k_smooth_mean", "k_smooth_sub"])
+@pytest.mark.parametrize("fn", ["k_smooth_mean", "k_smooth_sub", "k_smooth_mean_sub"])
 def test_k_mean_rejects(fn):
     f = getattr(b2.lib, fn)
 
@@ -74,7 +74,7 @@ def test_k_mean_rejects(fn):
     assert c(k=None) == 1 and c(m=None) == 1
     assert c(k=A + 8) == 5 and c(m=A + 4) == 5
     assert c(b=0) == 0 and c(hk=0) == 0
-    if fn == "k_smooth_sub":
+    if fn != "k_smooth_mean":
         assert f(A, A, None, 1, 2, 8, 64, None) == 1
         assert f(A, A, A + 2, 1, 2, 8, 64, None) == 5
 

@@ -206,6 +206,39 @@ def test_k_mean_small_shapes(b2, shape):
     assert np.all(np.abs(mg - m64) <= 1e-5 * scale)
 
 
+@pytest.mark.parametrize("shape", [None, (2, 3, 100, 64), (1, 1, 1, 128), (3, 5, 17, 256),
+                                   (1, 8, 4099, 128), (2, 40, 300, 256)])
+def test_k_mean_sub_fused_equals_two_calls(b2, shape):
+    """The one-launch mean and subtraction gives the bits of k_smooth_mean then k_smooth_sub, at
+    the K-mean workload's size (b1 hk16 4096 keys d256) and at small and ragged shapes."""
+    if shape is None:
+        c = config(4)
+        _, k, _ = config_inputs(c)
+        b, hk, sk, d = c["b"], c["hk"], c["sk"], c["dqk"]
+    else:
+        b, hk, sk, d = shape
+        _, k, _ = make_inputs(b, 1, hk, 1, sk, d, d, seed=78, kmean=True)
+    kd = k.cuda()
+    mean, ks = b2.k_smooth_mean_sub(kd)
+    mean_ref = b2.k_smooth_mean(kd)
+    ks_ref = b2.k_smooth_sub(kd, mean_ref)
+    torch.cuda.synchronize()
+    assert torch.equal(mean, mean_ref)
+    assert torch.equal(ks.view(torch.int16), ks_ref.view(torch.int16))
+    m64, m32 = oracle.k_mean(bf16_bits(k), b, hk, sk, d)
+    mg = mean.cpu().double().numpy()
+    scale = np.maximum(np.abs(m64), np.abs(k.double().numpy()).mean(axis=1))
+    assert np.all(np.abs(mg - m64) <= 1e-5 * scale)
+    if b * sk * hk * d <= 1 << 21:
+        # the oracle's subtraction (exact, one rounding to bf16) with the GPU's mean; the kernel
+        # rounds the fp32 difference to bf16, so a rare double rounding may move one unit
+        ref = oracle.k_sub(bf16_bits(k), mean.cpu().numpy().astype(np.float32), b, hk, sk, d)
+        got = ks.cpu().view(torch.int16).numpy().view(np.uint16)
+        gv, rv = oracle.bf16_to_f64(got), oracle.bf16_to_f64(ref)
+        assert np.all(np.abs(gv - rv) <= np.abs(rv) * 2.0 ** -7 + 2.0 ** -133)
+        assert np.mean(got == ref) > 0.999
+
+
 def test_kmean_leaves_output_invariant(b2):
     """Subtracting the K channel mean changes O only by rounding and shifts LSE by scale*q.mean."""
     c = config(4)

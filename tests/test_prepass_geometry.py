@@ -113,10 +113,23 @@ def test_fold_covers_every_column_and_chunk_once():
         ranges = [c for w in range(FOLD_WARPS)
                   for c in range(w * nchunks // FOLD_WARPS, (w + 1) * nchunks // FOLD_WARPS)]
         assert ranges == list(range(nchunks))
-        # gate fold: (batch, kv head) items, 512/d channel groups over the chunks
-        groups = THREADS // d
+        # gate fold: (batch, kv head) items; the head's 2d partial columns as d/2 float4 columns
+        # (d/4 of channel sums, then d/4 of sums of squares), 1024/d chunk groups
+        c4s = d // 2
+        groups = THREADS // c4s
+        assert groups * c4s == THREADS
         heads = [f for cta in range(grid) for f in range(cta, b * hk, grid)]
         assert sorted(heads) == list(range(b * hk))
+        for grp in range(groups):
+            got = []
+            for t in range(grp * c4s, (grp + 1) * c4s):
+                c4 = t % c4s
+                plane = 0 if c4 < d // 4 else 1
+                ch = 4 * (c4 - plane * (d // 4))
+                got += [(plane, ch + k) for k in range(4)]
+                # the float index of the column in the group's shared row: d sums, then d squares
+                assert [4 * c4 + k for k in range(4)] == [plane * d + ch + k for k in range(4)]
+            assert sorted(got) == [(pl, c) for pl in range(2) for c in range(d)]
         ranges = [c for g in range(groups)
                   for c in range(g * nchunks // groups, (g + 1) * nchunks // groups)]
         assert ranges == list(range(nchunks))
