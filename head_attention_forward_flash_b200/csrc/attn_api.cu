@@ -203,13 +203,16 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     // L2 or the kv heads are few, in weight-major order (all heads' heaviest units first), which
     // evens them out best; where many heads' K/V far exceed L2, head-major, so that the CTAs
     // working at the same time share a few heads' K/V. Equal-cost units (no causal mask, or a
-    // window band) take plain round robin, and so do packed sequences, whose unit costs depend
-    // on lengths the host does not see (measured: weight-major order was slower there).
+    // window band) take plain round robin. Packed sequences rank each sequence's units from its
+    // own last query tile (unit_info), so weight-major order hands out every sequence's k-th
+    // most expensive unit in round k.
     {
         const double kv_bytes =
             (double)(b * sk) * (double)hk * (double)(T::DQK + T::DV) * (double)T::EB;
-        if (!CAUSAL || VARLEN || (EXT && sh.window >= 0))
+        if (!CAUSAL || (EXT && sh.window >= 0))
             p.order = 0;
+        else if (VARLEN)
+            p.order = 2;
         else if (b * hk <= 16 || kv_bytes <= 64.0e6)
             p.order = 2;
         else

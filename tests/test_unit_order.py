@@ -89,3 +89,20 @@ def test_causal_balance_by_order():
         rr = per_cta_balance(b, hq, sq, 2, 0)
         wm = per_cta_balance(b, hq, sq, 2, 2)
         assert wm <= 1.02 < 1.1 < rr, (b, hq, sq, rr, wm)
+
+
+def test_packed_sequence_ranks():
+    """Packed sequences: rank k of a (sequence, head) is its query unit nqu_seq - 1 - k (the k-th
+    most expensive under a causal mask); ranks past the sequence's units are empty. Every unit
+    of every sequence gets exactly one rank."""
+    rnd = random.Random(3)
+    for _ in range(200):
+        NT = rnd.choice([1, 2])
+        lens = [rnd.randint(0, 3000) for _ in range(rnd.randint(1, 9))]
+        nqu = max(1, (max(lens) + NT * 128 - 1) // (NT * 128))
+        for sq in lens:
+            nqu_seq = (sq + NT * 128 - 1) // (NT * 128)
+            q0s = [(nqu_seq - 1 - k) * NT * 128 if k < nqu_seq else sq for k in range(nqu)]
+            busy = [q for q in q0s if q < sq]
+            assert sorted(busy) == list(range(0, sq, NT * 128))
+            assert busy == sorted(busy, reverse=True)  # most keys first
