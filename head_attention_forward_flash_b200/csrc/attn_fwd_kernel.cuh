@@ -214,33 +214,21 @@ struct UnitInfo {
     int n_blocks;   // key blocks j_begin .. n_blocks-1 are visited
     int mask_lo;    // blocks < mask_lo need the window's lower per-key bound
     int mask_from;  // blocks >= mask_from need the per-key mask (causal diagonal, ragged tail)
-    // Per query tile (PT: the pipelined two-tile layout, whose tiles have their own issuers and
-    // score buffers): the key blocks tile tt visits, [tj_begin, tj_end) within the unit's range,
-    // and its mask bounds. Without PT every tile takes the unit's range and bounds.
-    // (Read through the accessors: a runtime index into these arrays would put the whole
-    // struct in local memory.)
-    int tj_begin[2], tj_end[2], tmask_lo[2], tmask_from[2];
-    __device__ __forceinline__ int tb(int tt) const { return tt ? tj_begin[1] : tj_begin[0]; }
-    __device__ __forceinline__ int te(int tt) const { return tt ? tj_end[1] : tj_end[0]; }
-    __device__ __forceinline__ int tlo(int tt) const { return tt ? tmask_lo[1] : tmask_lo[0]; }
-    __device__ __forceinline__ int tfrom(int tt) const {
-        return tt ? tmask_from[1] : tmask_from[0];
-    }
 };
 
-template <int BN, int NT, bool CAUSAL, bool VARLEN, bool EXT, bool PT>
+template <int BN, int NT, bool CAUSAL, bool VARLEN, bool EXT>
 __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
 {
     UnitInfo t;
     const uint32_t uu = (uint32_t)u;
     const uint32_t bh = fast_div(uu, p.div_nqu);
-    const uint32_t rank = uu - bh * p.div_nqu.d;  // within a head: rank 0 sees the most keys
+    const uint32_t qu = p.div_nqu.d - 1 - (uu - bh * p.div_nqu.d);  // within a head: most keys first
     const uint32_t bi = fast_div(bh, p.div_hq);
     const uint32_t h = bh - bi * p.div_hq.d;
     t.bi = bi;
     t.h = h;
     t.g = fast_div(h, p.div_group);
-    t.q0 = (int64_t)(p.div_nqu.d - 1 - rank) * (NT * 128);
+    t.q0 = qu * (NT * 128);
     if (VARLEN) {
         // offsets clamped into the packed tensors, so no row outside them is ever addressed
         int64_t qs = __ldg(p.cu_q + bi), qe = __ldg(p.cu_q + bi + 1);
@@ -253,8 +241,9 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
         t.sk = ke - ks;
         // ranks count from this sequence's own last query tile, so that rank k of every
         // sequence is its k-th most expensive unit; ranks past its tiles are empty
+        const int64_t rank = (int64_t)(p.div_nqu.d - 1 - qu);
         const int64_t nqu_seq = (t.sq + NT * 128 - 1) / (NT * 128);
-        t.q0 = (int64_t)rank < nqu_seq ? (nqu_seq - 1 - (int64_t)rank) * (NT * 128) : t.sq;
+        t.q0 = rank < nqu_seq ? (nqu_seq - 1 - rank) * (NT * 128) : t.sq;
         t.qrow = qs;
         t.krow = ks;
         t.obase = qs;
@@ -271,7 +260,6 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
     }
     t.j_begin = 0;
     t.mask_lo = 0;
-    for (int tt = 0; tt < 2; ++tt) t.tj_begin[tt] = t.tj_end[tt] = t.tmask_lo[tt] = t.tmask_from[tt] = 0;
     if (t.q0 >= t.sq) {  // (packed sequences) no query row of this sequence here
         t.n_blocks = 0;
         t.mask_from = 0;
@@ -300,43 +288,6 @@ __device__ __forceinline__ UnitInfo unit_info(const AttnParams& p, int64_t u)
         jb = jb < t.n_blocks ? jb : t.n_blocks;
         t.j_begin = (int)jb;
         t.mask_lo = (int)(lo_last <= 0 ? 0 : (lo_last + BN - 1) / BN);
-    }
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt) {
-        int jb = t.j_begin, nb = t.n_blocks, mlo = t.mask_lo, mfrom = t.mask_from;
-        if (PT) {
-            const int64_t r0 = t.q0 + tt * 128;  // the tile's first and last query rows
-            const int64_t r1 = (r0 + 127 < t.sq - 1) ? r0 + 127 : t.sq - 1;
-            if (r0 > r1) {
-                nb = jb;  // no query row here (a short last tile)
-            } else {
-                if (CAUSAL) {
-                    const int64_t last_key = r1 + t.sk - t.sq;
-                    const int64_t nbt = last_key < 0 ? 0 : last_key / BN + 1;
-                    nb = nbt < nb ? (int)nbt : nb;
-                    const int64_t first_lim = r0 + t.sk - t.sq + 1;
-                    int64_t full = first_lim <= 0 ? 0 : first_lim / BN;
-                    full = full < t.sk / BN ? full : t.sk / BN;
-                    mfrom = full < nb ? (int)full : nb;
-                }
-                if (EXT && p.window >= 0) {
-                    const int64_t lo_first = r0 + t.sk - t.sq - p.window;
-                    const int64_t jbt = lo_first <= 0 ? 0 : lo_first / BN;
-                    jb = jbt > jb ? (int)(jbt < nb ? jbt : nb) : jb;
-                    const int64_t lo_last = r1 + t.sk - t.sq - p.window;
-                    mlo = (int)(lo_last <= 0 ? 0 : (lo_last + BN - 1) / BN);
-                }
-            }
-            if (nb <= jb) {  // no allowed key for any row of the tile: one masked block
-                jb = t.j_begin;
-                nb = jb + 1;
-                mfrom = jb;
-            }
-        }
-        t.tj_begin[tt] = jb;
-        t.tj_end[tt] = nb;
-        t.tmask_lo[tt] = mlo;
-        t.tmask_from[tt] = mfrom;
     }
     return t;
 }
@@ -407,9 +358,6 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
 {
     constexpr int BN = T::BN;
     constexpr int NT = T::NT;
-    // per-tile key ranges (see UnitInfo), computed where they are used: the issuers and the
-    // softmax (the producer and the epilogue need only the unit's range)
-    constexpr bool PT = T::PIPE;
     // O through the staging tile and TMA stores, except for packed sequences, where a store box
     // could reach into the next sequence's rows
     constexpr bool OTMA = T::O_TMA && !VARLEN;
@@ -517,7 +465,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         for (;; ++r) {
             const int64_t u = unit_of(r);
             if (u < 0) return -1;
-            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, false>(p, u);
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
             if (t.n_blocks > t.j_begin) return r;
         }
     };
@@ -536,7 +484,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int q_cnt = 0;       // Q units issued
             bool ok = true;
             auto load_q = [&](int64_t u) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, false>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 if (!mbar_wait(bar_q_empty, (uint32_t)(q_cnt & 1) ^ 1u, wc, kErrTimeout)) {
                     ok = false;
                     return;
@@ -583,7 +531,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
             int64_t r = busy_from(0);
             if (r >= 0) load_q(unit_of(r));
             while (r >= 0 && ok) {
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, false>(p, unit_of(r));
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, unit_of(r));
                 const int64_t rn = busy_from(r + 1);
                 const int64_t un = rn >= 0 ? unit_of(rn) : -1;
                 // PIPE: each tile's issuer takes K(j+1) before V(j), as with one tile
@@ -640,12 +588,9 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 return __all_sync(FULL, mbar_wait(bar, parity, wc, kErrTimeout));
             };
             // Q K^T of tile tt's current block into score buffer sb. Every issuer takes K(j)
-            // itself: the slot is freed when all NT issuers have committed kempty. With
-            // compute = false (PIPE: a block outside this tile's key range, see UnitInfo) the
-            // slot is released unread, once its load has landed: arriving earlier could complete
-            // the slot's previous phase, still owed by the other tile.
-            auto qk = [&](int sb, bool first, int tt, bool last_item, bool compute) {
-                if (T::Q_TMEM && first && compute) {  // this tile's Q of the new unit in TMEM
+            // itself: the slot is freed when all NT issuers have committed kempty.
+            auto qk = [&](int sb, bool first, int tt, bool last_item) {
+                if (T::Q_TMEM && first) {  // this tile's Q of the new unit must be in TMEM
                     if (!wait_all(bar_q_tmem(tt), (uint32_t)(units & 1))) {
                         ok = false;
                         return;
@@ -660,17 +605,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     return;
                 }
                 if (elect_one()) {
-                    if (compute) {
-                        issue_qk_mmas<T>(tmem + (uint32_t)sb * BN,
-                                         T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
-                                                   : q_stage + tt * T::Q_TILE_BYTES,
-                                         k_slots + kslot * T::K_TILE_BYTES, p.idesc_qk);
-                        tc_commit(bar_s_full(sb));
-                        tc_commit(bar_kempty(kslot));
-                        if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
-                    } else {
-                        mbar_arrive(bar_kempty(kslot));
-                    }
+                    issue_qk_mmas<T>(tmem + (uint32_t)sb * BN,
+                                     T::Q_TMEM ? tmem + T::Q_COL0 + tt * (T::DQK / 2)
+                                               : q_stage + tt * T::Q_TILE_BYTES,
+                                     k_slots + kslot * T::K_TILE_BYTES, p.idesc_qk);
+                    tc_commit(bar_s_full(sb));
+                    tc_commit(bar_kempty(kslot));
+                    if (!T::Q_TMEM && last_item) tc_commit(bar_q_empty);
                 }
                 __syncwarp();
             };
@@ -702,33 +643,16 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 }
                 __syncwarp();
             };
-            // PIPE: the V slot of a block outside this tile's key range, released unread once its
-            // load has landed (as qk with compute = false does for K)
-            auto skip_v = [&]() {
-                const int vslot = vq % NV;
-                const uint32_t phase = (uint32_t)(vq / NV) & 1u;
-                ++vq;
-                if (!wait_all(bar_vfull(vslot), phase)) {
-                    ok = false;
-                    return;
-                }
-                if (elect_one()) mbar_arrive(bar_vempty(vslot));
-                __syncwarp();
-            };
             // NT = 1 and PIPE: the P V of each block is issued after the next block's Q K^T (also
             // across units), so the tensor core computes the next S while the softmax works on
-            // this one. The pending step may be a V slot to release unread (pend_skip).
-            bool pend = false, pend_last = false, pend_first = false, pend_skip = false;
+            // this one.
+            bool pend = false, pend_last = false, pend_first = false;
             int pend_u = 0, pend_sb = 0;
             uint32_t pend_ph = 0;
-            auto settle = [&](int tt) {
-                if (pend_skip) skip_v();
-                else pv(pend_sb, pend_ph, pend_first, tt, pend_last, pend_u);
-            };
             for (int64_t r = 0; ok; ++r) {
                 const int64_t u = unit_of(r);
                 if (u < 0) break;
-                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, PT>(p, u);
+                const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
                 if (t.n_blocks <= t.j_begin) continue;
                 if (!T::Q_TMEM) {  // the unit's Q in the staging buffer (read by the MMA)
                     if (!wait_all(bar_q_full, (uint32_t)(units & 1))) {
@@ -737,32 +661,28 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     }
                     tc_fence_after_sync();
                 }
-                for (int j = t.j_begin; j < t.n_blocks && ok; ++j) {
+                for (int j = t.j_begin; j < t.n_blocks && ok; ++j, ++jg) {
+                    const bool first = j == t.j_begin, last = j == t.n_blocks - 1;
                     if constexpr (NT == 2 && !T::PIPE) {
-                        const bool first = j == t.j_begin, last = j == t.n_blocks - 1;
-                        qk(my_tt, first, my_tt, last, true);
+                        qk(my_tt, first, my_tt, last);
                         if (ok) pv(my_tt, (uint32_t)jg & 1u, first, my_tt, last, units);
-                        ++jg;
                     } else {
                         const int tt = T::PIPE ? my_tt : 0;
-                        const int jb = t.tb(tt), je = t.te(tt);
-                        const bool mine = j >= jb && j < je;
-                        qk(sbuf_of(jg, tt), j == jb, tt, j == je - 1, mine);
+                        qk(sbuf_of(jg, tt), first, tt, last);
                         if (!ok) break;
-                        if (pend) settle(tt);
+                        if (pend) pv(pend_sb, pend_ph, pend_first, tt, pend_last, pend_u);
                         pend = true;
-                        pend_skip = !mine;
                         pend_sb = sbuf_of(jg, tt);
                         pend_ph = sphase_of(jg);
-                        pend_first = j == jb;
-                        pend_last = j == je - 1;
+                        pend_first = first;
+                        pend_last = last;
                         pend_u = units;
-                        if (mine) ++jg;
                     }
                 }
                 ++units;
             }
-            if ((NT == 1 || T::PIPE) && ok && pend) settle(T::PIPE ? my_tt : 0);
+            if ((NT == 1 || T::PIPE) && ok && pend)
+                pv(pend_sb, pend_ph, pend_first, T::PIPE ? my_tt : 0, pend_last, pend_u);
             // drain every MMA this warp issued before teardown
             if (elect_one()) tc_commit(bar_mma_done);
             __syncwarp();
@@ -814,7 +734,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         // Epilogue of tile tt of busy unit number uidx: wait for that tile's last P V, read this
         // row of its O from TMEM (then free the accumulator), write O / l in bf16 and the LSE.
         auto epilogue = [&](int64_t u, int tt, float m_ref, float l, int uidx) -> bool {
-            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, false>(p, u);
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
             if (!__all_sync(FULL,
                             mbar_wait(bar_o_full(tt), (uint32_t)(uidx & 1), wc, kErrTimeout)))
                 return false;
@@ -1039,7 +959,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         for (int64_t r = 0; ok; ++r) {
             const int64_t u = unit_of(r);
             if (u < 0) break;
-            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT, PT>(p, u);
+            const UnitInfo t = unit_info<BN, NT, CAUSAL, VARLEN, EXT>(p, u);
             if (t.n_blocks <= t.j_begin) {  // no key for any row of this unit: O = 0, LSE = -inf
                 // (or the head's sink logit)
 #pragma unroll
@@ -1079,10 +999,8 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                 m_ref[k] = sink_l2;
                 l[k] = has_sink ? 1.f : 0.f;
             }
-            // this warpgroup's tile range (NSM = 2: one tile; NSM = 1: the unit's range)
-            const int tw = tile_of(0);
-            j_begin = t.tb(tw);
-            const int n_blocks = t.te(tw), mask_lo = t.tlo(tw), mask_from = t.tfrom(tw);
+            j_begin = t.j_begin;
+            const int n_blocks = t.n_blocks, mask_lo = t.mask_lo, mask_from = t.mask_from;
 
             for (int j = j_begin; j < n_blocks && ok; ++j, ++jg) {
 #pragma unroll

@@ -38,8 +38,6 @@ MUTANTS = {
     "s_full_wrong_parity": "the softmax waits for the wrong phase of its score buffer",
     "p_full_early": "the softmax hands over P before writing it",
     "kempty_wrong_parity": "the producer waits for the wrong phase of a free K slot",
-    "skip_without_kfull_wait": "in the pipelined layout, an issuer releases the K slot of a block "
-                               "outside its tile's range without waiting for that K to land",
 }
 
 
@@ -92,9 +90,7 @@ class Bar:
 
 
 def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
-    """One random schedule over `units` (dicts with 'id' and 'n' = key blocks, 0 = skipped; with
-    `pipe`, optionally 'rng' = per tile the blocks [lo, hi) it computes, as the kernel's per-tile
-    key ranges: the tile's issuer releases the other blocks' K and V slots unread)."""
+    """One random schedule over `units` (dicts with 'id' and 'n' = key blocks, 0 = skipped)."""
     rnd = random.Random(seed)
     clock = [0]
     kfull = [Bar(1, f"kfull{i}", clock) for i in range(NK)]
@@ -136,9 +132,6 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
     landings = []       # TMA loads in flight
     tensor = []         # issued MMAs and commits: (issuer, kind, x); in order per issuer
     busy = [u for u in units if u["n"] > 0]
-
-    def rng(u, tt):
-        return u["rng"][tt] if (pipe and "rng" in u) else (0, u["n"])
     current = [None]  # the role being stepped
     waits = {}        # role -> (barrier, parity, completed phases) it last blocked on
 
@@ -231,19 +224,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                     b[h] = (item, "S")
             return op
 
-        def skip(kind):  # release a slot of a block outside this tile's range, unread
-            slots, full, empty, nslot = (("k", kfull, kempty, NK) if kind == "k"
-                                         else ("v", vfull, vempty, NV))
-            s = st[slots] % nslot
-            ph = (st[slots] // nslot) & 1
-            st[slots] += 1
-            if not (kind == "k" and mutant == "skip_without_kfull_wait"):
-                yield from wait(full[s], ph)
-            empty[s].arrive(1)
-            yield True
-
         def qk(u, j, tt, sb, last):  # a whole Q K^T (both key halves) into score buffer sb
-            if q_tmem and j == rng(u, tt)[0]:
+            if q_tmem and j == 0:
                 yield from wait(q_tmem_bar[tt], st["units"] & 1)
             yield from take_k()
             s = st["kslot"]
@@ -256,9 +238,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
 
         def pv(sb, ph, u, j, tt, last_block, uidx):
             item = (u["id"], j, tt)
-            rel = j - rng(u, tt)[0]  # blocks of this tile before this one
             yield from wait(p_full[sb], ph)
-            if rel == 0 and uidx > 0 and mutant != "no_o_free_wait":
+            if j == 0 and uidx > 0 and mutant != "no_o_free_wait":
                 yield from wait(o_free[tt], (uidx - 1) & 1)
             s = st["v"] % NV
             ph = (st["v"] // NV) & 1
@@ -271,11 +252,11 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                 check(lo == (item, "P"), f"P V {item} reads {lo}")
                 sbuf[sb]["lo"] = (item, "consumed")
                 o = obuf.get(item[2])
-                if rel == 0:
+                if item[1] == 0:
                     check(o is None or o[2] == "read", f"P V {item} overwrites unread O {o}")
                     obuf[item[2]] = [item[0], 1, "acc"]
                 else:
-                    check(o[0] == item[0] and o[1] == rel, f"P V {item} finds O {o}")
+                    check(o[0] == item[0] and o[1] == item[1], f"P V {item} finds O {o}")
                     o[1] += 1
             Q.append(("op", op))
             if NT == 1 or pipe:
@@ -285,40 +266,27 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                 Q.append(("commit", o_full[tt]))
             yield True
 
-        def settle(pend):
-            if pend[0] == "skip":
-                yield from skip("v")
-            else:
-                yield from pv(*pend)
-
         pend = None
         jg = 0
         for u in busy:
             if not q_tmem:
                 yield from wait(q_full, st["units"] & 1)
             for j in range(u["n"]):
+                last = j == u["n"] - 1
                 for tt in tiles:
-                    lo, hi = rng(u, tt)
-                    last = j == hi - 1
                     sb = sbuf_of(jg, tt)
                     if NT == 2 and not pipe:
                         yield from qk(u, j, tt, sb, last)
                         yield from pv(sb, sphase_of(jg), u, j, tt, last, st["units"])
-                        jg += 1
-                    elif not lo <= j < hi:
-                        yield from skip("k")
-                        if pend:
-                            yield from settle(pend)
-                        pend = ("skip",)
                     else:
                         yield from qk(u, j, tt, sb, last)
                         if pend:
-                            yield from settle(pend)
+                            yield from pv(*pend)
                         pend = (sb, sphase_of(jg), u, j, tt, last, st["units"])
-                        jg += 1
+                jg += 1
             st["units"] += 1
         if pend:
-            yield from settle(pend)
+            yield from pv(*pend)
         Q.append(("commit", mma_done))
         yield True
 
@@ -337,8 +305,7 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
         def epilogue(u, tt, uidx):
             yield from wait(o_full[tt], uidx & 1)
             o = obuf[tt]
-            lo, hi = rng(u, tt)
-            check(o[0] == u["id"] and o[1] == hi - lo and o[2] == "acc",
+            check(o[0] == u["id"] and o[1] == u["n"] and o[2] == "acc",
                   f"epilogue of unit {u['id']} tile {tt} finds O {o}")
             o[2] = "read"
             o_free[tt].arrive(128)
@@ -353,9 +320,6 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
             nxt = busy[ui + 1] if ui + 1 < len(busy) else None
             for j in range(u["n"]):
                 for tt in tiles:
-                    lo, hi = rng(u, tt)
-                    if not lo <= j < hi:
-                        continue
                     sb = sbuf_of(jg, tt)
                     item = (u["id"], j, tt)
                     if NT == 2 and not pipe:  # the two tiles' softmax take turns, block by block
@@ -365,17 +329,17 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                             yield from wait(p_full[1], (jg - 1) & 1)
                     parity = sphase_of(jg) ^ (1 if mutant == "s_full_wrong_parity" else 0)
                     yield from wait(s_full[sb], parity)
-                    if q_tmem and j == hi - 1 and nxt:
+                    if q_tmem and j == u["n"] - 1 and nxt:
                         yield from copy_q(ui + 1, tt, nxt["id"])
                     b = sbuf[sb]
                     check(b["lo"] == (item, "S") and b["hi"] == (item, "S"),
                           f"softmax of {item} reads {b}")
                     b["lo"], b["hi"] = (item, "read"), (item, "read")
-                    if j > lo and rnd.random() < 0.3:  # the running max grew: rescale O
+                    if j > 0 and rnd.random() < 0.3:  # the running max grew: rescale O
                         if (NT == 1 or pipe) and mutant != "no_pv_done_wait":
                             yield from wait(pv_done[tt], (jg - 1) & 1)
                         o = obuf.get(tt)
-                        check(o is not None and o[0] == u["id"] and o[1] == j - lo,
+                        check(o is not None and o[0] == u["id"] and o[1] == j,
                               f"rescale of {item} finds O {o}")
                     if mutant == "p_full_early":
                         p_full[sb].arrive(128)
@@ -385,9 +349,9 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                         yield True
                         b["lo"] = (item, "P")
                         p_full[sb].arrive(128)
-                    if j == lo and pend:
+                    if j == 0 and pend:
                         yield from epilogue(pend[0], tt, pend[1])
-                    jg += 1
+                jg += 1
             pend = (u, ui)
         if pend:
             for tt in tiles:
@@ -449,18 +413,7 @@ LAYOUTS = [(2, 2, True, 8, 8, True), (2, 2, False, 3, 2, False), (2, 2, False, 2
            (2, 2, False, 2, 2, True), (2, 2, True, 5, 5, False)]
 
 
-def random_units(rnd, ranges=False):
-    """Random units; with `ranges`, per-tile key ranges as the pipelined layout's (a nonempty
-    [lo, hi) of [0, n) for each of two tiles, tile 0's starting first, tile 1's ending last)."""
+def random_units(rnd):
     n = rnd.randint(1, 6)
-    units = [{"id": i, "n": rnd.choice([0, 1, 1, 2, 3, 5]) if rnd.random() < 0.5
-              else rnd.randint(1, 4)} for i in range(n)]
-    if ranges:
-        for u in units:
-            n = u["n"]
-            if n == 0:
-                continue
-            hi0 = rnd.randint(1, n)
-            lo1 = rnd.randint(0, n - 1)
-            u["rng"] = [(0, hi0), (lo1, n)]
-    return units
+    return [{"id": i, "n": rnd.choice([0, 1, 1, 2, 3, 5]) if rnd.random() < 0.5
+             else rnd.randint(1, 4)} for i in range(n)]

@@ -11,9 +11,6 @@ j >= i + sk - sq - window with a window) and checks:
     either end);
   - every block the kernel leaves unmasked is allowed for every key and every real row;
   - a unit with no visited block has no allowed key at all.
-The pipelined two-tile layout narrows the range per query tile (tile_ranges below); the same
-checks hold per tile within the unit's range, and a tile whose rows allow no key (or that has no
-row) visits exactly one block, masked.
 """
 import random
 
@@ -49,37 +46,6 @@ def unit_ranges(q0, sq, sk, NT, BN, causal, window):
     return j_begin, n_blocks, mask_lo, mask_from
 
 
-def tile_ranges(q0, sq, sk, NT, BN, causal, window, unit):
-    """unit_info's per-tile ranges (the pipelined layout): per tile (jb, nb, mask_lo, mask_from)."""
-    j_begin, n_blocks, mask_lo, mask_from = unit
-    out = []
-    for tt in range(NT):
-        jb, nb, mlo, mfrom = j_begin, n_blocks, mask_lo, mask_from
-        r0 = q0 + tt * 128
-        r1 = min(r0 + 127, sq - 1)
-        if r0 > r1:
-            nb = jb
-        else:
-            if causal:
-                last_key = r1 + sk - sq
-                nbt = 0 if last_key < 0 else last_key // BN + 1
-                nb = min(nb, nbt)
-                first_lim = r0 + sk - sq + 1
-                full = 0 if first_lim <= 0 else first_lim // BN
-                full = min(full, sk // BN)
-                mfrom = min(full, nb)
-            if window >= 0:
-                lo_first = r0 + sk - sq - window
-                jbt = 0 if lo_first <= 0 else lo_first // BN
-                jb = min(jbt, nb) if jbt > jb else jb
-                lo_last = r1 + sk - sq - window
-                mlo = 0 if lo_last <= 0 else (lo_last + BN - 1) // BN
-        if nb <= jb:
-            jb, nb, mfrom = j_begin, j_begin + 1, j_begin
-        out.append((jb, nb, mlo, mfrom))
-    return out
-
-
 def allowed(q0, sq, sk, NT, causal, window):
     rows = np.arange(q0, min(q0 + NT * 128, sq))[:, None]
     keys = np.arange(sk)[None, :]
@@ -109,23 +75,6 @@ def check_shape(sq, sk, NT, BN, causal, window):
                 continue
             lo, hi = b * BN, (b + 1) * BN
             assert hi <= sk and ok[:, lo:hi].all(), f"unmasked block {b} is not all allowed {ctx}"
-        if NT != 2:
-            continue
-        for tt, (tb, te, tlo, tfrom) in enumerate(tile_ranges(q0, sq, sk, NT, BN, causal, window,
-                                                              (jb, nb, mlo, mfrom))):
-            tok = ok[tt * 128:(tt + 1) * 128]
-            tblocks = np.nonzero(tok.any(axis=0))[0] // BN if tok.shape[0] else np.array([], int)
-            tctx = ctx + (tt, (tb, te, tlo, tfrom))
-            assert jb <= tb < te <= nb, f"tile range outside the unit's {tctx}"
-            if tblocks.size == 0:
-                assert (tb, te, tfrom) == (jb, jb + 1, jb), f"keyless tile not one masked block {tctx}"
-                continue
-            assert tblocks.min() == tb and tblocks.max() == te - 1, f"tile range wrong {tctx}"
-            for b in range(tb, te):
-                if (window >= 0 and b < tlo) or b >= tfrom:
-                    continue
-                lo, hi = b * BN, (b + 1) * BN
-                assert hi <= sk and tok[:, lo:hi].all(), f"unmasked tile block {b} {tctx}"
 
 
 @pytest.mark.parametrize("seed", range(6))
