@@ -324,9 +324,9 @@ def run_gpu(args):
     window = c["window"] if c.get("window") is not None else -1
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
-    # K-mean workload: k_smooth_mean_sub + attention; FP8: the gate, two kernels per quantised
+    # K-mean workload: k_smooth_mean_sub + attention; FP8: the gate, one launch per quantised
     # tensor, attention
-    launches_per_step = 2 if c["kmean"] else (8 if fp8 else 1)
+    launches_per_step = 2 if c["kmean"] else (5 if fp8 else 1)
 
     def step():
         kk = k
@@ -643,7 +643,7 @@ def run_gpu(args):
             stride = (c["sk"] + 2047) // 2048
             sampled = c["b"] * ((c["sk"] + stride - 1) // stride) * c["hk"] * c["dqk"] * 2
             pre_bytes = sampled + 5 * (n_q + n_k + n_v)
-            kernels = "k_gate_onepass, 3 x (fp8_amax_partial, fp8_convert)"
+            kernels = "k_gate_onepass, 3 x fp8_quant_onepass"
         else:
             pre_bytes = 3 * n_k * 2
             kernels = "k_mean_sub_onepass (K mean and K - mean in one launch)"

@@ -3,30 +3,41 @@
 // "[HIP] Mha v4: run the K-smoothing gate as one HIP call", Summary: smoothing before K is
 // quantized).
 //
-// Two passes over x, both HBM-bound. A head's slice x[bi, :, hh, :] is s rows of d contiguous
-// elements, 16-byte loads with one 8-element group per thread. (1) Every CTA takes one
-// (batch, head) and a chunk of its rows and writes the chunk's amax to a partial. (2) Every CTA
-// folds its head's partials (max is exact, so any order gives the same amax), derives the
-// factor 448 / amax, converts its rows and writes 8 codes per thread; the first chunk's CTA also
-// writes the descale. Both passes compute x' = x - mean with the same fp32 subtraction, so the
-// codes are exactly those of the definition in the header.
+// Two passes over x, both HBM-bound, in ONE cooperative launch (every CTA resident). A head's
+// slice x[bi, :, hh, :] is s rows of d contiguous elements, 16-byte loads with one 8-element
+// group per thread. Items are (batch, head, chunk of rows).
+//   pass 1  each CTA takes its item's amax;
+//   pass 2  it derives the factor 448 / amax of the item's head and converts the item's rows
+//           (re-read, from L2 where they are still cached), 8 codes per thread; the head's first
+//           chunk also writes the descale.
+// With several chunks per head (few heads), every CTA holds at most one item; the chunk amaxes go
+// to partials, and pass 2 starts once every CTA has published its partial (grid_sync.cuh) and
+// folds its head's partials (max is exact, so any order gives the same amax). With one chunk per
+// head (many heads), a CTA takes its items one after another and needs no grid-wide wait. Both
+// passes compute x' = x - mean with the same fp32 subtraction, so the codes are exactly those of
+// the definition in the header.
 #include <cfloat>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
+#include "grid_sync.cuh"
 #include "host_common.h"
 
 namespace b200 {
 namespace {
 
-constexpr int kQThreads = 256;
-constexpr int kQTargetCtas = 4 * 148;  // about four waves on the 148 SMs
+constexpr int kQThreads = 512;
+constexpr int kQMaxChunks = 64;   // chunks per head slice at most (the fold: one load per thread)
+constexpr int kQMaxGrid = 1024;   // CTAs of the launch at most (flag words)
+constexpr uint64_t kQTagMagic = 0x6670387175ULL << 24;  // high bits of every flag tag
 
-// The 8 elements of a 16-byte bf16 group, minus the mean when given (one fp32 subtraction).
-__device__ __forceinline__ void load_group(const uint4* src, const float* m, float (&x)[8])
+// The 8 elements of a 16-byte bf16 group (already loaded), minus the mean when given (one fp32
+// subtraction).
+__device__ __forceinline__ void unpack_group(const uint4& v, const float* m, float (&x)[8])
 {
-    const uint4 v = __ldg(src);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
@@ -39,13 +50,23 @@ __device__ __forceinline__ void load_group(const uint4* src, const float* m, flo
     }
 }
 
-// Problem geometry of both passes. Grid: x = (batch, head) slice bh = bi * h + hh, y = row
-// chunk. Thread t of a CTA takes 16-byte group gi = t % G of a row and rows t / G, t / G + R,
-// ... of its chunk, with G = d / 8 groups per row and R = 256 / G rows per step.
-struct QGeom {
-    int64_t s, h, d8;  // rows, heads, 16-byte groups per row
+// Problem geometry. Item it = (slice bh = bi * h + hh, chunk it % nch). Thread t of a CTA takes
+// 16-byte group gi = t % G of a row and rows t / G, t / G + R, ... of its chunk, with G = d / 8
+// groups per row and R = 512 / G rows per step.
+struct QOnePass {
+    const uint4* x;
+    const float* mean;  // [b, h, d] or null
+    uint2* x8;
+    float* descale;
+    float* partial;               // [n_items] chunk amaxes (nch > 1)
+    unsigned long long* flags;    // [gridDim.x] flag words, then the go word at kQMaxGrid
+    int64_t s, h, d8;             // rows, heads, 16-byte groups per row
     int64_t rows_per_chunk;
-    int nch;           // row chunks per head slice
+    int nch;                      // row chunks per head slice
+    int64_t n_items;              // b * h * nch
+    unsigned long long tag;
+    int* status;
+    unsigned long long timeout_ns;
 };
 
 // The 8 mean values of group gi of head slice bh (mean is [b, h, d] fp32).
@@ -58,12 +79,13 @@ __device__ __forceinline__ void head_mean(const float* mean, int64_t bh, int64_t
     mv[4] = c.x; mv[5] = c.y; mv[6] = c.z; mv[7] = c.w;
 }
 
-// Max over the CTA's 256 threads (non-negative inputs); the result is valid in warp 0.
+// Max over the CTA's threads (non-negative inputs); the result is valid in warp 0.
 __device__ __forceinline__ float block_max(float v, float* red)
 {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();  // red is free (a previous use has been read)
     if (lane == 0) red[warp] = v;
     __syncthreads();
     if (warp == 0) {
@@ -74,86 +96,152 @@ __device__ __forceinline__ float block_max(float v, float* red)
     return v;  // valid in warp 0
 }
 
-// Pass 1: partial[bh * nch + chunk] = max |x'| over the chunk's rows of head slice bh.
-__global__ void __launch_bounds__(kQThreads)
-    fp8_amax_partial(const uint4* __restrict__ x, const float* __restrict__ mean,
-                     float* __restrict__ partial, QGeom g)
+// max |x'| over the rows [s0, s1) of slice bh that this thread takes (twelve 16-byte loads in
+// flight).
+__device__ __forceinline__ float chunk_amax(const QOnePass& a, int64_t bh, int64_t s0, int64_t s1)
 {
-    __shared__ float red[kQThreads / 32];
-    const int64_t bh = blockIdx.x;  // bi * h + hh
-    const int chunk = blockIdx.y;
-    const int G = (int)g.d8;
+    const int G = (int)a.d8;
     const int gi = threadIdx.x % G;
     const int R = kQThreads / G;
-    const int64_t bi = bh / g.h, hh = bh - bi * g.h;
+    const int64_t bi = bh / a.h, hh = bh - bi * a.h;
     float mv[8];
-    if (mean) head_mean(mean, bh, g.d8, gi, mv);
-    const int64_t s0 = (int64_t)chunk * g.rows_per_chunk;
-    const int64_t s1 = s0 + g.rows_per_chunk < g.s ? s0 + g.rows_per_chunk : g.s;
-    const int64_t row_stride = g.h * g.d8;  // uint4 per sequence row
-    const uint4* base = x + (bi * g.s * g.h + hh) * g.d8 + gi;
+    if (a.mean) head_mean(a.mean, bh, a.d8, gi, mv);
+    const int64_t row_stride = a.h * a.d8;  // uint4 per sequence row
+    const uint4* base = a.x + (bi * a.s * a.h + hh) * a.d8 + gi;
     float m = 0.f;
     int64_t r = s0 + threadIdx.x / G;
-    for (; r + 3 * R < s1; r += 4 * R) {  // four 16-byte loads in flight
-        float a[8], b[8], c[8], e[8];
-        load_group(base + r * row_stride, mean ? mv : nullptr, a);
-        load_group(base + (r + R) * row_stride, mean ? mv : nullptr, b);
-        load_group(base + (r + 2 * R) * row_stride, mean ? mv : nullptr, c);
-        load_group(base + (r + 3 * R) * row_stride, mean ? mv : nullptr, e);
+    for (; r + 11 * R < s1; r += 12 * R) {
+        uint4 raw[12];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            m = fmaxf(fmaxf(m, fmaxf(fabsf(a[k]), fabsf(b[k]))), fmaxf(fabsf(c[k]), fabsf(e[k])));
+        for (int e = 0; e < 12; ++e) raw[e] = __ldg(base + (r + e * R) * row_stride);
+#pragma unroll
+        for (int e = 0; e < 12; ++e) {
+            float v[8];
+            unpack_group(raw[e], a.mean ? mv : nullptr, v);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
+        }
     }
     for (; r < s1; r += R) {
-        float a[8];
-        load_group(base + r * row_stride, mean ? mv : nullptr, a);
+        float v[8];
+        unpack_group(__ldg(base + r * row_stride), a.mean ? mv : nullptr, v);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(a[k]));
+        for (int k = 0; k < 8; ++k) m = fmaxf(m, fabsf(v[k]));
     }
-    m = block_max(m, red);
-    if (threadIdx.x == 0) partial[bh * g.nch + chunk] = m;
+    return m;
 }
 
-// Pass 2: fold the head's partials, then write the chunk's codes (and, chunk 0, the descale).
-__global__ void __launch_bounds__(kQThreads)
-    fp8_convert(const uint4* __restrict__ x, const float* __restrict__ mean,
-                const float* __restrict__ partial, uint2* __restrict__ x8,
-                float* __restrict__ descale, QGeom g)
+// Codes of rows [s0, s1) of slice bh with factor f.
+__device__ __forceinline__ void chunk_convert(const QOnePass& a, int64_t bh, int64_t s0,
+                                              int64_t s1, float f)
+{
+    const int G = (int)a.d8;
+    const int gi = threadIdx.x % G;
+    const int R = kQThreads / G;
+    const int64_t bi = bh / a.h, hh = bh - bi * a.h;
+    float mv[8];
+    if (a.mean) head_mean(a.mean, bh, a.d8, gi, mv);
+    const int64_t row_stride = a.h * a.d8;
+    const int64_t off = (bi * a.s * a.h + hh) * a.d8 + gi;
+    int64_t r = s0 + threadIdx.x / G;
+    for (; r < s1; r += 8 * R) {  // eight groups in flight
+        uint4 raw[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (r + e * R < s1) raw[e] = __ldg(a.x + off + (r + e * R) * row_stride);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (r + e * R >= s1) break;
+            float v[8];
+            unpack_group(raw[e], a.mean ? mv : nullptr, v);
+            uint32_t w[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                w[t] = (uint32_t)__nv_cvt_float2_to_fp8x2(
+                    make_float2(__fmul_rn(v[2 * t], f), __fmul_rn(v[2 * t + 1], f)),
+                    __NV_SATFINITE, __NV_E4M3);
+            a.x8[off + (r + e * R) * row_stride] =
+                make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+        }
+    }
+}
+
+__device__ __forceinline__ float factor_of(float amax)
+{
+    return amax > 0.f ? fminf(448.f / amax, FLT_MAX) : 1.f;
+}
+
+__global__ void __launch_bounds__(kQThreads) fp8_quant_onepass(const QOnePass a)
 {
     __shared__ float red[kQThreads / 32];
     __shared__ float amax_s;
-    const int64_t bh = blockIdx.x;
-    const int chunk = blockIdx.y;
-    float m = 0.f;
-    for (int c = threadIdx.x; c < g.nch; c += kQThreads) m = fmaxf(m, partial[bh * g.nch + c]);
-    m = block_max(m, red);
-    if (threadIdx.x == 0) amax_s = m;
-    __syncthreads();
-    const float amax = amax_s;
-    const float f = amax > 0.f ? fminf(448.f / amax, FLT_MAX) : 1.f;
-    if (chunk == 0 && threadIdx.x == 0) descale[bh] = amax > 0.f ? amax / 448.f : 1.f;
-
-    const int G = (int)g.d8;
-    const int gi = threadIdx.x % G;
-    const int R = kQThreads / G;
-    const int64_t bi = bh / g.h, hh = bh - bi * g.h;
-    float mv[8];
-    if (mean) head_mean(mean, bh, g.d8, gi, mv);
-    const int64_t s0 = (int64_t)chunk * g.rows_per_chunk;
-    const int64_t s1 = s0 + g.rows_per_chunk < g.s ? s0 + g.rows_per_chunk : g.s;
-    const int64_t row_stride = g.h * g.d8;
-    const int64_t off = (bi * g.s * g.h + hh) * g.d8 + gi;
-    for (int64_t r = s0 + threadIdx.x / G; r < s1; r += R) {
-        float a[8];
-        load_group(x + off + r * row_stride, mean ? mv : nullptr, a);
-        uint32_t w[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-            w[t] = (uint32_t)__nv_cvt_float2_to_fp8x2(
-                make_float2(__fmul_rn(a[2 * t], f), __fmul_rn(a[2 * t + 1], f)), __NV_SATFINITE,
-                __NV_E4M3);
-        x8[off + r * row_stride] = make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+    auto rows = [&](int64_t it, int64_t& s0, int64_t& s1) {
+        s0 = (it % a.nch) * a.rows_per_chunk;
+        s1 = s0 + a.rows_per_chunk < a.s ? s0 + a.rows_per_chunk : a.s;
+    };
+    if (a.nch == 1) {  // whole head slices, one after another: no grid-wide wait
+        for (int64_t bh = blockIdx.x; bh < a.n_items; bh += gridDim.x) {
+            float m = block_max(chunk_amax(a, bh, 0, a.s), red);
+            if (threadIdx.x == 0) {
+                amax_s = m;
+                a.descale[bh] = m > 0.f ? m / 448.f : 1.f;
+            }
+            __syncthreads();
+            chunk_convert(a, bh, 0, a.s, factor_of(amax_s));
+        }
+        return;
     }
+    // several chunks per head: at most one item per CTA (the host sizes the split so)
+    const int64_t it = blockIdx.x;
+    int64_t s0 = 0, s1 = 0;
+    if (it < a.n_items) {
+        rows(it, s0, s1);
+        const float m = block_max(chunk_amax(a, it / a.nch, s0, s1), red);
+        if (threadIdx.x == 0) a.partial[it] = m;
+    }
+    publish_cta(a.flags, a.tag);
+    if (!wait_all_published(a.flags, a.tag, (int)gridDim.x, (int)gridDim.x, a.flags + kQMaxGrid,
+                            a.status, a.timeout_ns))
+        return;
+    if (it >= a.n_items) return;
+    const int64_t bh = it / a.nch;
+    float m = 0.f;
+    if ((int)threadIdx.x < a.nch) m = __ldcg(a.partial + bh * a.nch + threadIdx.x);
+    m = block_max(m, red);
+    if (threadIdx.x == 0) {
+        amax_s = m;
+        if (it % a.nch == 0) a.descale[bh] = m > 0.f ? m / 448.f : 1.f;
+    }
+    __syncthreads();
+    chunk_convert(a, bh, s0, s1, factor_of(amax_s));
+}
+
+std::atomic<int> g_quant_grid[64];
+std::atomic<unsigned> g_quant_calls{0};
+
+// Grid of the one-pass quantiser on the current device: one CTA per SM when one fits (cached per
+// device; atomics: concurrent first calls store the same value), 0 on error.
+int quant_grid()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 0;
+    }
+    int n = g_quant_grid[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        int per_sm = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8_quant_onepass, kQThreads,
+                                                          0) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return 0;
+        }
+        n = per_sm >= 1 ? sms : 0;
+        n = n < kQMaxGrid ? n : kQMaxGrid;
+        g_quant_grid[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
 }
 
 }  // namespace
@@ -179,37 +267,53 @@ extern "C" int fp8_quantize(const void* x, const float* mean, void* x8, float* d
     if (rc != B200ATTN_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    QGeom g;
-    g.s = s;
-    g.h = h;
-    g.d8 = d / 8;
-    const int64_t R = kQThreads / g.d8;  // rows per step of one CTA
-    int64_t nch = (kQTargetCtas + nbh - 1) / nbh;
+    const int grid_max = quant_grid();
+    int* status = status_word();
+    if (grid_max <= 0 || !status) return B200ATTN_ERR_CUDA;
+
+    QOnePass a{};
+    a.x = static_cast<const uint4*>(x);
+    a.mean = mean;
+    a.x8 = static_cast<uint2*>(x8);
+    a.descale = descale;
+    a.s = s;
+    a.h = h;
+    a.d8 = d / 8;
+    // Chunks per head: as many as keep every CTA at one item at most (few heads), else one (many
+    // heads: whole slices, several per CTA); never more chunks than steps of R rows.
+    const int64_t R = kQThreads / a.d8;  // rows per step of one CTA
+    int64_t nch = nbh < grid_max ? grid_max / nbh : 1;
     const int64_t max_ch = (s + R - 1) / R;
     if (nch > max_ch) nch = max_ch;
-    if (nch > 1024) nch = 1024;
+    if (nch > kQMaxChunks) nch = kQMaxChunks;
     if (nch < 1) nch = 1;
-    int64_t rpc = (s + nch - 1) / nch;
-    rpc = (rpc + R - 1) / R * R;
-    if (rpc < R) rpc = R;
-    nch = s > 0 ? (s + rpc - 1) / rpc : 1;
-    g.rows_per_chunk = rpc;
-    g.nch = (int)nch;
+    const int64_t rpc = s > 0 ? (s + nch - 1) / nch : 0;
+    if (s > 0) nch = (s + rpc - 1) / rpc;
+    a.rows_per_chunk = rpc;
+    a.nch = (int)nch;
+    a.n_items = nbh * nch;
+    const int grid = (int)(a.n_items < grid_max ? a.n_items : grid_max);
+    a.tag = kQTagMagic | (unsigned long long)(g_quant_calls.fetch_add(1, std::memory_order_relaxed) + 1);
+    a.status = status;
+    a.timeout_ns = 4000000000ull;
 
-    float* partial = nullptr;
+    void* scratch = nullptr;
+    const size_t part_bytes = ((size_t)a.n_items * sizeof(float) + 255) / 256 * 256;
+    const size_t nbytes = part_bytes + (kQMaxGrid + 32) * sizeof(unsigned long long);
     cudaMemPool_t pool = scratch_pool();
-    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&partial),
-                                         (size_t)(nbh * nch) * sizeof(float), pool,
-                                         st) != cudaSuccess) {
+    if (!pool || cudaMallocFromPoolAsync(&scratch, nbytes, pool, st) != cudaSuccess) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
-    const dim3 grid((unsigned)nbh, (unsigned)nch);
-    fp8_amax_partial<<<grid, kQThreads, 0, st>>>(static_cast<const uint4*>(x), mean, partial, g);
-    fp8_convert<<<grid, kQThreads, 0, st>>>(static_cast<const uint4*>(x), mean, partial,
-                                            static_cast<uint2*>(x8), descale, g);
-    const bool launched = cudaGetLastError() == cudaSuccess;
-    if (cudaFreeAsync(partial, st) != cudaSuccess) {
+    a.partial = static_cast<float*>(scratch);
+    a.flags = reinterpret_cast<unsigned long long*>(static_cast<char*>(scratch) + part_bytes);
+    void* args[] = {&a};
+    const bool launched =
+        cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(fp8_quant_onepass),
+                                    dim3((unsigned)grid), dim3(kQThreads), args, 0, st) ==
+        cudaSuccess;
+    if (!launched) cudaGetLastError();
+    if (cudaFreeAsync(scratch, st) != cudaSuccess) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }

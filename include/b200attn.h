@@ -272,7 +272,8 @@ B200ATTN_API int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int6
  *   descale   device fp32 [b, h], 4-byte aligned. Fully written.
  *   b, h      >= 0 (0: nothing to do);  s >= 0 (0: every descale is 1);  d in {64, 128, 256}.
  * Scratch: taken from and returned to a library-owned stream-ordered memory pool on `stream`.
- * Two kernels (per-chunk amax, then fold and convert). Concurrency as in the conventions above.
+ * One cooperative launch (per-chunk amax, a grid-wide wait, then fold and convert). Concurrency
+ * as in the conventions above.
  */
 B200ATTN_API int fp8_quantize(const void* x, const float* mean, void* x8, float* descale,
                               int64_t b, int64_t s, int64_t h, int64_t d, void* stream);
