@@ -646,7 +646,7 @@ def run_gpu(args):
             kernels = "k_gate_onepass, 3 x fp8_quant_onepass"
         else:
             pre_bytes = 3 * n_k * 2
-            kernels = "k_mean_sub_onepass (K mean and K - mean in one launch)"
+            kernels = "k_mean_cols (K mean and K - mean in one launch)"
         pre_us = 1e3 * statistics.median(pre_ms)
         gbs = pre_bytes / (pre_us * 1e-6) / 1e9
         hbm = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])

@@ -384,6 +384,102 @@ __global__ void __launch_bounds__(kThreads) k_mean_sub_onepass(const OnePass a)
                       (int64_t)gridDim.x * kThreads, a.b, a.sk, a.c8);
 }
 
+// Column-partitioned K mean (and, with SUB, K - mean), used when K has many (batch, 8-channel
+// group) pairs: CTA c owns the G consecutive pairs p = bi * c8 + g8 in [c*G, c*G + G) and sums
+// them over ALL sk rows itself, so no cross-CTA fold, scratch or grid-wide wait is needed.
+// Thread t takes pair slot t % G at rows t / G, + L, + 2L, ... (L = 512 / G row lanes, G a power
+// of two; sixteen 16-byte loads in flight, added in row order); the L lane sums of each pair are
+// then added by a fixed tree in shared memory, so the mean is bit-identical from run to run. With
+// SUB every thread then rewrites its rows as K - mean, re-reading them through L2.
+template <bool SUB>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_mean_cols(const uint4* __restrict__ k, float* __restrict__ mean, uint4* __restrict__ k_out,
+                int64_t b, int64_t sk, int64_t c8, int G)
+{
+    __shared__ float4 red[kThreads * 2];  // [thread][2]: its 8 channel sums, then the tree's
+    const int gs = threadIdx.x % G, ln = threadIdx.x / G, L = kThreads / G;
+    const int64_t pair = (int64_t)blockIdx.x * G + gs;
+    const bool active = pair < b * c8;
+    const int64_t bi = active ? pair / c8 : 0, g8 = active ? pair - bi * c8 : 0;
+    const uint4* src = k + (bi * sk) * c8 + g8;
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    if (active) {
+        int64_t r = ln;
+        for (; r + 15 * L < sk; r += 16 * L) {
+            uint4 x[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) x[e] = __ldg(src + (r + e * L) * c8);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) acc_bf16x8(s, x[e]);
+        }
+        for (; r < sk; r += L) acc_bf16x8(s, __ldg(src + r * c8));
+    }
+    red[2 * threadIdx.x] = make_float4(s[0], s[1], s[2], s[3]);
+    red[2 * threadIdx.x + 1] = make_float4(s[4], s[5], s[6], s[7]);
+    __syncthreads();
+    for (int w = L / 2; w > 0; w >>= 1) {  // lane ln += lane ln + w, same slot
+        if (ln < w) {
+            const int o = threadIdx.x + w * G;
+            float4 a = red[2 * threadIdx.x], c = red[2 * threadIdx.x + 1];
+            const float4 a2 = red[2 * o], c2 = red[2 * o + 1];
+            a.x += a2.x; a.y += a2.y; a.z += a2.z; a.w += a2.w;
+            c.x += c2.x; c.y += c2.y; c.z += c2.z; c.w += c2.w;
+            red[2 * threadIdx.x] = a;
+            red[2 * threadIdx.x + 1] = c;
+        }
+        __syncthreads();
+    }
+    const float4 t0 = red[2 * gs], t1 = red[2 * gs + 1];  // lane 0's sums of this slot
+    const float n = (float)sk;
+    float mv[8] = {__fdiv_rn(t0.x, n), __fdiv_rn(t0.y, n), __fdiv_rn(t0.z, n), __fdiv_rn(t0.w, n),
+                   __fdiv_rn(t1.x, n), __fdiv_rn(t1.y, n), __fdiv_rn(t1.z, n), __fdiv_rn(t1.w, n)};
+    if (active && ln == 0) {
+        float4* m4 = reinterpret_cast<float4*>(mean + pair * 8);  // [b][cols] = pair-major
+        m4[0] = make_float4(mv[0], mv[1], mv[2], mv[3]);
+        m4[1] = make_float4(mv[4], mv[5], mv[6], mv[7]);
+    }
+    if constexpr (SUB) {
+        if (!active) return;
+        uint4* dst = k_out + (bi * sk) * c8 + g8;
+        int64_t r = ln;
+        for (; r + 7 * L < sk; r += 8 * L) {
+            uint4 x[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = __ldcg(src + (r + e * L) * c8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dst[(r + e * L) * c8] = sub8(x[e], mv);
+        }
+        for (; r < sk; r += L) dst[r * c8] = sub8(__ldcg(src + r * c8), mv);
+    }
+}
+
+// The column-partitioned split: G = the least power of two whose ceil(pairs / G) CTAs fit on
+// the SMs; taken when that grid keeps at least half of the SMs busy (else 0: the one-pass
+// row-chunk kernel).
+int cols_group(int64_t pairs, int n_sm)
+{
+    if (n_sm <= 0) return 0;
+    int G = 1;
+    while (G < kThreads && (pairs + G - 1) / G > n_sm) G <<= 1;
+    const int64_t grid = (pairs + G - 1) / G;
+    return (grid <= n_sm && 2 * grid >= n_sm) ? G : 0;
+}
+
+int launch_cols(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, int64_t cols,
+                int G, cudaStream_t st)
+{
+    const int64_t pairs = b * (cols / 8);
+    const unsigned grid = (unsigned)((pairs + G - 1) / G);
+    if (k_out)
+        k_mean_cols<true><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(k), mean,
+                                                      static_cast<uint4*>(k_out), b, sk,
+                                                      cols / 8, G);
+    else
+        k_mean_cols<false><<<grid, kThreads, 0, st>>>(static_cast<const uint4*>(k), mean, nullptr,
+                                                       b, sk, cols / 8, G);
+    return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
 // Fixed scratch for k_smooth_mean_noalloc: file-scope device memory that every GPU loading this
 // library holds until the process exits: 2^20 floats of partial sums (4 MiB), then one set of
 // flag words (1024 + 32 64-bit words: one per CTA of the one-pass kernel, then the go words).
@@ -556,6 +652,9 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
     if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
+    const int G = cols_group(b * (cols / 8), onepass_grid(k_mean_onepass, g_mean_grid));
+    if (G > 0)
+        return launch_cols(k, mean, nullptr, b, sk, cols, G, static_cast<cudaStream_t>(stream));
     return mean_pooled(k, mean, nullptr, b, sk, cols, onepass_grid(k_mean_onepass, g_mean_grid),
                        static_cast<cudaStream_t>(stream));
 }
@@ -573,6 +672,9 @@ extern "C" int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int64_
     // The mean's split must be the one k_smooth_mean takes (same bits): both grids are the SM
     // count whenever one CTA of each kernel fits on an SM, which the occupancy query confirms.
     const int grid = onepass_grid(k_mean_onepass, g_mean_grid);
+    const int G = cols_group(b * (cols / 8), grid);  // the same choice as k_smooth_mean's
+    if (G > 0)
+        return launch_cols(k, mean, k_out, b, sk, cols, G, static_cast<cudaStream_t>(stream));
     const int grid2 = onepass_grid(k_mean_sub_onepass, g_mean_sub_grid);
     if (grid2 != grid) return B200ATTN_ERR_CUDA;
     return mean_pooled(k, mean, k_out, b, sk, cols, grid, static_cast<cudaStream_t>(stream));
@@ -611,9 +713,12 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     if (b * cols > kNoAllocScratchFloats) return B200ATTN_ERR_SCRATCH;
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
+    const int grid_max = onepass_grid(k_mean_onepass, g_mean_grid);
+    const int G = cols_group(b * (cols / 8), grid_max);  // no scratch at all on this path
+    if (G > 0)
+        return launch_cols(k, mean, nullptr, b, sk, cols, G, static_cast<cudaStream_t>(stream));
     float* scratch = noalloc_scratch();
     int* status = status_word();
-    const int grid_max = onepass_grid(k_mean_onepass, g_mean_grid);
     if (!scratch || !status || grid_max <= 0) return B200ATTN_ERR_CUDA;
     // The partials of as many chunks as fit in the fixed scratch; the flags after them. Every
     // partial the fold reads is written earlier in the same launch, and a flag counts only when

@@ -157,9 +157,11 @@ B200ATTN_API int attn_fwd_varlen(const void* q, const void* k, const void* v, vo
  * "[HIP] Mha v4: run the K-smoothing gate as one HIP call" computes in two deterministic kernels
  * behind one host call (Summary; commit message). Here the sample is every key and no gate is
  * applied. Sums run in fp32 over sequence chunks, then the chunk partials are folded in a fixed
- * order, so repeated calls give bit-identical results. Both steps run as two phases of one
- * cooperative launch, with a bounded grid-wide wait between them (a wait that runs out sets the
- * error word read by attn_debug_status).
+ * order, so repeated calls give bit-identical results. One launch: when K has many (batch,
+ * 8-channel group) pairs, each CTA sums its own pairs over every key (no cross-CTA fold, no
+ * scratch); otherwise the sums over key chunks and their fold are two phases of one cooperative
+ * launch with a bounded grid-wide wait between them (a wait that runs out sets the error word
+ * read by attn_debug_status).
  *
  *   k     device bf16 [b, sk, hk, d], 16-byte aligned.
  *   mean  device fp32 [b, hk, d], 16-byte aligned. Fully written.
@@ -179,8 +181,9 @@ B200ATTN_API int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk
  * library allocate during a call -- for example a serving process that reserves all device
  * memory for its own pool at start-up (so a cudaMallocAsync inside the call could fail, or
  * stall the stream while the driver maps memory), or code that must keep its memory use fixed
- * and known in advance. It computes the same mean as k_smooth_mean with the same kernel, but
- * takes the partial sums from a fixed file-scope device array of 2^20 floats (4 MiB) that
+ * and known in advance. It computes the same mean as k_smooth_mean with the same kernels; where
+ * those fold partial sums, it takes them from a fixed file-scope device array of 2^20 floats
+ * (4 MiB) that
  * every GPU which loads this library holds until the process exits. It never calls cudaMalloc,
  * cudaFree or any allocating routine.
  *

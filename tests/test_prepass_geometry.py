@@ -142,3 +142,54 @@ def test_noalloc_split_fits_the_fixed_scratch():
             continue  # refused with ERR_SCRATCH
         _, _, nchunks, _, grid = make_split(b, cols, sk, NOALLOC_FLOATS // (b * cols), SMS)
         assert b * nchunks * cols <= NOALLOC_FLOATS and grid <= 1024
+
+
+def cols_group(pairs, n_sm):
+    """The column-partitioned split's pairs per CTA (0: the row-chunk kernel is used)."""
+    G = 1
+    while G < THREADS and (pairs + G - 1) // G > n_sm:
+        G <<= 1
+    grid = (pairs + G - 1) // G
+    return G if grid <= n_sm and 2 * grid >= n_sm else 0
+
+
+@pytest.mark.parametrize("seed", range(2))
+def test_column_path_sums_every_row_once(seed):
+    """k_mean_cols: CTA c owns (batch, 8-channel group) pairs [c*G, c*G + G); thread t takes pair
+    slot t % G at rows t // G, + L, ... (L = 512 / G); the tree over lanes folds every lane into
+    lane 0 exactly once. The K-mean workload (16 x 256 channels) takes it with G = 4 on 128 CTAs;
+    narrow K falls back to the row-chunk kernel."""
+    assert cols_group(1 * 16 * 256 // 8, SMS) == 4
+    assert (512 + 3) // 4 == 128
+    assert cols_group(2 * 3 * 64 // 8, SMS) == 0  # 48 pairs: too few CTAs
+    rnd = random.Random(20 + seed)
+    cases = [(1, 16, 4096, 256), (2, 40, 300, 256), (1, 64, 77, 128), (4, 20, 33, 64), (1, 148, 9, 64)]
+    cases += [(rnd.randint(1, 4), rnd.randint(1, 200), rnd.randint(1, 300),
+               rnd.choice([64, 128, 256])) for _ in range(30)]
+    for b, hk, sk, d in cases:
+        pairs = b * hk * d // 8
+        G = cols_group(pairs, SMS)
+        if G == 0:
+            continue
+        assert G & (G - 1) == 0 and 1 <= G <= THREADS
+        grid = (pairs + G - 1) // G
+        assert SMS / 2 <= grid <= SMS
+        L = THREADS // G
+        if pairs * sk <= 2_000_000:
+            seen = {}
+            for cta in range(grid):
+                for t in range(THREADS):
+                    pair = cta * G + t % G
+                    if pair >= pairs:
+                        continue
+                    for r in range(t // G, sk, L):
+                        seen[(pair, r)] = seen.get((pair, r), 0) + 1
+            assert len(seen) == pairs * sk and set(seen.values()) == {1}
+        held = [{ln} for ln in range(L)]  # the tree: lane ln absorbs lane ln + w
+        w = L // 2
+        while w > 0:
+            for ln in range(w):
+                assert not (held[ln] & held[ln + w])
+                held[ln] |= held[ln + w]
+            w //= 2
+        assert held[0] == set(range(L))
