@@ -262,8 +262,8 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
 // The share of score pairs whose exp2 runs on the FMA pipe is the measured best per head dim:
 // 3 of 8 at d128 (pairs 0, 2, 5 of every 8: 1141 vs 1060 with 2 of 8 at 65536^2, interleaved
 // A/B), 2 of 8 at d192 (3 of 8 is no faster there) and for E4M3 inputs (3 of 8 loses 1-3 %),
-// none at d256, bound by the tensor core. At d64 the share makes no measurable difference
-// (3 of 8 kept).
+// none at d256, bound by the tensor core. At d64, 3 of 8 (pairs 1, 4, 7) measured best (none:
+// -7 %, 4 of 8: -3 %).
 using T64P = AttnTraits<64, 64, 64, 2, 2, true, 8, 8, 0x92u, false, true>;  // 32 + 64 + 64 (+32) KB
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x25u>;         // 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;         // 96 + 96 + 32 KB
