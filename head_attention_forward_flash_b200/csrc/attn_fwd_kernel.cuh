@@ -131,6 +131,11 @@ struct AttnTraits {
     static constexpr bool PIPE = PIPE_;
     static_assert(!PIPE || NT == 2, "");
     static constexpr int NSBUF = PIPE ? 2 * NT : 2;  // score buffers
+    // One copy of the softmax body (two tiles, one score buffer each): a masked block first
+    // sets its disallowed scores to -inf, then runs the body of the unmasked blocks. The other
+    // layouts keep a second, masked body that skips chunks no row of the warp allows (measured
+    // on B200: one body is 1-2.5 % faster at d128, d192/128 and E4M3, 4 % slower at d64).
+    static constexpr bool ONE_BODY = NT == 2 && !PIPE;
     // tensor memory columns
     static constexpr uint32_t O_COL0 = NSBUF * BN;
     static constexpr uint32_t Q_COL0 = NSBUF * BN + NT * DV;
@@ -825,6 +830,30 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         float m_ref[NTW] = {};  // exponent reference (log2 units); moves lazily
         float l[NTW] = {};      // sum of exp2(x - m_ref) over the keys seen so far
         int j_begin = 0;
+        // ONE_BODY layouts: keys j*BN + c with lor <= c <= rel are allowed; every other score of
+        // the block becomes -inf (its max term and its p = exp2(-inf) then vanish). Chunks that
+        // every row of the warp allows entirely are left as they are.
+        auto mask_scores = [&](uint32_t(&sr)[BN], int k, int j) {
+            int64_t rel64 = lim[k] - (int64_t)j * BN;
+            rel64 = rel64 < -1 ? -1 : (rel64 > BN ? BN : rel64);
+            int lor = 0;  // no lower bound without a window
+            if (EXT) {
+                int64_t lor64 = lol[k] - (int64_t)j * BN;
+                lor = (int)(lor64 < 0 ? 0 : (lor64 > BN ? BN : lor64));
+            }
+            const int rel = (int)rel64;
+            const int rel_lo = __reduce_min_sync(FULL, rel);
+            const int lor_hi = EXT ? __reduce_max_sync(FULL, lor) : 0;
+#pragma unroll
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                if (ch * 32 + 31 <= rel_lo && ch * 32 >= lor_hi) continue;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = ch * 32 + e;
+                    sr[c] = (c <= rel && c >= lor) ? sr[c] : 0xff800000u;
+                }
+            }
+        };
         auto softmax_block = [&](const bool MASKED, uint32_t(&sr)[BN], int k, int tt, int j,
                                  int64_t jgb, uint32_t s_col) -> bool {
             // Keys j*BN + c with lor <= c <= rel are allowed. Per 32-key chunk the warp takes
@@ -1036,10 +1065,14 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
                     for (int c = 0; c < BN / 32; ++c)
                         tmem_ld32(s_col + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
                     tmem_wait_ld();
-                    if ((EXT && j < mask_lo) || j >= mask_from)
-                        ok = softmax_block(true, sr, k, tt, j, jg, s_col);
-                    else
+                    if constexpr (T::ONE_BODY) {
+                        if ((EXT && j < mask_lo) || j >= mask_from) mask_scores(sr, k, j);
                         ok = softmax_block(false, sr, k, tt, j, jg, s_col);
+                    } else if ((EXT && j < mask_lo) || j >= mask_from) {
+                        ok = softmax_block(true, sr, k, tt, j, jg, s_col);
+                    } else {
+                        ok = softmax_block(false, sr, k, tt, j, jg, s_col);
+                    }
                     if (!ok) break;
                     tmem_wait_st();
                     tc_fence_before_sync();
