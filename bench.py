@@ -437,6 +437,49 @@ def run_gpu(args):
                  "gbs": g_bytes / (g_us * 1e-6) / 1e9, "threshold": GATE_THRESHOLD,
                  "launches": 2, "note": "k_smooth_gate alone, L2 flushed before each call"}
 
+    # Workloads whose step has no pre-pass: the K-smoothing pre-pass kernels timed beside the
+    # step (not inside it) on this workload's own K, so that every bench line carries their
+    # HBM rate. Each call alone, event-timed, L2 flushed before it.
+    prepass_beside = None
+    if not (c["kmean"] or fp8 or varlen) and c["dqk"] in (64, 128, 256):
+        hbm = measured_peaks()[0].get("hbm_gbs", FALLBACK["hbm_gbs"])
+        n_kb = k.numel() * 2
+        k_tmp = torch.empty_like(k)
+        m_tmp = torch.empty_like(mean)
+        calls = {
+            "k_smooth_mean": (lambda: b2.k_smooth_mean(k, m_tmp), n_kb,
+                              "read K once"),
+            "k_smooth_mean_sub": (lambda: b2.k_smooth_mean_sub(k, m_tmp, k_tmp), 3 * n_kb,
+                                  "read K, read it again, write K - mean"),
+            "k_smooth_gate": (lambda: b2.k_smooth_gate(k, GATE_THRESHOLD, mean=m_tmp,
+                                                       return_ratio=False),
+                              c["b"] * ((c["sk"] + (c["sk"] + 2047) // 2048 - 1)
+                                        // ((c["sk"] + 2047) // 2048)) * c["hk"] * c["dqk"] * 2,
+                              "read the strided key sample"),
+        }
+        prepass_beside = {"note": "not part of the step: each kernel alone on this workload's K, "
+                                  "L2 flushed before each call, median of 10",
+                          "measured_hbm_gbs": hbm}
+        for name, (fn, nbytes, what) in calls.items():
+            e0 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+            e1 = [torch.cuda.Event(enable_timing=True) for _ in range(10)]
+            for _ in range(3):
+                fn()
+            for s_ in range(10):
+                flush.zero_()
+                e0[s_].record(stream)
+                fn()
+                e1[s_].record(stream)
+            torch.cuda.synchronize()
+            us = 1e3 * statistics.median(e0[s_].elapsed_time(e1[s_]) for s_ in range(10))
+            gbs = nbytes / (us * 1e-6) / 1e9
+            prepass_beside[name] = {"us_median": us, "bytes": nbytes, "bytes_are": what,
+                                    "gbs": gbs, "frac_of_measured_hbm": gbs / hbm,
+                                    "frac_of_datasheet_8tbs": gbs / 8000.0}
+        del k_tmp, m_tmp
+        if b2.attn_debug_status() != 0:
+            raise RuntimeError("a pre-pass kernel reported a bounded-wait timeout")
+
     # end to end through the public API with host buffers (pinned), copies inside the timing.
     # Every step copies its own inputs in and its own result out. Two timings:
     #   serial     one stream, step after step (copy in, compute, copy out);
@@ -632,6 +675,8 @@ def run_gpu(args):
             "peak_source": "B200 datasheet dense E4M3"}
     if kgate is not None:
         line["k_smooth_gate"] = kgate
+    if prepass_beside is not None:
+        line["prepass_beside_step"] = prepass_beside
     if c["kmean"] or fp8:
         # bytes the pre-pass kernels move by design. K mean: read K; subtract: read K, write K'.
         # FP8: the gate's sampled rows, then per tensor two reads (amax, convert) of bf16 and

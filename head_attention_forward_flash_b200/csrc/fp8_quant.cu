@@ -32,7 +32,7 @@ namespace {
 constexpr int kQThreads = 512;
 constexpr int kQMaxChunks = 64;   // chunks per head slice at most (the fold: one load per thread)
 constexpr int kQMaxGrid = 1024;   // CTAs of the launch at most (flag words)
-constexpr uint64_t kQTagMagic = 0x6670387175ULL << 24;  // high bits of every flag tag
+constexpr unsigned kQTagKind = 0x6638u;  // top 16 bits of every flag tag of the quantiser
 
 // The 8 elements of a 16-byte bf16 group (already loaded), minus the mean when given (one fp32
 // subtraction).
@@ -217,7 +217,6 @@ __global__ void __launch_bounds__(kQThreads) fp8_quant_onepass(const QOnePass a)
 }
 
 std::atomic<int> g_quant_grid[64];
-std::atomic<unsigned> g_quant_calls{0};
 
 // Grid of the one-pass quantiser on the current device: one CTA per SM when one fits (cached per
 // device; atomics: concurrent first calls store the same value), 0 on error.
@@ -293,7 +292,7 @@ extern "C" int fp8_quantize(const void* x, const float* mean, void* x8, float* d
     a.nch = (int)nch;
     a.n_items = nbh * nch;
     const int grid = (int)(a.n_items < grid_max ? a.n_items : grid_max);
-    a.tag = kQTagMagic | (unsigned long long)(g_quant_calls.fetch_add(1, std::memory_order_relaxed) + 1);
+    a.tag = next_call_tag(kQTagKind);
     a.status = status;
     a.timeout_ns = 4000000000ull;
 

@@ -2,16 +2,40 @@
 // K-smoothing gate, the FP8 quantiser), launched cooperatively so that every CTA is resident.
 //
 // Each CTA publishes a per-call tag in its own flag word (st.release after its stores); a call
-// never clears flags, since each launch carries a tag no earlier launch of the process used. Every
+// never clears flags, since each launch carries a tag (next_call_tag) that no flag word left in
+// memory by an earlier launch, of this or of another loaded copy of the library, holds. Every
 // wait is bounded: past timeout_ns it sets the error word and returns false, and the caller
 // leaves the kernel.
 #pragma once
 
+#include <atomic>
+#include <chrono>
 #include <cstdint>
 
 #include "host_common.h"
 
 namespace b200 {
+
+// A fresh tag for one launch's flag words: `kind` (the kernel family) in the top 16 bits, a
+// 48-bit call counter below. The counter starts at a point drawn once per loaded copy of the
+// library (the clock and the counter's own address, mixed by the SplitMix64 finaliser), so flag
+// words that recycled memory still holds, from earlier calls or from another copy of the library
+// loaded into the same process, never carry a tag that a later call uses. 2^48 calls do not wrap
+// in practice.
+inline unsigned long long next_call_tag(unsigned kind)
+{
+    static std::atomic<unsigned long long> counter{[] {
+        unsigned long long z =
+            (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() ^
+            (unsigned long long)(uintptr_t)&counter;
+        z += 0x9E3779B97F4A7C15ull;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        return z ^ (z >> 31);
+    }()};
+    const unsigned long long c = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+    return ((unsigned long long)(kind & 0xFFFFu) << 48) | (c & 0xFFFFFFFFFFFFull);
+}
 
 __device__ __forceinline__ uint64_t global_ns()
 {

@@ -24,6 +24,7 @@
 
 #include "grid_sync.cuh"
 #include "host_common.h"
+#include "sm100_ptx.cuh"
 
 namespace b200 {
 namespace {
@@ -32,10 +33,15 @@ constexpr int kThreads = 512;  // one-pass kernels: each thread owns 8 consecuti
 constexpr int kColsPerCta = kThreads * 8;
 constexpr int kFoldWarps = kThreads / 32;
 constexpr int kSubThreads = 256;
-constexpr uint64_t kTagMagic = 0x6B6D65616EULL << 24;  // high bits of every flag tag
+constexpr unsigned kTagKind = 0x6B6Du;  // top 16 bits of every flag tag of these kernels
 constexpr int kMaxGrid = 1024;  // CTAs of a one-pass launch at most (flag words per set)
 constexpr int kGo1 = kMaxGrid, kGo2 = kMaxGrid + 16;  // go words after the phase-1 flags
 constexpr int kFlagWords = kMaxGrid + 32;  // one flag set with its go words (16 words apart)
+// The mean's phase 1 when a CTA spans whole rows: a ring of kStages shared-memory buffers of
+// kStageBytes each, filled by bulk copies (dynamic shared memory of the one-pass mean kernels).
+constexpr int kStages = 4;
+constexpr int kStageBytes = 32768;
+constexpr int kRingBytes = kStages * kStageBytes;
 
 __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& x)
 {
@@ -92,6 +98,8 @@ struct OnePass {
     int64_t n_rows;             // rows summed per (bi, column): sk, or the sample size
     int64_t rows_per_chunk;
     int nchunks;
+    int lanes;                  // mean, whole rows per CTA: row lanes of the bulk-copy phase 1;
+                                // 0: the register path (sum_chunks)
     int64_t n_items;            // b * colgroups * nchunks
     int64_t hk, d;              // gate: kv heads and channels per head
     float n_rows_f;             // n_rows as fp32, the divisor
@@ -147,6 +155,114 @@ __device__ __forceinline__ void sum_chunks(const OnePass& a)
     }
 }
 
+// Phase 1 of the mean when one CTA spans whole rows (colgroups = 1): each item's chunk of rows
+// is one contiguous range of K, streamed through the shared-memory ring by bulk copies that
+// thread 0 issues (kStages in flight, completion on one mbarrier per buffer), so the bytes in
+// flight per SM do not depend on registers. Thread t owns group t % c8 at rows t0 + t / c8, + R,
+// + 2R, ... of the chunk (R = lanes = kThreads / c8 row lanes; threads past R * c8 idle) and adds
+// them in row order; the R lane sums of a group are then added in lane order through shared
+// memory, so the split alone fixes the bits. `fills` counts the buffers filled so far (the
+// barrier phases), the same in every thread. False, with the status word set, if a copy does not
+// land within the time limit; the copies still in flight are then waited for (bounded) first.
+__device__ __forceinline__ bool sum_chunks_bulk(const OnePass& a, float4 (&lred)[kThreads * 2],
+                                                uint8_t* ring, uint64_t* full,
+                                                volatile int* abort_flag)
+{
+    const int c8 = (int)a.c8, R = a.lanes;
+    const int tid = (int)threadIdx.x;
+    const int lane = tid / c8, g8 = tid - lane * c8;
+    const int64_t row_bytes = a.c8 * 16;
+    const int rps = (int)(kStageBytes / row_bytes);  // rows per buffer (row_bytes <= 8 KB)
+    const WaitCtx w{abort_flag, a.status, a.timeout_ns};
+    uint32_t fills = 0;
+    for (int64_t it = blockIdx.x; it < a.n_items; it += gridDim.x) {
+        const int chunk = (int)(it % a.nchunks);
+        const int64_t bi = it / a.nchunks;
+        const int64_t t0 = (int64_t)chunk * a.rows_per_chunk;
+        int64_t t1 = t0 + a.rows_per_chunk;
+        t1 = t1 < a.n_rows ? t1 : a.n_rows;
+        const int nst = (int)((t1 - t0 + rps - 1) / rps);
+        const char* src = reinterpret_cast<const char*>(a.k) + (bi * a.sk + t0) * row_bytes;
+        auto issue = [&](int st) {  // thread 0: buffer st of this chunk
+            const uint32_t slot = (fills + (uint32_t)st) % kStages;
+            const int64_t r0 = (int64_t)st * rps;
+            const int64_t n = (t1 - t0 - r0) < rps ? (t1 - t0 - r0) : rps;
+            const uint32_t bar = smem_addr(full + slot);
+            mbar_arrive_expect_tx(bar, (uint32_t)(n * row_bytes));
+            bulk_load(smem_addr(ring + (size_t)slot * kStageBytes), src + r0 * row_bytes,
+                      (uint32_t)(n * row_bytes), bar);
+        };
+        if (tid == 0)
+            for (int st = 0; st < nst && st < kStages; ++st) issue(st);
+        float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int st = 0; st < nst; ++st) {
+            const uint32_t f = fills + (uint32_t)st;
+            const uint32_t slot = f % kStages;
+            const bool ok = mbar_wait(smem_addr(full + slot), (f / kStages) & 1u, w,
+                                      B200ATTN_ERR_TIMEOUT);
+            if (__syncthreads_or(!ok)) {
+                if (tid == 0) {  // let the copies in flight land before leaving (bounded)
+                    const int last = (st + kStages < nst ? st + kStages : nst);
+                    for (int q = st; q < last; ++q) {
+                        const uint32_t fq = fills + (uint32_t)q;
+                        const uint64_t tq = global_timer_ns();
+                        while (!mbar_try_wait(smem_addr(full + fq % kStages), (fq / kStages) & 1u) &&
+                               global_timer_ns() - tq < 1000000000ull) {
+                        }
+                    }
+                }
+                __syncthreads();
+                return false;
+            }
+            if (lane < R) {
+                const int64_t r0 = (int64_t)st * rps;  // the buffer's first row, from t0
+                const int64_t n64 = (t1 - t0 - r0) < rps ? (t1 - t0 - r0) : rps;
+                const int n = (int)n64;
+                int r = (int)((lane - r0 % R + R) % R);  // first row with (row - t0) % R == lane
+                const uint4* rows = reinterpret_cast<const uint4*>(ring + (size_t)slot * kStageBytes);
+                for (; r < n; r += R) acc_bf16x8(s, rows[r * c8 + g8]);
+            }
+            __syncthreads();  // every thread is done with the buffer
+            if (tid == 0 && st + kStages < nst) issue(st + kStages);
+        }
+        fills += (uint32_t)nst;
+        lred[2 * tid] = make_float4(s[0], s[1], s[2], s[3]);
+        lred[2 * tid + 1] = make_float4(s[4], s[5], s[6], s[7]);
+        __syncthreads();
+        if (tid < c8) {
+            float4 u = lred[2 * tid], v = lred[2 * tid + 1];
+            for (int q = 1; q < R; ++q) {
+                const float4 u2 = lred[2 * (q * c8 + tid)], v2 = lred[2 * (q * c8 + tid) + 1];
+                u.x += u2.x; u.y += u2.y; u.z += u2.z; u.w += u2.w;
+                v.x += v2.x; v.y += v2.y; v.z += v2.z; v.w += v2.w;
+            }
+            float4* dst = reinterpret_cast<float4*>(
+                a.partial + (bi * a.nchunks + chunk) * a.cols + tid * 8);
+            dst[0] = u;
+            dst[1] = v;
+        }
+        __syncthreads();
+    }
+    return true;
+}
+
+// The mean's phase 1 by either path; false if it gave up (the status word is set).
+__device__ __forceinline__ bool mean_phase1(const OnePass& a, float4 (&lred)[kThreads * 2],
+                                            uint8_t* ring, uint64_t* full, int* abort_flag)
+{
+    if (a.lanes == 0) {
+        sum_chunks<false>(a);
+        return true;
+    }
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        for (int q = 0; q < kStages; ++q) mbar_init(smem_addr(full + q), 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    return sum_chunks_bulk(a, lred, ring, full, abort_flag);
+}
+
 // mean[bi][col] = (sum of partial[bi][chunk][col] over the chunks) / sk. Fold items are blocks of
 // 32 columns of one batch; warp w of the CTA sums the chunks of its fixed contiguous range
 // [w*nchunks/16, (w+1)*nchunks/16) in order, then the 16 warp sums are added in warp order.
@@ -180,7 +296,11 @@ __device__ __forceinline__ void fold_mean(const OnePass& a, float (&red)[kFoldWa
 __global__ void __launch_bounds__(kThreads) k_mean_onepass(const OnePass a)
 {
     __shared__ float red[kFoldWarps][32];
-    sum_chunks<false>(a);
+    __shared__ float4 lred[kThreads * 2];
+    __shared__ uint64_t full[kStages];
+    __shared__ int abort_flag;
+    extern __shared__ __align__(128) uint8_t ring[];
+    if (!mean_phase1(a, lred, ring, full, &abort_flag)) return;
     publish_cta(a.flags, a.tag);
     const int64_t nf = n_fold(a);
     if ((int64_t)blockIdx.x >= nf) return;
@@ -366,7 +486,11 @@ __global__ void __launch_bounds__(kSubThreads)
 __global__ void __launch_bounds__(kThreads) k_mean_sub_onepass(const OnePass a)
 {
     __shared__ float red[kFoldWarps][32];
-    sum_chunks<false>(a);
+    __shared__ float4 lred[kThreads * 2];
+    __shared__ uint64_t full[kStages];
+    __shared__ int abort_flag;
+    extern __shared__ __align__(128) uint8_t ring[];
+    if (!mean_phase1(a, lred, ring, full, &abort_flag)) return;
     publish_cta(a.flags, a.tag);
     const int64_t nf = n_fold(a);
     const int fold_ctas = (int)(nf < (int64_t)gridDim.x ? nf : (int64_t)gridDim.x);
@@ -454,15 +578,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // The column-partitioned split: G = the least power of two whose ceil(pairs / G) CTAs fit on
-// the SMs; taken when that grid keeps at least half of the SMs busy (else 0: the one-pass
-// row-chunk kernel).
+// the SMs; taken when that grid keeps at least half of the SMs busy and G >= kColsMinG (each
+// CTA then reads G * 16 contiguous bytes of every row); else 0: the one-pass row-chunk kernel.
+constexpr int kColsMinG = 2;
 int cols_group(int64_t pairs, int n_sm)
 {
     if (n_sm <= 0) return 0;
     int G = 1;
     while (G < kThreads && (pairs + G - 1) / G > n_sm) G <<= 1;
     const int64_t grid = (pairs + G - 1) / G;
-    return (grid <= n_sm && 2 * grid >= n_sm) ? G : 0;
+    return (grid <= n_sm && 2 * grid >= n_sm && G >= kColsMinG) ? G : 0;
 }
 
 int launch_cols(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, int64_t cols,
@@ -506,7 +631,7 @@ int check_kmean_args(const void* k, const void* mean, int64_t b, int64_t hk, int
 // at most one per SM and at most kMaxGrid; cached per device (atomics: concurrent first calls
 // store the same value).
 template <class K>
-int onepass_grid(K kernel, std::atomic<int> (&cache)[64])
+int onepass_grid(K kernel, std::atomic<int> (&cache)[64], int dyn_smem = 0)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -516,7 +641,10 @@ int onepass_grid(K kernel, std::atomic<int> (&cache)[64])
     int n = cache[dev].load(std::memory_order_relaxed);
     if (n == 0) {
         int per_sm = 0, sms = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) !=
+        if ((dyn_smem > 0 &&
+             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  dyn_smem) != cudaSuccess) ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, dyn_smem) !=
                 cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
             cudaGetLastError();
@@ -531,32 +659,31 @@ int onepass_grid(K kernel, std::atomic<int> (&cache)[64])
 
 std::atomic<int> g_mean_grid[64];
 std::atomic<int> g_gate_grid[64];
-std::atomic<unsigned> g_calls{0};
 
-// A tag no earlier call of this process used, with high bits no partial sum's bits resemble.
-unsigned long long next_tag()
-{
-    const unsigned c = g_calls.fetch_add(1, std::memory_order_relaxed) + 1;
-    return kTagMagic | (unsigned long long)c;
-}
+unsigned long long next_tag() { return next_call_tag(kTagKind); }
 
 // Work split of the one-pass kernels: the rows of every (bi, column group of 4096 channels) cut
-// into chunks, so that the grid's CTAs get about one item each; at least 16 rows per chunk, at
-// most max_chunks chunks (the scratch), at most 1024. (Splitting a chunk's rows among several
-// row lanes of a CTA, for K with few channels, made the gate of the b1 hk5 d128 65536-key
-// workload slower: 17.7 vs 13.7 us. Fewer CTAs then issue the loads, and each SM's outstanding
-// loads queue.)
+// into chunks, so that the grid's CTAs get about one item each; at least 16 rows per chunk (per
+// row lane), at most max_chunks chunks (the scratch), at most 1024. With lanes_ok (the mean) and
+// rows of at most 4096 channels (one column group), a chunk is one contiguous range of K: the
+// bulk-copy phase 1 streams it, spread over kThreads / c8 row lanes. (The gate keeps the register
+// path and one lane: its 2048-row sample is latency-bound, and row lanes made the gate of the
+// b1 hk5 d128 65536-key workload slower, 17.7 vs 13.7 us, as fewer SMs then had loads in flight.)
 struct Split {
     int64_t colgroups, rows_per_chunk, n_items;
-    int nchunks, grid;
+    int nchunks, grid, lanes;
 };
 
-Split make_split(int64_t b, int64_t cols, int64_t n_rows, int64_t max_chunks, int grid_max)
+Split make_split(int64_t b, int64_t cols, int64_t n_rows, int64_t max_chunks, int grid_max,
+                 bool lanes_ok)
 {
     Split s;
     s.colgroups = (cols + kColsPerCta - 1) / kColsPerCta;
+    const int64_t c8 = cols / 8;
+    s.lanes = (lanes_ok && s.colgroups == 1) ? (int)(kThreads / c8) : 0;
     int64_t nch = (grid_max + b * s.colgroups - 1) / (b * s.colgroups);
-    const int64_t by_rows = (n_rows + 15) / 16;
+    const int64_t per = 16 * (int64_t)(s.lanes > 0 ? s.lanes : 1);
+    const int64_t by_rows = (n_rows + per - 1) / per;
     if (nch > by_rows) nch = by_rows;
     if (nch > max_chunks) nch = max_chunks;
     if (nch > 1024) nch = 1024;
@@ -568,11 +695,12 @@ Split make_split(int64_t b, int64_t cols, int64_t n_rows, int64_t max_chunks, in
     return s;
 }
 
-int launch_onepass(void (*kernel)(const OnePass), OnePass& a, int grid, cudaStream_t st)
+int launch_onepass(void (*kernel)(const OnePass), OnePass& a, int grid, cudaStream_t st,
+                   int dyn_smem = 0)
 {
     void* args[] = {&a};
     if (cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kernel), dim3((unsigned)grid),
-                                    dim3(kThreads), args, 0, st) != cudaSuccess) {
+                                    dim3(kThreads), args, (size_t)dyn_smem, st) != cudaSuccess) {
         cudaGetLastError();
         return B200ATTN_ERR_CUDA;
     }
@@ -602,12 +730,14 @@ int run_mean(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, int
     a.n_rows = sk;
     a.rows_per_chunk = sp.rows_per_chunk;
     a.nchunks = sp.nchunks;
+    a.lanes = sp.lanes;
     a.n_items = sp.n_items;
     a.n_rows_f = (float)sk;
     a.tag = next_tag();
     a.status = status;
     a.timeout_ns = 4000000000ull;
-    return launch_onepass(k_out ? k_mean_sub_onepass : k_mean_onepass, a, sp.grid, st);
+    return launch_onepass(k_out ? k_mean_sub_onepass : k_mean_onepass, a, sp.grid, st,
+                          kRingBytes);
 }
 
 // k_smooth_mean and k_smooth_mean_sub: scratch (the split's partials, then two flag arrays) from
@@ -617,7 +747,7 @@ int mean_pooled(const void* k, float* mean, void* k_out, int64_t b, int64_t sk, 
 {
     int* status = status_word();
     if (!status || grid_max <= 0) return B200ATTN_ERR_CUDA;
-    const Split sp = make_split(b, cols, sk, 1024, grid_max);
+    const Split sp = make_split(b, cols, sk, 1024, grid_max, true);
     const size_t part_bytes = (size_t)(b * sp.nchunks * cols) * sizeof(float);
     const size_t nbytes = part_bytes + 2 * kFlagWords * sizeof(unsigned long long);
     char* scratch = nullptr;
@@ -652,11 +782,11 @@ extern "C" int k_smooth_mean(const void* k, float* mean, int64_t b, int64_t hk, 
     if (rc != B200ATTN_OK || b == 0 || hk == 0) return rc;
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
-    const int G = cols_group(b * (cols / 8), onepass_grid(k_mean_onepass, g_mean_grid));
+    const int grid = onepass_grid(k_mean_onepass, g_mean_grid, kRingBytes);
+    const int G = cols_group(b * (cols / 8), grid);
     if (G > 0)
         return launch_cols(k, mean, nullptr, b, sk, cols, G, static_cast<cudaStream_t>(stream));
-    return mean_pooled(k, mean, nullptr, b, sk, cols, onepass_grid(k_mean_onepass, g_mean_grid),
-                       static_cast<cudaStream_t>(stream));
+    return mean_pooled(k, mean, nullptr, b, sk, cols, grid, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int64_t b, int64_t hk,
@@ -671,11 +801,11 @@ extern "C" int k_smooth_mean_sub(const void* k, float* mean, void* k_out, int64_
     if (rc != B200ATTN_OK) return rc;
     // The mean's split must be the one k_smooth_mean takes (same bits): both grids are the SM
     // count whenever one CTA of each kernel fits on an SM, which the occupancy query confirms.
-    const int grid = onepass_grid(k_mean_onepass, g_mean_grid);
+    const int grid = onepass_grid(k_mean_onepass, g_mean_grid, kRingBytes);
     const int G = cols_group(b * (cols / 8), grid);  // the same choice as k_smooth_mean's
     if (G > 0)
         return launch_cols(k, mean, k_out, b, sk, cols, G, static_cast<cudaStream_t>(stream));
-    const int grid2 = onepass_grid(k_mean_sub_onepass, g_mean_sub_grid);
+    const int grid2 = onepass_grid(k_mean_sub_onepass, g_mean_sub_grid, kRingBytes);
     if (grid2 != grid) return B200ATTN_ERR_CUDA;
     return mean_pooled(k, mean, k_out, b, sk, cols, grid, static_cast<cudaStream_t>(stream));
 }
@@ -713,7 +843,7 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     if (b * cols > kNoAllocScratchFloats) return B200ATTN_ERR_SCRATCH;
     rc = check_arch();
     if (rc != B200ATTN_OK) return rc;
-    const int grid_max = onepass_grid(k_mean_onepass, g_mean_grid);
+    const int grid_max = onepass_grid(k_mean_onepass, g_mean_grid, kRingBytes);
     const int G = cols_group(b * (cols / 8), grid_max);  // no scratch at all on this path
     if (G > 0)
         return launch_cols(k, mean, nullptr, b, sk, cols, G, static_cast<cudaStream_t>(stream));
@@ -723,7 +853,8 @@ extern "C" int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, int6
     // The partials of as many chunks as fit in the fixed scratch; the flags after them. Every
     // partial the fold reads is written earlier in the same launch, and a flag counts only when
     // it carries this call's tag, so nothing needs clearing between calls.
-    const Split sp = make_split(b, cols, sk, kNoAllocScratchFloats / (b * cols), grid_max);
+    const Split sp =
+        make_split(b, cols, sk, kNoAllocScratchFloats / (b * cols), grid_max, true);
     return run_mean(k, mean, nullptr, b, sk, cols, sp, scratch,
                     reinterpret_cast<unsigned long long*>(scratch + kNoAllocScratchFloats),
                     status, static_cast<cudaStream_t>(stream));
@@ -749,7 +880,7 @@ extern "C" int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* r
 
     const int64_t stride = (sk + 2047) / 2048;  // every key up to 2048, else a strided sample
     const int64_t n_samp = (sk + stride - 1) / stride;
-    const Split sp = make_split(b, cols, n_samp, 1024, grid_max);
+    const Split sp = make_split(b, cols, n_samp, 1024, grid_max, false);
     const size_t part_bytes = (size_t)(b * sp.nchunks * 2 * cols) * sizeof(float);
     const size_t nbytes = part_bytes + kFlagWords * sizeof(unsigned long long);
     char* scratch = nullptr;
@@ -775,6 +906,7 @@ extern "C" int k_smooth_gate(const void* k, float* mean, int32_t* gate, float* r
     a.n_rows = n_samp;
     a.rows_per_chunk = sp.rows_per_chunk;
     a.nchunks = sp.nchunks;
+    a.lanes = 1;
     a.n_items = sp.n_items;
     a.hk = hk;
     a.d = d;

@@ -136,6 +136,18 @@ __device__ __forceinline__ void tma_store_4d(const void* desc, uint32_t src, int
                  : "memory");
 }
 
+// Untiled bulk copy of `bytes` bytes (a multiple of 16; both addresses 16-byte aligned) from
+// global memory to this CTA's shared memory, counted on mbarrier `bar` (complete_tx). No
+// multicast.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group()
 {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");

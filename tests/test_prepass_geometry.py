@@ -1,8 +1,11 @@
 """The work split of the one-pass K-mean and K-smoothing-gate kernels (csrc/kmean.cu: make_split,
-sum_chunks and the two folds), transcribed and checked on the CPU:
+sum_chunks, sum_chunks_bulk and the two folds), transcribed and checked on the CPU:
   - phase 1 sums every (key row, 8-channel group) of every batch exactly once (the gate: exactly
     the strided sample 0, stride, 2*stride, ... < sk, every key up to 2048 keys, at most 2048
     samples beyond), and every partial it writes lies inside the scratch sized for the split;
+  - the mean's bulk-copy phase 1 (rows of at most 4096 channels): every copy is a whole number
+    of 16-byte units inside K and inside one ring buffer, and each row lane reads its own rows in
+    order;
   - the fold covers every (batch, column) of the mean once (the gate: every (batch, kv head)),
     and its chunk ranges (per warp, per channel group) cover every chunk exactly once;
   - the allocation-free entry point's split never needs more partials than its fixed array holds.
@@ -16,17 +19,68 @@ COLS_PER_CTA = THREADS * 8
 FOLD_WARPS = THREADS // 32
 SMS = 148
 NOALLOC_FLOATS = 1 << 20
+STAGES, STAGE_BYTES = 4, 32768  # the bulk-copy ring
+COLS_MIN_G = 2
 
 
-def make_split(b, cols, n_rows, max_chunks, grid_max):
+def lanes_of(cols, lanes_ok):
+    """Row lanes of the mean's bulk-copy phase 1 (0: the register path)."""
     colgroups = (cols + COLS_PER_CTA - 1) // COLS_PER_CTA
+    return THREADS // (cols // 8) if lanes_ok and colgroups == 1 else 0
+
+
+def make_split(b, cols, n_rows, max_chunks, grid_max, lanes_ok=False):
+    colgroups = (cols + COLS_PER_CTA - 1) // COLS_PER_CTA
+    per = 16 * max(lanes_of(cols, lanes_ok), 1)
     nch = (grid_max + b * colgroups - 1) // (b * colgroups)
-    nch = min(nch, (n_rows + 15) // 16, max_chunks, 1024)
+    nch = min(nch, (n_rows + per - 1) // per, max_chunks, 1024)
     nch = max(nch, 1)
     rpc = (n_rows + nch - 1) // nch
     nchunks = (n_rows + rpc - 1) // rpc
     n_items = b * colgroups * nchunks
     return colgroups, rpc, nchunks, n_items, min(n_items, grid_max)
+
+
+def phase1_bulk(b, cols, sk, split):
+    """(bi, row, 8-channel group) -> times summed by the bulk-copy phase 1; checks every copy
+    and every shared-memory read on the way."""
+    colgroups, rpc, nchunks, n_items, grid = split
+    assert colgroups == 1
+    c8 = cols // 8
+    R = THREADS // c8
+    row_bytes = c8 * 16
+    rps = STAGE_BYTES // row_bytes
+    assert rps >= 1
+    seen = {}
+    for cta in range(grid):
+        fills = 0
+        for it in range(cta, n_items, grid):
+            chunk, bi = it % nchunks, it // nchunks
+            t0 = chunk * rpc
+            t1 = min(t0 + rpc, sk)
+            nst = (t1 - t0 + rps - 1) // rps
+            src = (bi * sk + t0) * row_bytes
+            last = [-1] * (R * c8)
+            for st in range(nst):
+                r0 = st * rps
+                n = min(rps, t1 - t0 - r0)
+                nbytes = n * row_bytes
+                assert nbytes % 16 == 0 and 0 < nbytes <= STAGE_BYTES and src % 16 == 0
+                assert src + r0 * row_bytes + nbytes <= b * sk * row_bytes
+                slot = (fills + st) % STAGES
+                assert (slot + 1) * STAGE_BYTES <= STAGES * STAGE_BYTES
+                for tid in range(R * c8):
+                    lane, g8 = divmod(tid, c8)
+                    r = (lane - r0 % R + R) % R
+                    while r < n:
+                        assert (r * c8 + g8 + 1) * 16 <= STAGE_BYTES
+                        row = t0 + r0 + r
+                        assert (row - t0) % R == lane and row > last[tid]
+                        last[tid] = row
+                        seen[(bi, row, g8)] = seen.get((bi, row, g8), 0) + 1
+                        r += R
+            fills += nst
+    return seen
 
 
 def phase1(b, cols, n_rows, stride, split, planes):
@@ -66,14 +120,18 @@ def test_mean_sums_every_row_once_inside_its_scratch(seed):
     rnd = random.Random(seed)
     for b, hk, sk, d in CASES + random_cases(rnd, 3000):
         cols = hk * d
-        split = make_split(b, cols, sk, 1024, SMS)
+        split = make_split(b, cols, sk, 1024, SMS, lanes_ok=True)
         colgroups, rpc, nchunks, n_items, grid = split
         assert 1 <= nchunks <= 1024 and 1 <= grid <= SMS
         if sk * b * cols > 4_000_000:  # the full transcription is slow: check the row split only
             rows = [t for ch in range(nchunks) for t in range(ch * rpc, min(ch * rpc + rpc, sk))]
             assert sorted(rows) == list(range(sk))
             continue
-        seen, top = phase1(b, cols, sk, 1, split, 1)
+        if lanes_of(cols, True):
+            seen = phase1_bulk(b, cols, sk, split)
+            top = (b * nchunks - 1) * cols + cols - 1  # thread t < c8 writes chunk row t*8..t*8+7
+        else:
+            seen, top = phase1(b, cols, sk, 1, split, 1)
         assert set(seen.values()) == {1}
         assert len(seen) == b * sk * (cols // 8), (b, hk, sk, d)
         assert top < b * nchunks * cols  # the partials the host allocates
@@ -104,7 +162,7 @@ def test_gate_reads_the_strided_sample_once(seed):
 def test_fold_covers_every_column_and_chunk_once():
     for b, hk, sk, d in CASES:
         cols = hk * d
-        _, _, nchunks, _, grid = make_split(b, cols, sk, 1024, SMS)
+        _, _, nchunks, _, grid = make_split(b, cols, sk, 1024, SMS, lanes_ok=True)
         nblk = (cols + 31) // 32
         outs = [(f // nblk, (f % nblk) * 32 + lane) for cta in range(grid)
                 for f in range(cta, b * nblk, grid) for lane in range(32)
@@ -140,7 +198,8 @@ def test_noalloc_split_fits_the_fixed_scratch():
         cols = hk * d
         if b * cols > NOALLOC_FLOATS:
             continue  # refused with ERR_SCRATCH
-        _, _, nchunks, _, grid = make_split(b, cols, sk, NOALLOC_FLOATS // (b * cols), SMS)
+        _, _, nchunks, _, grid = make_split(b, cols, sk, NOALLOC_FLOATS // (b * cols), SMS,
+                                            lanes_ok=True)
         assert b * nchunks * cols <= NOALLOC_FLOATS and grid <= 1024
 
 
@@ -150,7 +209,7 @@ def cols_group(pairs, n_sm):
     while G < THREADS and (pairs + G - 1) // G > n_sm:
         G <<= 1
     grid = (pairs + G - 1) // G
-    return G if grid <= n_sm and 2 * grid >= n_sm else 0
+    return G if grid <= n_sm and 2 * grid >= n_sm and G >= COLS_MIN_G else 0
 
 
 @pytest.mark.parametrize("seed", range(2))
@@ -158,10 +217,12 @@ def test_column_path_sums_every_row_once(seed):
     """k_mean_cols: CTA c owns (batch, 8-channel group) pairs [c*G, c*G + G); thread t takes pair
     slot t % G at rows t // G, + L, ... (L = 512 / G); the tree over lanes folds every lane into
     lane 0 exactly once. The K-mean workload (16 x 256 channels) takes it with G = 4 on 128 CTAs;
-    narrow K falls back to the row-chunk kernel."""
+    narrow K falls back to the row-chunk kernel, and so does K whose pairs would need G = 1
+    (16 bytes of a row per CTA: the 5 x 128-channel K of the long-context workload)."""
     assert cols_group(1 * 16 * 256 // 8, SMS) == 4
     assert (512 + 3) // 4 == 128
     assert cols_group(2 * 3 * 64 // 8, SMS) == 0  # 48 pairs: too few CTAs
+    assert cols_group(1 * 5 * 128 // 8, SMS) == 0  # 80 pairs: G = 1
     rnd = random.Random(20 + seed)
     cases = [(1, 16, 4096, 256), (2, 40, 300, 256), (1, 64, 77, 128), (4, 20, 33, 64), (1, 148, 9, 64)]
     cases += [(rnd.randint(1, 4), rnd.randint(1, 200), rnd.randint(1, 300),
