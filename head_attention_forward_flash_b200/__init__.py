@@ -11,7 +11,8 @@ importing this package fails loudly when the library is missing.
 Raw C entry points, with the header's names and argument order, are exposed through ``lib``
 (a ``ctypes.CDLL``): every name in ``EXPORTS`` (``lib.attn_fwd``, ``lib.attn_fwd_varlen``,
 ``lib.attn_fwd_window_sink``, ``lib.attn_fwd_fp8``, ``lib.fp8_quantize``, ``lib.k_smooth_gate``,
-``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``, ``lib.k_smooth_sub``,
+``lib.k_smooth_mean``, ``lib.k_smooth_mean_noalloc``, ``lib.k_smooth_mean_strided``,
+``lib.k_smooth_sub``,
 ``lib.k_smooth_mean_sub``, ``lib.attn_status_string``, ``lib.attn_debug_status``, ``lib.attn_debug_starve``).
 """
 from __future__ import annotations
@@ -29,7 +30,8 @@ STATUS = {
     11: "ERR_SCRATCH",
 }
 EXPORTS = ("attn_fwd", "attn_fwd_varlen", "attn_fwd_window_sink", "attn_fwd_fp8", "fp8_quantize",
-           "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_sub",
+           "k_smooth_gate", "k_smooth_mean", "k_smooth_mean_noalloc", "k_smooth_mean_strided",
+           "k_smooth_sub",
            "k_smooth_mean_sub", "attn_status_string", "attn_debug_status", "attn_debug_starve")
 
 
@@ -64,6 +66,8 @@ def _load() -> ctypes.CDLL:
     lib.k_smooth_mean.restype = ctypes.c_int
     lib.k_smooth_mean_noalloc.argtypes = [vp, vp, i64, i64, i64, i64, vp]
     lib.k_smooth_mean_noalloc.restype = ctypes.c_int
+    lib.k_smooth_mean_strided.argtypes = [vp, vp, i64, i64, i64, i64, i64, i64, i64, vp]
+    lib.k_smooth_mean_strided.restype = ctypes.c_int
     lib.k_smooth_gate.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, ctypes.c_float, vp]
     lib.k_smooth_gate.restype = ctypes.c_int
     lib.k_smooth_sub.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp]
@@ -331,6 +335,29 @@ def k_smooth_mean_noalloc(k, mean):
     _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
     _check("k_smooth_mean_noalloc", lib.k_smooth_mean_noalloc(k.data_ptr(), mean.data_ptr(), b, hk,
                                                               sk, d, _stream_ptr(k)))
+    return mean
+
+
+def k_smooth_mean_strided(k, mean=None):
+    """k_smooth_mean of any 4-dim bf16 view ``k`` [b, sk, hk, d] of device memory whose last
+    dimension is contiguous (a slice of heads or keys, an offset view): fp32 [b, hk, d]."""
+    import torch
+    if not isinstance(k, torch.Tensor):
+        raise TypeError("k must be a torch.Tensor")
+    if k.dim() != 4 or not k.is_cuda:
+        raise ValueError("k must be a 4-dim CUDA tensor [b, sk, hk, d]")
+    if k.dtype != torch.bfloat16:
+        raise TypeError("k must be bfloat16")
+    if k.shape[3] > 1 and k.stride(3) != 1:
+        raise ValueError("k's last dimension must be contiguous")
+    b, sk, hk, d = k.shape
+    if mean is None:
+        mean = torch.empty((b, hk, d), dtype=torch.float32, device=k.device)
+    else:
+        _want_out(mean, "mean", (b, hk, d), torch.float32, k.device)
+    _check("k_smooth_mean_strided",
+           lib.k_smooth_mean_strided(k.data_ptr(), mean.data_ptr(), b, hk, sk, d, k.stride(0),
+                                     k.stride(1), k.stride(2), _stream_ptr(k)))
     return mean
 
 

@@ -577,6 +577,84 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---- K mean of a strided view (k_smooth_mean_strided): 2-byte loads, any alignment ----
+// Element (bi, s, g, c) of the view is k[bi*sb + s*ss + g*sh + c]. Phase A: CTA (chunk, bi,
+// channel block) sums rows [chunk*rpc, +rpc) of kStrChannels channels, thread t owning channels
+// cb*kStrChannels + t + kStrThreads*q (q < kStrPerThread); a warp's loads of one row are 32
+// consecutive channels of one head (64 contiguous bytes), four rows in flight per channel, added
+// in row order. Phase B: each thread folds one (bi, channel) over the chunks in chunk order.
+constexpr int kStrThreads = 256;
+constexpr int kStrPerThread = 4;
+constexpr int kStrChannels = kStrThreads * kStrPerThread;
+
+__device__ __forceinline__ float bf16_at(const uint16_t* k, int64_t off)
+{
+    return __uint_as_float((uint32_t)__ldg(k + off) << 16);
+}
+
+__global__ void __launch_bounds__(kStrThreads)
+    k_mean_strided_partial(const uint16_t* __restrict__ k, float* __restrict__ partial,
+                           int64_t sk, int64_t d, int64_t cols, int64_t sb, int64_t ss,
+                           int64_t sh, int64_t rpc, int nchunks)
+{
+    const int chunk = blockIdx.x;
+    const int64_t bi = blockIdx.y;
+    const int64_t t0 = (int64_t)chunk * rpc;
+    const int64_t t1 = t0 + rpc < sk ? t0 + rpc : sk;
+    int64_t off[kStrPerThread];
+    bool on[kStrPerThread];
+#pragma unroll
+    for (int q = 0; q < kStrPerThread; ++q) {
+        const int64_t c = (int64_t)blockIdx.z * kStrChannels + threadIdx.x + q * kStrThreads;
+        on[q] = c < cols;
+        const int64_t g = on[q] ? c / d : 0;
+        off[q] = bi * sb + g * sh + (on[q] ? c - g * d : 0);
+    }
+    float acc[kStrPerThread] = {0.f, 0.f, 0.f, 0.f};
+    int64_t t = t0;
+    for (; t + 4 <= t1; t += 4) {
+        float x[kStrPerThread][4];
+#pragma unroll
+        for (int q = 0; q < kStrPerThread; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[q][e] = on[q] ? bf16_at(k, off[q] + (t + e) * ss) : 0.f;
+#pragma unroll
+        for (int q = 0; q < kStrPerThread; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[q] += x[q][e];
+    }
+    for (; t < t1; ++t)
+#pragma unroll
+        for (int q = 0; q < kStrPerThread; ++q)
+            if (on[q]) acc[q] += bf16_at(k, off[q] + t * ss);
+#pragma unroll
+    for (int q = 0; q < kStrPerThread; ++q) {
+        const int64_t c = (int64_t)blockIdx.z * kStrChannels + threadIdx.x + q * kStrThreads;
+        if (on[q]) partial[(bi * nchunks + chunk) * cols + c] = acc[q];
+    }
+}
+
+__global__ void __launch_bounds__(kStrThreads)
+    k_mean_strided_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t n,
+                        int64_t cols, int nchunks, float n_rows)
+{
+    const int64_t i = (int64_t)blockIdx.x * kStrThreads + threadIdx.x;  // bi * cols + c
+    if (i >= n) return;
+    const int64_t bi = i / cols, c = i - bi * cols;
+    const float* src = partial + bi * nchunks * cols + c;
+    float sum = 0.f;
+    int q = 0;
+    for (; q + 8 <= nchunks; q += 8) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = src[(int64_t)(q + e) * cols];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum += v[e];
+    }
+    for (; q < nchunks; ++q) sum += src[(int64_t)q * cols];
+    mean[i] = __fdiv_rn(sum, n_rows);
+}
+
 // The column-partitioned split: G = the least power of two whose ceil(pairs / G) CTAs fit on
 // the SMs; taken when that grid keeps at least half of the SMs busy and G >= kColsMinG (each
 // CTA then reads G * 16 contiguous bytes of every row); else 0: the one-pass row-chunk kernel.
@@ -939,4 +1017,62 @@ extern "C" int k_smooth_sub(const void* k, const float* mean, void* k_out, int64
     k_sub_kernel<<<(unsigned)blocks, kSubThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint4*>(k), mean, static_cast<uint4*>(k_out), b, sk, cols / 8);
     return cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+}
+
+extern "C" int k_smooth_mean_strided(const void* k, float* mean, int64_t b, int64_t hk, int64_t sk,
+                                     int64_t d, int64_t stride_b, int64_t stride_s,
+                                     int64_t stride_h, void* stream)
+{
+    if (b < 0 || hk < 0 || sk <= 0 || stride_b < 0 || stride_s < 0 || stride_h < 0)
+        return B200ATTN_ERR_SHAPE;
+    if (!(d == 64 || d == 128 || d == 256)) return B200ATTN_ERR_HEADDIM;
+    int64_t cols, n, last = 0, t;
+    if (!numel({hk, d}, &cols) || !numel({b, cols}, &n) || b >= 65536 || sk >= ((int64_t)1 << 40) ||
+        (cols + kStrChannels - 1) / kStrChannels >= 65536 || n >= ((int64_t)1 << 36))
+        return B200ATTN_ERR_RANGE;
+    // the largest element offset the view reaches must fit in int64
+    if (b > 0 && hk > 0) {
+        if (!mul_ok(b - 1, stride_b, &t) || (last += t) < 0 || !mul_ok(sk - 1, stride_s, &t) ||
+            (last += t) < 0 || !mul_ok(hk - 1, stride_h, &t) || (last += t) < 0 ||
+            (last += d) < 0 || last > INT64_MAX / 2)
+            return B200ATTN_ERR_RANGE;
+    }
+    if (b == 0 || hk == 0) return B200ATTN_OK;
+    if (!k || !mean) return B200ATTN_ERR_NULL;
+    if (!aligned(k, 2) || !aligned(mean, 4)) return B200ATTN_ERR_ALIGN;
+    // The contiguous layout at 16-byte alignment is k_smooth_mean itself (same kernels, same bits).
+    if (stride_h == d && stride_s == cols && stride_b == sk * cols && aligned(k, 16) &&
+        aligned(mean, 16))
+        return k_smooth_mean(k, mean, b, hk, sk, d, stream);
+    int rc = check_arch();
+    if (rc != B200ATTN_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t cblocks = (cols + kStrChannels - 1) / kStrChannels;
+    // about four CTAs per SM, at least 16 rows per chunk, at most 1024 chunks
+    int64_t nch = (4 * 148 + b * cblocks - 1) / (b * cblocks);
+    const int64_t by_rows = (sk + 15) / 16;
+    if (nch > by_rows) nch = by_rows;
+    if (nch > 1024) nch = 1024;
+    if (nch < 1) nch = 1;
+    const int64_t rpc = (sk + nch - 1) / nch;
+    const int nchunks = (int)((sk + rpc - 1) / rpc);
+    float* partial = nullptr;
+    cudaMemPool_t pool = scratch_pool();
+    const size_t nbytes = (size_t)(n * nchunks) * sizeof(float);
+    if (!pool || cudaMallocFromPoolAsync(reinterpret_cast<void**>(&partial), nbytes, pool, st) !=
+                     cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    k_mean_strided_partial<<<dim3((unsigned)nchunks, (unsigned)b, (unsigned)cblocks), kStrThreads,
+                             0, st>>>(static_cast<const uint16_t*>(k), partial, sk, d, cols,
+                                      stride_b, stride_s, stride_h, rpc, nchunks);
+    k_mean_strided_fold<<<(unsigned)((n + kStrThreads - 1) / kStrThreads), kStrThreads, 0, st>>>(
+        partial, mean, n, cols, nchunks, (float)sk);
+    rc = cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
+    if (cudaFreeAsync(partial, st) != cudaSuccess) {
+        cudaGetLastError();
+        return B200ATTN_ERR_CUDA;
+    }
+    return rc;
 }

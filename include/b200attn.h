@@ -200,6 +200,34 @@ B200ATTN_API int k_smooth_mean_noalloc(const void* k, float* mean, int64_t b, in
                                        int64_t sk, int64_t d, void* stream);
 
 /*
+ * k_smooth_mean_strided -- k_smooth_mean of a strided view of K: a slice of its heads or keys, a
+ * view into a larger buffer, or one whose address or strides are not 16-byte aligned.
+ *     mean[bi,g,c] = (1/sk) * sum_{s < sk} K(bi, s, g, c),
+ *     K(bi, s, g, c) = k[bi*stride_b + s*stride_s + g*stride_h + c]   (bf16 elements)
+ * "[HIP] Mha v4: run the K-smoothing gate as one HIP call" (PR Self-Review: PR-specific question;
+ * Changed op tests; commit message): the op's host check takes BSHD K whose last dimension is
+ * contiguous, misaligned views take a scalar-load path, and its test covers head-sliced and
+ * misaligned K views. Here: when the view is the contiguous layout (stride_h = d,
+ * stride_s = hk*d, stride_b = sk*hk*d) and k and mean are 16-byte aligned, this is
+ * k_smooth_mean (same kernels, same bits). Otherwise two launches on `stream`: fp32 partial sums
+ * per (batch, chunk of keys) with 2-byte loads, added in key order, then a fold of the chunks in
+ * chunk order, so repeated calls give bit-identical results.
+ *
+ *   k         device bf16, 2-byte aligned; element (bi, s, g, c) as above. The channel stride
+ *             is 1 (the page's contiguous last dimension).
+ *   stride_b, stride_s, stride_h  element strides >= 0 (any values; views may overlap).
+ *   mean      device fp32 [b, hk, d], 4-byte aligned. Fully written.
+ *   d         64, 128 or 256. sk > 0.
+ * Errors as for k_smooth_mean, plus B200ATTN_ERR_SHAPE for a negative stride and
+ * B200ATTN_ERR_RANGE when the largest element offset of the view overflows int64. Scratch
+ * (b * hk * d * chunks floats) from the library's stream-ordered pool, as k_smooth_mean.
+ * Concurrency as in the conventions above.
+ */
+B200ATTN_API int k_smooth_mean_strided(const void* k, float* mean, int64_t b, int64_t hk,
+                                       int64_t sk, int64_t d, int64_t stride_b, int64_t stride_s,
+                                       int64_t stride_h, void* stream);
+
+/*
  * k_smooth_gate -- the K-smoothing gate: sampled channel mean of K and a per-head decision.
  *
  * "[HIP] Mha v4: run the K-smoothing gate as one HIP call" (Summary, commit message) runs the

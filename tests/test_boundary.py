@@ -79,6 +79,22 @@ def test_k_mean_rejects(fn):
         assert f(A, A, A + 2, 1, 2, 8, 64, None) == 5
 
 
+def test_k_mean_strided_rejects():
+    f = b2.lib.k_smooth_mean_strided
+
+    def c(k=A, m=A, b=1, hk=2, sk=8, d=64, sb=2048, ss=256, sh=64):
+        return f(k, m, b, hk, sk, d, sb, ss, sh, None)
+
+    assert c(d=96) == 4 and c(d=192) == 4
+    assert c(sk=0) == 2 and c(b=-1) == 2 and c(hk=-1) == 2
+    assert c(sb=-1) == 2 and c(ss=-64) == 2 and c(sh=-1) == 2
+    assert c(k=None) == 1 and c(m=None) == 1
+    assert c(k=A + 1) == 5 and c(m=A + 2) == 5
+    assert c(b=0) == 0 and c(hk=0) == 0
+    assert c(ss=1 << 62) == 6 and c(b=2, sb=1 << 62) == 6
+    assert c(hk=1 << 20, d=256) == 6  # more channel blocks than a grid dimension holds
+
+
 def call_varlen(q=A, k=A, v=A, o=A, lse=A, cq=A, ck=A, b=2, hq=2, hk=1, tq=32, tk=32, max_sq=16,
                 dqk=64, dv=64, causal=0, scale=0.125):
     return b2.lib.attn_fwd_varlen(q, k, v, o, lse, cq, ck, b, hq, hk, tq, tk, max_sq, dqk, dv,
