@@ -581,8 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Element (bi, s, g, c) of the view is k[bi*sb + s*ss + g*sh + c]. Phase A: CTA (chunk, bi,
 // channel block) sums rows [chunk*rpc, +rpc) of kStrChannels channels, thread t owning channels
 // cb*kStrChannels + t + kStrThreads*q (q < kStrPerThread); a warp's loads of one row are 32
-// consecutive channels of one head (64 contiguous bytes), four rows in flight per channel, added
-// in row order. Phase B: each thread folds one (bi, channel) over the chunks in chunk order.
+// consecutive channels of one head (64 contiguous bytes), eight rows in flight per channel, added
+// in row order. Phase B: CTA (bi, 32 channels); warp w adds the chunks of its fixed contiguous
+// range in chunk order for its lane's channel, then the warp sums are added in warp order.
 constexpr int kStrThreads = 256;
 constexpr int kStrPerThread = 4;
 constexpr int kStrChannels = kStrThreads * kStrPerThread;
@@ -612,16 +613,16 @@ __global__ void __launch_bounds__(kStrThreads)
     }
     float acc[kStrPerThread] = {0.f, 0.f, 0.f, 0.f};
     int64_t t = t0;
-    for (; t + 4 <= t1; t += 4) {
-        float x[kStrPerThread][4];
+    for (; t + 8 <= t1; t += 8) {
+        float x[kStrPerThread][8];
 #pragma unroll
         for (int q = 0; q < kStrPerThread; ++q)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) x[q][e] = on[q] ? bf16_at(k, off[q] + (t + e) * ss) : 0.f;
+            for (int e = 0; e < 8; ++e) x[q][e] = on[q] ? bf16_at(k, off[q] + (t + e) * ss) : 0.f;
 #pragma unroll
         for (int q = 0; q < kStrPerThread; ++q)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[q] += x[q][e];
+            for (int e = 0; e < 8; ++e) acc[q] += x[q][e];
     }
     for (; t < t1; ++t)
 #pragma unroll
@@ -635,24 +636,37 @@ __global__ void __launch_bounds__(kStrThreads)
 }
 
 __global__ void __launch_bounds__(kStrThreads)
-    k_mean_strided_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t n,
-                        int64_t cols, int nchunks, float n_rows)
+    k_mean_strided_fold(const float* __restrict__ partial, float* __restrict__ mean, int64_t cols,
+                        int nchunks, float n_rows)
 {
-    const int64_t i = (int64_t)blockIdx.x * kStrThreads + threadIdx.x;  // bi * cols + c
-    if (i >= n) return;
-    const int64_t bi = i / cols, c = i - bi * cols;
-    const float* src = partial + bi * nchunks * cols + c;
+    constexpr int W = kStrThreads / 32;
+    __shared__ float red[W][32];
+    const int64_t nblk = (cols + 31) / 32;
+    const int64_t bi = blockIdx.x / nblk;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t c = (blockIdx.x - bi * nblk) * 32 + lane;
+    const int c_lo = (int)((int64_t)w * nchunks / W), c_hi = (int)((int64_t)(w + 1) * nchunks / W);
     float sum = 0.f;
-    int q = 0;
-    for (; q + 8 <= nchunks; q += 8) {
-        float v[8];
+    if (c < cols) {
+        const float* src = partial + bi * nchunks * cols + c;
+        int q = c_lo;
+        for (; q + 8 <= c_hi; q += 8) {
+            float v[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = src[(int64_t)(q + e) * cols];
+            for (int e = 0; e < 8; ++e) v[e] = src[(int64_t)(q + e) * cols];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sum += v[e];
+            for (int e = 0; e < 8; ++e) sum += v[e];
+        }
+        for (; q < c_hi; ++q) sum += src[(int64_t)q * cols];
     }
-    for (; q < nchunks; ++q) sum += src[(int64_t)q * cols];
-    mean[i] = __fdiv_rn(sum, n_rows);
+    red[w][lane] = sum;
+    __syncthreads();
+    if (w == 0 && c < cols) {
+        float tsum = 0.f;
+#pragma unroll
+        for (int q = 0; q < W; ++q) tsum += red[q][lane];
+        mean[bi * cols + c] = __fdiv_rn(tsum, n_rows);
+    }
 }
 
 // The column-partitioned split: G = the least power of two whose ceil(pairs / G) CTAs fit on
@@ -1048,8 +1062,8 @@ extern "C" int k_smooth_mean_strided(const void* k, float* mean, int64_t b, int6
     if (rc != B200ATTN_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t cblocks = (cols + kStrChannels - 1) / kStrChannels;
-    // about four CTAs per SM, at least 16 rows per chunk, at most 1024 chunks
-    int64_t nch = (4 * 148 + b * cblocks - 1) / (b * cblocks);
+    // about two CTAs per SM, at least 16 rows per chunk, at most 1024 chunks
+    int64_t nch = (2 * 148 + b * cblocks - 1) / (b * cblocks);
     const int64_t by_rows = (sk + 15) / 16;
     if (nch > by_rows) nch = by_rows;
     if (nch > 1024) nch = 1024;
@@ -1067,8 +1081,8 @@ extern "C" int k_smooth_mean_strided(const void* k, float* mean, int64_t b, int6
     k_mean_strided_partial<<<dim3((unsigned)nchunks, (unsigned)b, (unsigned)cblocks), kStrThreads,
                              0, st>>>(static_cast<const uint16_t*>(k), partial, sk, d, cols,
                                       stride_b, stride_s, stride_h, rpc, nchunks);
-    k_mean_strided_fold<<<(unsigned)((n + kStrThreads - 1) / kStrThreads), kStrThreads, 0, st>>>(
-        partial, mean, n, cols, nchunks, (float)sk);
+    k_mean_strided_fold<<<(unsigned)(b * ((cols + 31) / 32)), kStrThreads, 0, st>>>(
+        partial, mean, cols, nchunks, (float)sk);
     rc = cudaGetLastError() == cudaSuccess ? B200ATTN_OK : B200ATTN_ERR_CUDA;
     if (cudaFreeAsync(partial, st) != cudaSuccess) {
         cudaGetLastError();
