@@ -46,6 +46,25 @@ def test_gate_matches_oracle(d, sk, offset):
     assert np.all(np.abs(mean[on] - mu[on]) <= 1e-5 * scale[on])
 
 
+def test_gate_long_context_k():
+    """The FP8 recipe's K (b1 hk5 65536 keys d128): a stride-32 sample of 2048 rows."""
+    b, hk, sk, d, thr = 1, 5, 65536, 128, 0.25
+    k = k_inputs(b, hk, sk, d, seed=95, offset=0.5)
+    mean, gate, ratio = b2.k_smooth_gate(k.to(DEV), thr)
+    torch.cuda.synchronize()
+    mean, gate, ratio = mean.cpu().numpy(), gate.cpu().numpy(), ratio.cpu().numpy()
+    _, _, r_ref, g_ref = oracle.k_gate(workloads.bf16_bits(k), b, hk, sk, d, thr)
+    mu, _, _, _ = oracle.k_gate(workloads.bf16_bits(k), b, hk, sk, d, 0.0)
+    ks = k[:, ::32].double().numpy()
+    scale = np.maximum(np.abs(mu), np.abs(ks).mean(axis=1))
+    assert np.max(np.abs(ratio - r_ref)) <= 1e-5
+    clear = np.abs(r_ref - thr) > BAND
+    assert np.array_equal(gate[clear], g_ref[clear])
+    on = gate == 1
+    assert np.all(mean[~on] == 0.0)
+    assert np.all(np.abs(mean[on] - mu[on]) <= 1e-5 * scale[on])
+
+
 def test_gate_is_deterministic():
     k = k_inputs(1, 16, 4096, 256, seed=90, offset=1.0).to(DEV)
     a = b2.k_smooth_gate(k, 0.2)

@@ -225,10 +225,11 @@ def test_k_mean_small_shapes(b2, shape):
 
 
 @pytest.mark.parametrize("shape", [None, (2, 3, 100, 64), (1, 1, 1, 128), (3, 5, 17, 256),
-                                   (1, 8, 4099, 128), (2, 40, 300, 256)])
+                                   (1, 8, 4099, 128), (2, 40, 300, 256), (1, 5, 65536, 128)])
 def test_k_mean_sub_fused_equals_two_calls(b2, shape):
     """The one-launch mean and subtraction gives the bits of k_smooth_mean then k_smooth_sub, at
-    the K-mean workload's size (b1 hk16 4096 keys d256) and at small and ragged shapes."""
+    the K-mean workload's size (b1 hk16 4096 keys d256), at the long-context K (b1 hk5 65536
+    keys d128: the bulk-copy row-chunk launch at full size) and at small and ragged shapes."""
     if shape is None:
         c = config(4)
         _, k, _ = config_inputs(c)
