@@ -89,8 +89,10 @@ class Bar:
         return (self.completed & 1) != parity
 
 
-def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
-    """One random schedule over `units` (dicts with 'id' and 'n' = key blocks, 0 = skipped)."""
+def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False, late_turn=False):
+    """One random schedule over `units` (dicts with 'id' and 'n' = key blocks, 0 = skipped).
+    late_turn: the two tiles' softmax take their turn after waiting for (and loading) their own
+    S, as the E4M3 layout does, instead of before."""
     rnd = random.Random(seed)
     clock = [0]
     kfull = [Bar(1, f"kfull{i}", clock) for i in range(NK)]
@@ -322,11 +324,13 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                 for tt in tiles:
                     sb = sbuf_of(jg, tt)
                     item = (u["id"], j, tt)
-                    if NT == 2 and not pipe:  # the two tiles' softmax take turns, block by block
+                    def take_turn():  # the two tiles' softmax take turns, block by block
                         if tt == 1:
                             yield from wait(p_full[0], jg & 1)
                         elif jg > 0:
                             yield from wait(p_full[1], (jg - 1) & 1)
+                    if NT == 2 and not pipe and not late_turn:
+                        yield from take_turn()
                     parity = sphase_of(jg) ^ (1 if mutant == "s_full_wrong_parity" else 0)
                     yield from wait(s_full[sb], parity)
                     if q_tmem and j == u["n"] - 1 and nxt:
@@ -335,6 +339,8 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False):
                     check(b["lo"] == (item, "S") and b["hi"] == (item, "S"),
                           f"softmax of {item} reads {b}")
                     b["lo"], b["hi"] = (item, "read"), (item, "read")
+                    if NT == 2 and not pipe and late_turn:
+                        yield from take_turn()
                     if j > 0 and rnd.random() < 0.3:  # the running max grew: rescale O
                         if (NT == 1 or pipe) and mutant != "no_pv_done_wait":
                             yield from wait(pv_done[tt], (jg - 1) & 1)

@@ -19,6 +19,16 @@ def test_protocol_holds(layout):
         run(units, NT, NSM, q_tmem, NK, NV, seed, pipe=pipe)
 
 
+@pytest.mark.parametrize("layout", [x for x in LAYOUTS if x[0] == 2 and not x[5]],
+                         ids=lambda x: f"k{x[3]}_v{x[4]}_qt{int(x[2])}")
+def test_protocol_holds_with_late_turn(layout):
+    """The E4M3 layout's order: each tile waits for and loads its own S before its turn."""
+    NT, NSM, q_tmem, NK, NV, pipe = layout
+    for seed in range(SEEDS):
+        units = random_units(random.Random(seed * 11 + NT))
+        run(units, NT, NSM, q_tmem, NK, NV, seed, pipe=pipe, late_turn=True)
+
+
 @pytest.mark.parametrize("mutant", sorted(MUTANTS))
 def test_model_catches_planted_mistake(mutant):
     caught = 0
