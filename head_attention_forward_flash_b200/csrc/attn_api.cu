@@ -268,9 +268,10 @@ using T64P = AttnTraits<64, 64, 64, 2, 2, true, 8, 8, 0x92u, false, true>;  // 3
 using T128 = AttnTraits<128, 128, 128, 2, 2, false, 3, 2, 0x25u>;         // 64 + 96 + 64 KB
 using T192 = AttnTraits<192, 128, 128, 2, 2, false, 2, 1, 0x11u>;         // 96 + 96 + 32 KB
 using T256 = AttnTraits<256, 256, 64, 1, 1, true, 2, 2>;                  // 64 + 64 + 64 KB
-// E4M3 inputs, (128, 128): the d128 layout with half-size tiles, so four K and four V slots fit
-// next to the Q staging buffer and the O staging tile.
-using T128F8 = AttnTraits<128, 128, 128, 2, 2, false, 4, 4, 0x11u, true>;  // 32 + 64 + 64 (+64) KB
+// E4M3 inputs, (128, 128): the d128 layout with half-size tiles, so eight K and V slots fit next
+// to the Q staging buffer and the O staging tile: five K and three V (measured on B200, 5 x
+// 65536^2 causal: +0.5-0.7 % against four and four, three and five in between).
+using T128F8 = AttnTraits<128, 128, 128, 2, 2, false, 5, 3, 0x11u, true>;  // 32 + 80 + 48 (+64) KB
 
 // Kernel variants: dense, dense with window / sinks (compiled apart so that the plain path
 // carries none of the extra bound logic), and packed sequences.

@@ -416,7 +416,7 @@ def run(units, NT, NSM, q_tmem, NK, NV, seed, mutant=None, pipe=False, late_turn
 LAYOUTS = [(2, 2, True, 8, 8, True), (2, 2, False, 3, 2, False), (2, 2, False, 2, 1, False),
            (1, 1, True, 2, 2, False), (2, 2, False, 4, 4, False), (1, 1, True, 6, 6, False),
            (2, 2, True, 1, 1, True), (1, 1, False, 1, 1, False), (2, 2, False, 1, 1, False),
-           (2, 2, False, 2, 2, True), (2, 2, True, 5, 5, False)]
+           (2, 2, False, 2, 2, True), (2, 2, True, 5, 5, False), (2, 2, False, 5, 3, False)]
 
 
 def random_units(rnd):
