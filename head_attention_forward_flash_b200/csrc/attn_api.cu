@@ -204,12 +204,16 @@ int launch_attn(const void* q, const void* k, const void* v, void* out, float* l
     // evens them out best; where many heads' K/V far exceed L2, head-major, so that the CTAs
     // working at the same time share a few heads' K/V. Equal-cost units (no causal mask, or a
     // window band) take plain round robin. Packed sequences rank each sequence's units from its
-    // own last query tile (unit_info), so weight-major order hands out every sequence's k-th
-    // most expensive unit in round k.
+    // own last query tile (unit_info); with at most kMaxUnitClasses (sequence, rank) classes the
+    // kernel sorts the classes by cost and hands them out heaviest first (order 3: interleaved
+    // A/B on B200, 8 packed sequences of 1024-2048 keys, hq48:hk8 d64 causal), else weight-major
+    // order hands out every sequence's k-th most expensive unit in round k.
     {
         const double kv_bytes =
             (double)(b * sk) * (double)hk * (double)(T::DQK + T::DV) * (double)T::EB;
-        if (!CAUSAL || (EXT && sh.window >= 0))
+        if (VARLEN && b * p.n_qu <= kMaxUnitClasses)
+            p.order = 3;
+        else if (!CAUSAL || (EXT && sh.window >= 0))
             p.order = 0;
         else if (VARLEN)
             p.order = 2;

@@ -60,6 +60,7 @@
 namespace b200 {
 
 constexpr int kErrTimeout = 10;  // B200ATTN_ERR_TIMEOUT
+constexpr int kMaxUnitClasses = 256;  // order 3: (sequence, rank) classes at most
 
 struct AttnParams {
     __nv_bfloat16* o;
@@ -82,7 +83,9 @@ struct AttnParams {
     // Order in which CTAs take units. Round r gives CTA c the position
     // r * grid + (r odd and order != 0 ? grid - 1 - c : c); position -> unit is the identity
     // (head-major, heaviest unit of a head first) for order 0 / 1, and for order 2 the
-    // weight-major order (the k-th heaviest unit of every head, then the (k+1)-th ...).
+    // weight-major order (the k-th heaviest unit of every head, then the (k+1)-th ...). Order 3
+    // (packed sequences): the (sequence, rank) classes sorted by decreasing cost, all query
+    // heads of a class in turn.
     int order;
     FastDiv div_bh;  // by b * hq
     float scale_log2; // |scale| * log2(e); the sign of scale is applied by the MMA (negate A)
@@ -154,13 +157,16 @@ struct AttnTraits {
     // 64-column box: slab o_slab(tile, box, warp % 4), 32 rows x 128 bytes) when the tiles fit
     // next to the rings; otherwise each thread stores its own row.
     static constexpr uint32_t O_STAGE_BYTES = NT * BM * DV * 2;
-    static constexpr bool O_TMA = 1024 + O_OFF + O_STAGE_BYTES + NBAR * 8 + 16 <= 232448;
+    // after the barriers: the TMEM base and the abort flag (16 bytes), then order 3's class list
+    // and class costs (uint16 each)
+    static constexpr uint32_t TAIL_BYTES = 16 + 4 * kMaxUnitClasses;
+    static constexpr bool O_TMA = 1024 + O_OFF + O_STAGE_BYTES + NBAR * 8 + TAIL_BYTES <= 232448;
     static constexpr uint32_t o_slab(int tt, int bx, int w4)
     {
         return (uint32_t)(((tt * (DV / 64) + bx) * 4 + w4) * 4096);
     }
     static constexpr uint32_t BARS_OFF = O_OFF + (O_TMA ? O_STAGE_BYTES : 0);
-    static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + 16;
+    static constexpr uint32_t SMEM_BYTES = 1024 + BARS_OFF + NBAR * 8 + TAIL_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(NSM == NT, "one softmax warpgroup per query tile (and one MMA issuer each)");
     // Threads. One softmax warpgroup: warps 0-3 softmax, warp 4 MMA issuer, warp 5 TMA producer.
@@ -379,6 +385,7 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BARS_OFF);
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + T::NBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    uint16_t* vcls = reinterpret_cast<uint16_t*>(smem + T::BARS_OFF + T::NBAR * 8 + 16);
 
     auto bar = [&](int i) { return smem_addr(&bars[i]); };
     auto bar_kfull = [&](int s) { return bar(s); };
@@ -446,6 +453,33 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
     }
+    if constexpr (VARLEN) {
+        // Order 3: every CTA sorts the (sequence, rank) classes by decreasing cost -- the key
+        // blocks a class's units visit, plus 2 for a unit's fixed cost; ties in class order --
+        // so that CTAs take the most expensive units first, whatever the sequence lengths.
+        if (p.order == 3) {
+            uint16_t* vcost = vcls + kMaxUnitClasses;
+            const int nqu = (int)p.n_qu;
+            const int ncls = (int)p.b * nqu;  // at most kMaxUnitClasses (checked on the host)
+            for (int c = threadIdx.x; c < ncls; c += blockDim.x) {
+                const int bi = c / nqu, k = c - (c / nqu) * nqu;
+                const UnitInfo t =
+                    unit_info<T::BN, T::NT, CAUSAL, VARLEN, EXT>(p, (int64_t)bi * p.hq * nqu + k);
+                const int nb = t.n_blocks - t.j_begin;
+                vcost[c] = (uint16_t)(nb > 0 ? (nb + 2 < 65535 ? nb + 2 : 65535) : 0);
+            }
+            __syncthreads();
+            for (int c = threadIdx.x; c < ncls; c += blockDim.x) {
+                const uint32_t w = vcost[c];
+                int rank = 0;
+                for (int c2 = 0; c2 < ncls; ++c2) {
+                    const uint32_t w2 = vcost[c2];
+                    rank += (w2 > w || (w2 == w && c2 < c)) ? 1 : 0;
+                }
+                vcls[rank] = (uint16_t)c;
+            }
+        }
+    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -458,6 +492,13 @@ __global__ void __launch_bounds__(T::NUM_THREADS, 1)
         const int64_t c = blockIdx.x;
         const int64_t pos = r * g + ((p.order != 0 && (r & 1)) ? g - 1 - c : c);
         if (pos >= p.n_units) return -1;
+        if (VARLEN && p.order == 3) {
+            const uint32_t cr = fast_div((uint32_t)pos, p.div_hq);  // class rank
+            const uint32_t h = (uint32_t)pos - cr * p.div_hq.d;
+            const uint32_t c = vcls[cr];
+            const uint32_t bi = fast_div(c, p.div_nqu), k = c - bi * p.div_nqu.d;
+            return ((int64_t)bi * p.hq + h) * p.div_nqu.d + k;
+        }
         if (p.order == 2) {
             const uint32_t k = fast_div((uint32_t)pos, p.div_bh);  // rank within its head
             const uint32_t bh = (uint32_t)pos - k * p.div_bh.d;
