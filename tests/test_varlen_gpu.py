@@ -86,6 +86,23 @@ def test_equal_lengths_match_dense_bitwise(dqk, dv):
     assert torch.equal(l_v.view(hq, b, s).permute(1, 0, 2), l_d)
 
 
+@pytest.mark.parametrize("b,s,causal", [(80, 1000, True), (80, 1000, False)])
+def test_many_sequences_match_dense_bitwise(b, s, causal):
+    """More (sequence, rank) classes than the cost-sorted schedule takes (80 x 4 = 320 > 256): the
+    weight-major (causal) and round-robin (non-causal) orders; equal lengths match the dense
+    batch bit for bit."""
+    hq, hk, d = 2, 1, 64
+    q, k, v = workloads.make_inputs(b, hq, hk, s, s, d, d, seed=29)
+    o_d, l_d = b2.attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), causal=causal)
+    cu = torch.arange(0, (b + 1) * s, s, dtype=torch.int32)
+    o_v, l_v = b2.attn_fwd_varlen(q.reshape(b * s, hq, d).to(DEV), k.reshape(b * s, hk, d).to(DEV),
+                                  v.reshape(b * s, hk, d).to(DEV), cu.to(DEV), cu.to(DEV), s,
+                                  causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o_v.view(b, s, hq, d), o_d)
+    assert torch.equal(l_v.view(hq, b, s).permute(1, 0, 2), l_d)
+
+
 def test_no_keys_anywhere():
     hq, hk, d = 2, 2, 128
     q, k, v, cq, ck = workloads.make_varlen_inputs([5, 9], [0, 0], hq, hk, d, d, seed=4)
